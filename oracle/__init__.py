@@ -1,0 +1,211 @@
+"""CPU oracle for the W4A16 AWQ g128 quantized linear layer (numpy front end).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the CPU-baseline leg of the
+benchmark are the only callers.  The product library never imports this package, and
+this package never imports the product library; they share only the seeded input
+generators in ``workloads``.
+
+The arithmetic lives in ``oracle.c`` (plain C, one IEEE-754 float operation per source
+operation, double accumulation for the matrix product); this module marshals numpy
+arrays into it.  ``build()`` compiles it with gcc.  Every function says which passage of
+the pages it follows in the C source.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+OK, ERR_NULL, ERR_SHAPE, ERR_VALUE = 0, 1, 2, 4
+GROUP = 128
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"oracle {what} failed with status {code}")
+        self.code = code
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, no FMA contraction, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-shared",
+               "-fPIC", "-std=c11", "-Wall", "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        F = ctypes.c_float
+        sig = {
+            "oracle_f32_to_f16": ([F], ctypes.c_uint16),
+            "oracle_f16_to_f32": ([ctypes.c_uint16], F),
+            "oracle_f32_to_bf16": ([F], ctypes.c_uint16),
+            "oracle_bf16_to_f32": ([ctypes.c_uint16], F),
+            "oracle_pack8": ([P, P], ctypes.c_int),
+            "oracle_unpack8": ([ctypes.c_uint32, P], None),
+            "oracle_awq_scales": ([P, I64, F, P], ctypes.c_int),
+            "oracle_quantize_with_scales": ([P, P, I64, I64, P, P, P], ctypes.c_int),
+            "oracle_awq_quantize_g128": ([P, P, F, I64, I64, P, P, P, P], ctypes.c_int),
+            "oracle_dequant": ([P, P, P, I64, I64, P], ctypes.c_int),
+            "oracle_linear": ([P, I64, I64, P, P, P, I64, P, P, P, I64, P, P], ctypes.c_int),
+            "oracle_linear_at": ([P, I64, I64, P, P, P, I64, P, P, P, I64, P, P, I64, P, P],
+                                 ctypes.c_int),
+            "oracle_split_outliers": ([P, P, F, I64, I64, I64, P, P, P, P], ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(_lib, name)
+            fn.argtypes = args
+            fn.restype = res
+    return _lib
+
+
+def _p(a):
+    return None if a is None else ctypes.c_void_p(a.ctypes.data)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _check(code, what):
+    if code != OK:
+        raise OracleError(code, what)
+
+
+# ---- scalar conversions (IEEE-754 round-to-nearest-even, from the definition) ----------
+
+def f32_to_f16_bits(f: float) -> int:
+    return int(_L().oracle_f32_to_f16(ctypes.c_float(f)))
+
+
+def f16_bits_to_f32(h: int) -> float:
+    return float(_L().oracle_f16_to_f32(ctypes.c_uint16(h)))
+
+
+def f32_to_bf16_bits(f: float) -> int:
+    return int(_L().oracle_f32_to_bf16(ctypes.c_float(f)))
+
+
+def bf16_bits_to_f32(h: int) -> float:
+    return float(_L().oracle_bf16_to_f32(ctypes.c_uint16(h)))
+
+
+def pack8(codes) -> int:
+    q = _c(codes, np.uint8)
+    w = np.zeros(1, np.uint32)
+    _check(_L().oracle_pack8(_p(q), _p(w)), "pack8")
+    return int(w[0])
+
+
+def unpack8(word: int) -> np.ndarray:
+    q = np.zeros(8, np.uint8)
+    _L().oracle_unpack8(ctypes.c_uint32(word), _p(q))
+    return q
+
+
+# ---- the method -------------------------------------------------------------------------
+
+def awq_scales(act_absmean, alpha: float) -> np.ndarray:
+    a = _c(act_absmean, np.float32)
+    s = np.empty_like(a)
+    _check(_L().oracle_awq_scales(_p(a), a.size, ctypes.c_float(alpha), _p(s)), "awq_scales")
+    return s
+
+
+def quantize_with_scales(W, s):
+    W = _c(W, np.float32)
+    s = _c(s, np.float32)
+    N, K = W.shape
+    qw = np.zeros((N, K // 8), np.uint32)
+    sc = np.zeros((N, K // 128), np.uint16)
+    z = np.zeros((N, max(K // 1024, 1)), np.uint32)
+    _check(_L().oracle_quantize_with_scales(_p(W), _p(s), N, K, _p(qw), _p(sc), _p(z)),
+           "quantize_with_scales")
+    return qw, sc, z
+
+
+def awq_quantize_g128(W, act_absmean, alpha: float):
+    """-> (qweight u32 [N][K/8], scales fp16 bits u16 [N][K/128], zeros u32 [N][K/1024], s f32 [K])"""
+    W = _c(W, np.float32)
+    a = _c(act_absmean, np.float32)
+    N, K = W.shape
+    qw = np.zeros((N, K // 8), np.uint32)
+    sc = np.zeros((N, K // 128), np.uint16)
+    z = np.zeros((N, max(K // 1024, 1)), np.uint32)
+    s = np.zeros(K, np.float32)
+    _check(_L().oracle_awq_quantize_g128(_p(W), _p(a), ctypes.c_float(alpha), N, K, _p(qw), _p(sc),
+                                         _p(z), _p(s)), "awq_quantize_g128")
+    return qw, sc, z, s
+
+
+def dequant(qweight, scales, zeros, N: int, K: int) -> np.ndarray:
+    qw, sc, z = _c(qweight, np.uint32), _c(scales, np.uint16), _c(zeros, np.uint32)
+    out = np.zeros((N, K), np.float32)
+    _check(_L().oracle_dequant(_p(qw), _p(sc), _p(z), N, K, _p(out)), "dequant")
+    return out
+
+
+def _csr_args(csr):
+    if csr is None:
+        return None, None, None, 0
+    rp, ci, v = csr
+    return _c(rp, np.int32), _c(ci, np.int32), _c(v, np.uint16), int(len(ci))
+
+
+def linear(x_bf16_bits, qweight, scales, zeros, N: int, csr=None, with_abs: bool = False):
+    """y[m][n] = sum_k x deq + sum_csr x val, in double.  x is bf16 bits (uint16) [M][K].
+    csr = (row_ptr int32 [N+1], col_idx int32 [nnz], values fp16 bits [nnz]) or None."""
+    x = _c(x_bf16_bits, np.uint16)
+    M, K = x.shape
+    qw, sc, z = _c(qweight, np.uint32), _c(scales, np.uint16), _c(zeros, np.uint32)
+    rp, ci, v, nnz = _csr_args(csr)
+    y = np.zeros((M, N), np.float64)
+    ya = np.zeros((M, N), np.float64) if with_abs else None
+    _check(_L().oracle_linear(_p(x), M, K, _p(qw), _p(sc), _p(z), N, _p(rp), _p(ci), _p(v), nnz,
+                              _p(y), _p(ya)), "linear")
+    return (y, ya) if with_abs else y
+
+
+def linear_at(x_bf16_bits, qweight, scales, zeros, N: int, m_idx, n_idx, csr=None,
+              with_abs: bool = False):
+    """The outputs of ``linear`` at the positions (m_idx[p], n_idx[p]) only."""
+    x = _c(x_bf16_bits, np.uint16)
+    M, K = x.shape
+    qw, sc, z = _c(qweight, np.uint32), _c(scales, np.uint16), _c(zeros, np.uint32)
+    mi, ni = _c(m_idx, np.int64), _c(n_idx, np.int64)
+    rp, ci, v, nnz = _csr_args(csr)
+    y = np.zeros(mi.size, np.float64)
+    ya = np.zeros(mi.size, np.float64) if with_abs else None
+    _check(_L().oracle_linear_at(_p(x), M, K, _p(qw), _p(sc), _p(z), N, _p(rp), _p(ci), _p(v), nnz,
+                                 _p(mi), _p(ni), mi.size, _p(y), _p(ya)), "linear_at")
+    return (y, ya) if with_abs else y
+
+
+def split_outliers(W, act_absmean, alpha: float, nnz: int):
+    """-> (W_dense f32 [N][K], row_ptr i32 [N+1], col_idx i32 [nnz], values fp16 bits [nnz])"""
+    W = _c(W, np.float32)
+    a = _c(act_absmean, np.float32)
+    N, K = W.shape
+    Wd = np.zeros_like(W)
+    rp = np.zeros(N + 1, np.int32)
+    ci = np.zeros(max(nnz, 1), np.int32)
+    v = np.zeros(max(nnz, 1), np.uint16)
+    _check(_L().oracle_split_outliers(_p(W), _p(a), ctypes.c_float(alpha), N, K, nnz, _p(Wd), _p(rp),
+                                      _p(ci), _p(v)), "split_outliers")
+    return Wd, rp, ci[:nnz], v[:nnz]

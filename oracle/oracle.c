@@ -1,0 +1,428 @@
+/*
+ * oracle.c -- plain CPU oracle for the W4A16 AWQ g128 quantized linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call this
+ * file: only the tests, the smoke check and the benchmark's CPU-baseline leg use it.
+ * It shares no code, header, table or constant with the CUDA library; the packed
+ * format it writes is the interface both sides agree on, restated here on its own.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no FMA contraction, so
+ * every float operation below is one IEEE-754 operation rounded to nearest-even).
+ *
+ * What it computes, and where the method comes from:
+ *   - per-input-channel activation-aware scale s_k = max(float(pow(a_k, alpha)), 1e-4)
+ *     [AWQ (MLSys 2024) translation, section 3.2 "protect salient weights by
+ *     activation-aware scaling"; the closed form mean|x|^alpha is the one the task
+ *     statement fixes, the pages truncate before it];
+ *   - group-wise asymmetric uint4 round-to-nearest on W*s, groups of 128 along K
+ *     [DeepCompressor README, perplexity table row "W4A16 g128"; AWQ translation,
+ *     section 2 "round-to-nearest (RTN)" and group-wise INT4];
+ *   - 4-bit weight packing, 8 codes per 32-bit word [AWQ translation, section 1:
+ *     TinyChat's 4-bit weight packing];
+ *   - the dense-and-sparse product  W x = W_dense x + W_sparse x  with an fp16 CSR
+ *     W_sparse [SqueezeLLM article, sections 2.2 and 2.3; the page lost the "=" and
+ *     "+" signs, read here as written above];
+ *   - the outlier split: the largest |w| * act_absmean entries go to W_sparse
+ *     [SqueezeLLM article, section 2.2 (sensitive weights kept in fp16) and
+ *     section 5.3 (sparsity ratio 0.0045)].
+ *
+ * Every function here has at least one independent pin in tests/ (brute force, closed
+ * forms, invariants, library routines); see the test files for which.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_NULL 1
+#define ORACLE_ERR_SHAPE 2
+#define ORACLE_ERR_VALUE 4
+
+#define GROUP 128
+
+/* ------------------------------------------------------------------------------------
+ * IEEE-754 binary16 / bfloat16 conversions written from the format definitions:
+ * round the exact value to the nearest point of the target grid, ties to the even
+ * significand, overflow to infinity.  All arithmetic is in double, where every step
+ * below is exact (scaling by powers of two, rint of a value with <= 25 significant
+ * bits).
+ * ---------------------------------------------------------------------------------- */
+
+/* binary16: 11 significant bits, normal exponents -14..15, subnormal step 2^-24. */
+uint16_t oracle_f32_to_f16(float f) {
+    uint16_t sign = signbit(f) ? 0x8000u : 0u;
+    if (isnan(f)) return (uint16_t)(sign | 0x7E00u);
+    double a = fabs((double)f);
+    /* The largest finite value is 65504 (significand 2047, odd); a tie at 65520 rounds
+     * to the even neighbour 65536, which overflows. */
+    if (isinf(f) || a >= 65520.0) return (uint16_t)(sign | 0x7C00u);
+    if (a < ldexp(1.0, -14)) {
+        double r = rint(a / ldexp(1.0, -24)); /* 0..1024; 1024 is the smallest normal */
+        return (uint16_t)(sign | (uint16_t)r);
+    }
+    int e;
+    frexp(a, &e);                   /* a = m * 2^e, m in [0.5, 1): leading bit 2^(e-1) */
+    double quantum = ldexp(1.0, e - 1 - 10);
+    double r = rint(a / quantum);   /* 1024..2048 */
+    int biased = e - 1 + 15;
+    if (r == 2048.0) { r = 1024.0; biased += 1; }
+    if (biased >= 31) return (uint16_t)(sign | 0x7C00u);
+    return (uint16_t)(sign | (uint16_t)(biased << 10) | (uint16_t)((int)r - 1024));
+}
+
+float oracle_f16_to_f32(uint16_t h) {
+    int s = (h >> 15) & 1, E = (h >> 10) & 31, m = h & 1023;
+    double v;
+    if (E == 31) v = m ? NAN : INFINITY;
+    else if (E == 0) v = ldexp((double)m, -24);
+    else v = ldexp((double)(1024 + m), E - 15 - 10);
+    return (float)(s ? -v : v);
+}
+
+/* bfloat16: 8 significant bits, the exponent range of binary32 (normal from 2^-126,
+ * subnormal step 2^-133). */
+uint16_t oracle_f32_to_bf16(float f) {
+    uint16_t sign = signbit(f) ? 0x8000u : 0u;
+    if (isnan(f)) return (uint16_t)(sign | 0x7FC0u);
+    double a = fabs((double)f);
+    /* largest finite: (2 - 2^-7) * 2^127, significand 255 (odd): the tie above it rounds
+     * up to 2^128 and overflows */
+    if (isinf(f) || a >= ldexp(2.0 - ldexp(1.0, -8), 127)) return (uint16_t)(sign | 0x7F80u);
+    if (a < ldexp(1.0, -126)) {
+        double r = rint(a / ldexp(1.0, -133)); /* 0..128; 128 is the smallest normal */
+        return (uint16_t)(sign | (uint16_t)r);
+    }
+    int e;
+    frexp(a, &e);
+    double quantum = ldexp(1.0, e - 1 - 7);
+    double r = rint(a / quantum);   /* 128..256 */
+    int biased = e - 1 + 127;
+    if (r == 256.0) { r = 128.0; biased += 1; }
+    if (biased >= 255) return (uint16_t)(sign | 0x7F80u);
+    return (uint16_t)(sign | (uint16_t)(biased << 7) | (uint16_t)((int)r - 128));
+}
+
+float oracle_bf16_to_f32(uint16_t h) {
+    int s = (h >> 15) & 1, E = (h >> 7) & 255, m = h & 127;
+    double v;
+    if (E == 255) v = m ? NAN : INFINITY;
+    else if (E == 0) v = ldexp((double)m, -133);
+    else v = ldexp((double)(128 + m), E - 127 - 7);
+    return (float)(s ? -v : v);
+}
+
+/* ------------------------------------------------------------------------------------
+ * Packed format (the interface shared with the CUDA library, restated here):
+ *   qweight[n][k/8]  uint32; nibble j (bits 4j..4j+3) holds element k = 8*(k/8) + ORDER[j]
+ *                    with ORDER = {0,2,4,6,1,3,5,7};
+ *   scales[n][g]     fp16 bits, g = k/128;
+ *   zeros[n][g/8]    uint32; nibble j holds the zero point of group 8*(g/8) + j.
+ * ---------------------------------------------------------------------------------- */
+static const int ORACLE_ORDER[8] = {0, 2, 4, 6, 1, 3, 5, 7};
+
+static int nibble_of_element(int e) { /* inverse of ORACLE_ORDER */
+    for (int j = 0; j < 8; ++j)
+        if (ORACLE_ORDER[j] == e) return j;
+    return -1;
+}
+
+int oracle_pack8(const uint8_t* q /* 8 codes, element order */, uint32_t* word) {
+    uint32_t w = 0;
+    for (int j = 0; j < 8; ++j) {
+        if (q[ORACLE_ORDER[j]] > 15) return ORACLE_ERR_VALUE;
+        w |= (uint32_t)q[ORACLE_ORDER[j]] << (4 * j);
+    }
+    *word = w;
+    return ORACLE_OK;
+}
+
+void oracle_unpack8(uint32_t word, uint8_t* q /* 8 codes, element order */) {
+    for (int e = 0; e < 8; ++e) q[e] = (uint8_t)((word >> (4 * nibble_of_element(e))) & 15u);
+}
+
+/* ------------------------------------------------------------------------------------
+ * Activation-aware scale [AWQ translation, section 3.2]:
+ *   s_k = max( float(pow(double(a_k), double(alpha))), 1e-4 ).
+ * a_k must be finite and >= 0, alpha finite; a non-finite s is a value error.
+ * ---------------------------------------------------------------------------------- */
+int oracle_awq_scales(const float* act_absmean, int64_t K, float alpha, float* s) {
+    if (!act_absmean || !s) return ORACLE_ERR_NULL;
+    if (K <= 0) return ORACLE_ERR_SHAPE;
+    if (!isfinite(alpha)) return ORACLE_ERR_VALUE;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = act_absmean[k];
+        if (!isfinite(a) || a < 0.0f) return ORACLE_ERR_VALUE;
+        float p = (float)pow((double)a, (double)alpha);
+        if (!isfinite(p)) return ORACLE_ERR_VALUE;
+        s[k] = p > 1e-4f ? p : 1e-4f;
+    }
+    return ORACLE_OK;
+}
+
+/* One group of 128 scaled weights -> fp16 scale bits, zero point, 128 codes.
+ *   scale32 = max((max - min) / 15, 1e-5)          (plain asymmetric min/max range)
+ *   sf      = float(fp16_rne(scale32))             (the stored scale is the one used)
+ *   z       = clamp(rint(-min / sf), 0, 15)
+ *   q_i     = clamp(rint(w_i / sf) + z, 0, 15)     (round first, then add the zero)
+ * rint is round-half-to-even; every operation is one IEEE float operation. */
+static int quantize_group(const float* wp, uint16_t* s16_out, uint8_t* z_out, uint8_t* q_out) {
+    float mx = wp[0], mn = wp[0];
+    for (int i = 0; i < GROUP; ++i) {
+        if (!isfinite(wp[i])) return ORACLE_ERR_VALUE;
+        if (wp[i] > mx) mx = wp[i];
+        if (wp[i] < mn) mn = wp[i];
+    }
+    float scale32 = (mx - mn) / 15.0f;
+    if (scale32 < 1e-5f) scale32 = 1e-5f;
+    if (isinf(scale32)) return ORACLE_ERR_VALUE; /* max - min overflowed */
+    uint16_t s16 = oracle_f32_to_f16(scale32);
+    if ((s16 & 0x7FFFu) == 0x7C00u) return ORACLE_ERR_VALUE; /* fp16 overflow */
+    float sf = oracle_f16_to_f32(s16);
+    float zf = rintf(-mn / sf);
+    if (zf < 0.0f) zf = 0.0f;
+    if (zf > 15.0f) zf = 15.0f;
+    for (int i = 0; i < GROUP; ++i) {
+        float qf = rintf(wp[i] / sf) + zf;
+        if (qf < 0.0f) qf = 0.0f;
+        if (qf > 15.0f) qf = 15.0f;
+        q_out[i] = (uint8_t)qf;
+    }
+    *s16_out = s16;
+    *z_out = (uint8_t)zf;
+    return ORACLE_OK;
+}
+
+static int check_qshape(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0 || K % 1024 != 0) return ORACLE_ERR_SHAPE;
+    return ORACLE_OK;
+}
+
+/* Quantize W (fp32 [N][K]) with a given per-channel scale s ([K]):
+ * w' = float(w * s_k), then quantize_group on each run of 128 along K, then pack. */
+int oracle_quantize_with_scales(const float* W, const float* s, int64_t N, int64_t K,
+                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros) {
+    if (!W || !s || !qweight || !scales || !zeros) return ORACLE_ERR_NULL;
+    int st = check_qshape(N, K);
+    if (st) return st;
+    const int64_t G = K / GROUP;
+    int err = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < N; ++n) {
+        float wp[GROUP];
+        uint8_t q[GROUP];
+        for (int64_t g = 0; g < G; ++g) {
+            for (int i = 0; i < GROUP; ++i) wp[i] = W[n * K + g * GROUP + i] * s[g * GROUP + i];
+            uint16_t s16;
+            uint8_t z;
+            int e = quantize_group(wp, &s16, &z, q);
+            if (e) {
+#pragma omp atomic write
+                err = e;
+                continue;
+            }
+            scales[n * G + g] = s16;
+            if (g % 8 == 0) zeros[n * (G / 8) + g / 8] = 0;
+            zeros[n * (G / 8) + g / 8] |= (uint32_t)z << (4 * (g % 8));
+            for (int w = 0; w < GROUP / 8; ++w) {
+                uint32_t word;
+                oracle_pack8(&q[8 * w], &word);
+                qweight[n * (K / 8) + g * (GROUP / 8) + w] = word;
+            }
+        }
+    }
+    return err;
+}
+
+/* awq_quantize_g128: the scale from act_absmean and alpha, then quantize W*s. */
+int oracle_awq_quantize_g128(const float* W, const float* act_absmean, float alpha, int64_t N,
+                             int64_t K, uint32_t* qweight, uint16_t* scales, uint32_t* zeros,
+                             float* s_out) {
+    if (!W || !act_absmean || !qweight || !scales || !zeros) return ORACLE_ERR_NULL;
+    int st = check_qshape(N, K);
+    if (st) return st;
+    float* s = (float*)malloc(sizeof(float) * (size_t)K);
+    if (!s) return ORACLE_ERR_VALUE;
+    st = oracle_awq_scales(act_absmean, K, alpha, s);
+    if (!st) st = oracle_quantize_with_scales(W, s, N, K, qweight, scales, zeros);
+    if (!st && s_out) memcpy(s_out, s, sizeof(float) * (size_t)K);
+    free(s);
+    return st;
+}
+
+/* deq[n][k] = (q - z) * sf, exact in fp32 (a 5-bit integer times an 11-bit scale). */
+int oracle_dequant(const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
+                   int64_t N, int64_t K, float* deq) {
+    if (!qweight || !scales || !zeros || !deq) return ORACLE_ERR_NULL;
+    int st = check_qshape(N, K);
+    if (st) return st;
+    const int64_t G = K / GROUP;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t g = k / GROUP;
+            uint8_t codes[8];
+            oracle_unpack8(qweight[n * (K / 8) + k / 8], codes);
+            int q = codes[k % 8];
+            int z = (int)((zeros[n * (G / 8) + g / 8] >> (4 * (g % 8))) & 15u);
+            float sf = oracle_f16_to_f32(scales[n * G + g]);
+            deq[n * K + k] = (float)(q - z) * sf;
+        }
+    }
+    return ORACLE_OK;
+}
+
+static int check_csr(const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                     int64_t nnz, int64_t N, int64_t K) {
+    if (nnz < 0) return ORACLE_ERR_SHAPE;
+    if (nnz == 0 && !row_ptr) return ORACLE_OK;
+    if (!row_ptr || (nnz > 0 && (!col_idx || !values))) return ORACLE_ERR_NULL;
+    if (row_ptr[0] != 0 || row_ptr[N] != nnz) return ORACLE_ERR_SHAPE;
+    for (int64_t n = 0; n < N; ++n) {
+        if (row_ptr[n + 1] < row_ptr[n]) return ORACLE_ERR_SHAPE;
+        for (int64_t j = row_ptr[n]; j < row_ptr[n + 1]; ++j) {
+            if (col_idx[j] < 0 || col_idx[j] >= K) return ORACLE_ERR_SHAPE;
+            if (j > row_ptr[n] && col_idx[j] <= col_idx[j - 1]) return ORACLE_ERR_SHAPE;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* One output y[m][n] = sum_k x[m][k] deq[n][k] + sum_{j in row n} x[m][col_j] val_j, summed
+ * in double (each product of a bf16 and a dequantized weight or fp16 value is exact in
+ * double), plus the sum of the absolute products, which bounds any rounding error. */
+static void one_output(const uint16_t* x, int64_t K, const uint32_t* qweight,
+                       const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
+                       const int32_t* col_idx, const uint16_t* values, int64_t m, int64_t n,
+                       double* y, double* yabs) {
+    const int64_t G = K / GROUP;
+    double acc = 0.0, aacc = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        int64_t g = k / GROUP;
+        uint8_t codes[8];
+        oracle_unpack8(qweight[n * (K / 8) + k / 8], codes);
+        int q = codes[k % 8];
+        int z = (int)((zeros[n * (G / 8) + g / 8] >> (4 * (g % 8))) & 15u);
+        double w = (double)((float)(q - z) * oracle_f16_to_f32(scales[n * G + g]));
+        double p = (double)oracle_bf16_to_f32(x[m * K + k]) * w;
+        acc += p;
+        aacc += fabs(p);
+    }
+    if (row_ptr) {
+        for (int64_t j = row_ptr[n]; j < row_ptr[n + 1]; ++j) {
+            double p = (double)oracle_bf16_to_f32(x[m * K + col_idx[j]]) *
+                       (double)oracle_f16_to_f32(values[j]);
+            acc += p;
+            aacc += fabs(p);
+        }
+    }
+    *y = acc;
+    if (yabs) *yabs = aacc;
+}
+
+/* y = x deq(Q)^T + x W_sparse^T for all (m, n): x bf16 [M][K]; y, yabs double [M][N].
+ * The CSR (row_ptr [N+1], col_idx/values [nnz], ascending columns per row) may be absent
+ * (row_ptr == NULL and nnz == 0). */
+int oracle_linear(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweight,
+                  const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                  const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                  int64_t nnz, double* y, double* yabs) {
+    if (!x || !qweight || !scales || !zeros || !y) return ORACLE_ERR_NULL;
+    if (M <= 0) return ORACLE_ERR_SHAPE;
+    int st = check_qshape(N, K);
+    if (st) return st;
+    st = check_csr(row_ptr, col_idx, values, nnz, N, K);
+    if (st) return st;
+#pragma omp parallel for collapse(2) schedule(dynamic, 16)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n)
+            one_output(x, K, qweight, scales, zeros, row_ptr, col_idx, values, m, n,
+                       &y[m * N + n], yabs ? &yabs[m * N + n] : NULL);
+    return ORACLE_OK;
+}
+
+/* The same outputs at P sampled positions (m_idx[p], n_idx[p]) only. */
+int oracle_linear_at(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweight,
+                     const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                     const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                     int64_t nnz, const int64_t* m_idx, const int64_t* n_idx, int64_t P,
+                     double* y, double* yabs) {
+    if (!x || !qweight || !scales || !zeros || !y || !m_idx || !n_idx) return ORACLE_ERR_NULL;
+    if (M <= 0 || P < 0) return ORACLE_ERR_SHAPE;
+    int st = check_qshape(N, K);
+    if (st) return st;
+    st = check_csr(row_ptr, col_idx, values, nnz, N, K);
+    if (st) return st;
+    for (int64_t p = 0; p < P; ++p)
+        if (m_idx[p] < 0 || m_idx[p] >= M || n_idx[p] < 0 || n_idx[p] >= N) return ORACLE_ERR_SHAPE;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t p = 0; p < P; ++p)
+        one_output(x, K, qweight, scales, zeros, row_ptr, col_idx, values, m_idx[p], n_idx[p],
+                   &y[p], yabs ? &yabs[p] : NULL);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------------------
+ * Outlier split [SqueezeLLM article, 2.2; the selection rule |w| * act_absmean replaces
+ * the Hessian sensitivity, which needs a trained model and data]:
+ *   score(n,k) = float(|w[n][k]| * a_k) on the original W;
+ *   the nnz largest scores are selected; equal scores are taken in increasing linear
+ *   index n*K + k;
+ *   W_dense = W with the selected entries set to 0;
+ *   CSR of the selected entries, rows in order, columns ascending,
+ *   value = fp16_rne(float(w * s_k)) (the same scaled space as the quantized weights).
+ * ---------------------------------------------------------------------------------- */
+static int cmp_desc_u64(const void* a, const void* b) {
+    uint64_t x = *(const uint64_t*)a, y = *(const uint64_t*)b;
+    return x < y ? 1 : (x > y ? -1 : 0);
+}
+
+int oracle_split_outliers(const float* W, const float* act_absmean, float alpha, int64_t N,
+                          int64_t K, int64_t nnz, float* W_dense, int32_t* row_ptr,
+                          int32_t* col_idx, uint16_t* values) {
+    if (!W || !act_absmean || !W_dense || !row_ptr) return ORACLE_ERR_NULL;
+    if (N <= 0 || K <= 0 || nnz < 0 || nnz > N * K) return ORACLE_ERR_SHAPE;
+    if (nnz > 0 && (!col_idx || !values)) return ORACLE_ERR_NULL;
+    if ((uint64_t)N * (uint64_t)K > 0xFFFFFFFFull || nnz > 0x7FFFFFFF) return ORACLE_ERR_SHAPE;
+    const int64_t NK = N * K;
+    float* s = (float*)malloc(sizeof(float) * (size_t)K);
+    uint64_t* key = (uint64_t*)malloc(sizeof(uint64_t) * (size_t)NK);
+    uint8_t* chosen = (uint8_t*)calloc((size_t)NK, 1);
+    int st = (s && key && chosen) ? ORACLE_OK : ORACLE_ERR_VALUE;
+    if (!st) st = oracle_awq_scales(act_absmean, K, alpha, s);
+    for (int64_t i = 0; !st && i < NK; ++i)
+        if (!isfinite(W[i])) st = ORACLE_ERR_VALUE;
+    if (!st) {
+        for (int64_t i = 0; i < NK; ++i) {
+            float score = fabsf(W[i]) * act_absmean[i % K];
+            uint32_t bits;
+            memcpy(&bits, &score, 4); /* non-negative floats order like their bit patterns */
+            /* larger score first; among equal scores the lower index first */
+            key[i] = ((uint64_t)bits << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)i);
+        }
+        qsort(key, (size_t)NK, sizeof(uint64_t), cmp_desc_u64);
+        for (int64_t t = 0; t < nnz; ++t) chosen[0xFFFFFFFFu - (uint32_t)(key[t] & 0xFFFFFFFFu)] = 1;
+        int64_t j = 0;
+        row_ptr[0] = 0;
+        for (int64_t n = 0; n < N && !st; ++n) {
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t i = n * K + k;
+                if (chosen[i]) {
+                    uint16_t h = oracle_f32_to_f16(W[i] * s[k]);
+                    if ((h & 0x7FFFu) == 0x7C00u) { st = ORACLE_ERR_VALUE; break; }
+                    col_idx[j] = (int32_t)k;
+                    values[j] = h;
+                    ++j;
+                    W_dense[i] = 0.0f;
+                } else {
+                    W_dense[i] = W[i];
+                }
+            }
+            row_ptr[n + 1] = (int32_t)j;
+        }
+    }
+    free(s);
+    free(key);
+    free(chosen);
+    return st;
+}
