@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 W4A16 quantized linear layer.
+
+Headline (one JSON line on rank 0): decode GEMV throughput in GB/s of algorithmic traffic on
+the Llama-3-8B linear shapes (K x N = 4096x6144, 4096x4096, 4096x28672, 14336x4096) at
+M = 1, 4, 8, 16 tokens, W4 g128 weights packed by the library's own quantize kernel.  One
+step is the 16 GEMV calls of that sweep, replayed as a CUDA graph.  Each (shape, M) call
+uses its own copy of the packed weights, so a step touches 453 MB, well above the 126 MB
+L2.  Extra keys report the prefill GEMM (TFLOP/s) on the same shapes at M = 512, 2048 and
+8192, and the quantize kernel (GB/s).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs one process per GPU (torchrun); the path does not shard, so every rank runs an
+independent replica of the workload ("scaling": "weak").  Time is the max over ranks.
+--impl reference times the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "W4A16 GEMV achieved GB/s (% HBM peak); GEMM TFLOPS (% bf16 TC peak)"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATA = "synthetic: seeded N(0, 0.02^2) weights, lognormal-channel activations (no checkpoints)"
+GEMV_SHAPES = workloads.LLAMA3_8B
+GEMV_MS = workloads.CONFIGS[1]["Ms"]
+GEMM_MS = workloads.CONFIGS[2]["Ms"]
+WORKLOAD = ("decode GEMV sweep, Llama-3-8B linear shapes (K x N = 4096x6144, 4096x4096, 4096x28672, "
+            "14336x4096) x M in {1, 4, 8, 16}, W4 g128 (alpha 0.5)")
+
+
+def gemv_bytes(N: int, K: int, M: int) -> int:
+    """Algorithmic bytes of one GEMV call: packed weights + bf16 x + bf16 y."""
+    return workloads.packed_bytes(N, K) + 2 * M * K + 2 * M * N
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK}, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------ distributed plumbing --
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(value: float, world: int) -> float:
+    """Max over ranks (the timed region's length of the slowest replica)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(ms_local: float, bytes_local: float, world: int):
+    """Whole-job throughput: the units all ranks processed over the max time of any rank."""
+    ms = reduce_max(ms_local, world)
+    return ms, bytes_local * world / (ms * 1e-3) / 1e9
+
+
+# ------------------------------------------------------------------ clocks -----------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.sel = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.sel = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.sel:
+            cmd += ["-i", self.sel]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing ------
+
+def oracle_sample(budget_s: float):
+    """Time the CPU oracle on sampled outputs of the GEMV sweep for about budget_s seconds.
+    Returns (GB/s-equivalent, seconds, outputs, description).  Each sampled output (m, n) of a
+    call accounts for bytes_call / (M * N) algorithmic bytes."""
+    import oracle
+    oracle.build()
+    rng = np.random.default_rng(12345)
+    calls = []
+    for si, (name, K, N) in enumerate(GEMV_SHAPES):
+        L = workloads.make_layer(workloads.seed_of(1, si), K=K, N=N)
+        qw, sc, z, _ = oracle.awq_quantize_g128(L.W, L.act_absmean, workloads.ALPHA)
+        for M in GEMV_MS:
+            x = workloads.make_activations(workloads.seed_of(1, si), M, L.mult)
+            calls.append((K, N, M, qw, sc, z, x))
+
+    def run(P):
+        t, b = 0.0, 0.0
+        for K, N, M, qw, sc, z, x in calls:
+            m = rng.integers(0, M, P)
+            n = rng.integers(0, N, P)
+            t0 = time.perf_counter()
+            oracle.linear_at(x, qw, sc, z, N, m, n)
+            t += time.perf_counter() - t0
+            b += gemv_bytes(N, K, M) / (M * N) * P
+        return t, b
+
+    t_cal, _ = run(64)
+    P = int(max(64, min(1 << 20, 64 * budget_s / max(t_cal, 1e-6))))
+    t, b = run(P)
+    desc = (f"oracle.linear_at (C, fp64 accumulation, OpenMP over outputs): {P} sampled outputs of each of "
+            f"the 16 calls of the sweep ({16 * P} outputs); each output counts call bytes / (M*N)")
+    return b / t / 1e9, t, 16 * P, desc
+
+
+def omp_threads() -> int:
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v and v.isdigit() else (os.cpu_count() or 1)
+
+
+# ------------------------------------------------------------------ reference arm ----------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    # one layer of the sweep per step, rotating; a fixed number of sampled outputs per step,
+    # sized so that warmup + steps take about two minutes
+    layers = []
+    for si, (name, K, N) in enumerate(GEMV_SHAPES):
+        L = workloads.make_layer(workloads.seed_of(1, si), K=K, N=N)
+        qw, sc, z, _ = oracle.awq_quantize_g128(L.W, L.act_absmean, workloads.ALPHA)
+        xs = {M: workloads.make_activations(workloads.seed_of(1, si), M, L.mult) for M in GEMV_MS}
+        layers.append((K, N, qw, sc, z, xs))
+    rng = np.random.default_rng(7)
+
+    def one_step(i, P):
+        K, N, qw, sc, z, xs = layers[i % len(layers)]
+        M = GEMV_MS[(i // len(layers)) % len(GEMV_MS)]
+        m = rng.integers(0, M, P)
+        n = rng.integers(0, N, P)
+        t0 = time.perf_counter()
+        oracle.linear_at(xs[M], qw, sc, z, N, m, n)
+        return time.perf_counter() - t0, gemv_bytes(N, K, M) / (M * N) * P
+
+    dt, _ = one_step(0, 512)
+    per_out = dt / 512
+    budget = 120.0
+    P = int(max(16, min(1 << 16, budget / max(args.steps + args.warmup, 1) / per_out)))
+    for i in range(args.warmup):
+        one_step(i, P)
+    t_tot, b_tot = 0.0, 0.0
+    for i in range(args.steps):
+        dt, b = one_step(i, P)
+        t_tot += dt
+        b_tot += b
+    value = b_tot / t_tot / 1e9
+    line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_tot / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
+            "config": {"workload": WORKLOAD, "sample": f"{P} sampled outputs per step, one layer/M per step"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": omp_threads(), "kind": "oracle",
+                             "sample": f"{P} sampled GEMV outputs per step over {args.steps} steps"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm ---------------
+
+def build_gemv_workload(torch, w4):
+    calls = []
+    quant = []
+    for si, (name, K, N) in enumerate(GEMV_SHAPES):
+        L = workloads.make_layer(workloads.seed_of(1, si), K=K, N=N)
+        W = torch.from_numpy(L.W).cuda()
+        act = torch.from_numpy(L.act_absmean).cuda()
+        qw, sc, z, s = w4.awq_quantize_g128(W, act, workloads.ALPHA)
+        w4.check_device_status()
+        quant.append((W, act, N, K))
+        for j, M in enumerate(GEMV_MS):
+            if j == 0:
+                packed = (qw, sc, z)
+            else:
+                packed = (qw.clone(), sc.clone(), z.clone())
+            xh = workloads.make_activations(workloads.seed_of(1, si), M, L.mult)
+            x = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).cuda()
+            y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            calls.append(dict(x=x, w=packed, y=y, M=M, N=N, K=K, bytes=gemv_bytes(N, K, M)))
+    return calls, quant
+
+
+def time_graph(torch, fn, steps, warmup):
+    """Capture fn() once, replay warmup + steps times; CUDA-event ms per replay."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, g
+
+
+def run_gpu(args, world, rank, local):
+    import torch
+
+    import w4a16_gemm_awq_b200 as w4
+    pk, pk_kind = peaks()
+    calls, quant = build_gemv_workload(torch, w4)
+
+    def step():
+        for c in calls:
+            qw, sc, z = c["w"]
+            w4.w4a16_gemv(c["x"], qw, sc, z, out=c["y"])
+
+    step_bytes = sum(c["bytes"] for c in calls)
+    # warmup (eager, then graph), then the timed region: barrier + sync on both sides
+    for _ in range(max(args.warmup, 3)):
+        step()
+    w4.check_device_status()
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        step()
+    torch.cuda.current_stream().wait_stream(cap)
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    e0.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    w4.check_device_status()
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms, gbs = aggregate(ms_local, step_bytes, world)
+    del g
+
+    # end to end through the public API with host buffers: pinned x -> device, GEMV, y -> host
+    hx = [c["x"].cpu().pin_memory() for c in calls]
+    hy = [torch.empty_like(c["y"], device="cpu").pin_memory() for c in calls]
+
+    def e2e_step():
+        for c, a, b in zip(calls, hx, hy):
+            c["x"].copy_(a, non_blocking=True)
+            qw, sc, z = c["w"]
+            w4.w4a16_gemv(c["x"], qw, sc, z, out=c["y"])
+            b.copy_(c["y"], non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 2000))
+    ms_e2e, ge = time_graph(torch, e2e_step, e2e_steps, max(args.warmup, 3))
+    del ge
+    ms_e2e = reduce_max(ms_e2e, world)
+    h2d = sum(c["x"].numel() * 2 for c in calls)
+    d2h = sum(c["y"].numel() * 2 for c in calls)
+
+    # prefill GEMM on the same shapes (weights of the M = 1 copy; M = 512, 2048, 8192)
+    gemm = None
+    if not args.skip_gemm:
+        flops, t_ms = 0.0, 0.0
+        per = []
+        for ci in range(0, len(calls), len(GEMV_MS)):
+            c = calls[ci]
+            qw, sc, z = c["w"]
+            for M in GEMM_MS:
+                x = torch.randn(M, c["K"], device="cuda").to(torch.bfloat16)
+                y = torch.empty(M, c["N"], dtype=torch.bfloat16, device="cuda")
+                ms1, gg = time_graph(torch, lambda: w4.w4a16_gemm(x, qw, sc, z, out=y), 20, 3)
+                del gg
+                f = 2.0 * M * c["N"] * c["K"]
+                flops += f
+                t_ms += ms1
+                per.append({"K": c["K"], "N": c["N"], "M": M, "tflops": round(f / ms1 / 1e9, 1)})
+                del x, y
+        w4.check_device_status()
+        tf = flops / t_ms / 1e9
+        peak = pk["bf16_tflops"]
+        gemm = {"value": tf, "unit": "TFLOP/s", "workload": "prefill GEMM, Llama-3-8B shapes x M in {512, 2048, "
+                "8192}", "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                      "frac": tf / peak, "peak_kind": f"{pk_kind} bf16 burst"},
+                "per_call": per}
+
+    # quantize throughput on the four layers (fp32 W -> packed), algorithmic 4.5195 B/weight
+    qinfo = None
+    if not args.skip_quant:
+        qb, qms = 0.0, 0.0
+        for W, act, N, K in quant:
+            ms1, gq = time_graph(torch, lambda: w4.awq_quantize_g128(W, act, workloads.ALPHA), 10, 2)
+            del gq
+            qb += N * K * 4 + workloads.packed_bytes(N, K) + K * 4
+            qms += ms1
+        qinfo = {"value": qb / qms / 1e6, "unit": "GB/s", "workload": "awq_quantize_g128 on the four Llama-3-8B "
+                 "layers (218 M fp32 weights)", "frac_of_hbm": qb / qms / 1e6 / pk["hbm_gbs"]}
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.skip_cpu:
+        v, secs, outs, desc = oracle_sample(args.cpu_budget)
+        cpu = {"value": v, "unit": "GB/s", "cores": omp_threads(), "kind": "oracle", "sample": desc,
+               "seconds": round(secs, 2)}
+    traffic = profile_traffic()
+    per_gpu_gbs = step_bytes / (ms_local * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": DATA,
+        "config": {"workload": WORKLOAD, "M": GEMV_MS, "step": "16 GEMV calls (4 shapes x 4 M), one CUDA graph",
+                   "l2": "inputs larger than L2: one packed-weight copy per call, %.0f MB per step" % (step_bytes / 1e6),
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": per_gpu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": per_gpu_gbs / pk["hbm_gbs"], "traffic": traffic, "peak_kind": f"{pk_kind} HBM copy",
+                     "kernel": "gemv_w4a16_kernel", "bytes_per_launch": step_bytes / len(calls)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": step_bytes * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "gpu_launches": len(calls) * args.steps,
+        "clocks": clocks,
+        "gemm": gemm,
+        "quantize": qinfo,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def profile_traffic():
+    """DRAM bytes per GEMV launch from the committed ncu summary, if one exists for the
+    current kernel (a line 'traffic_bytes_per_launch: <int>'); else None."""
+    path = os.path.join(ROOT, "profiles", "gemv_w4a16_llama3_8b_decode.md")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        if line.startswith("traffic_bytes_per_launch:"):
+            try:
+                return int(line.split(":", 1)[1].strip())
+            except ValueError:
+                return None
+    return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--skip-gemm", action="store_true")
+    ap.add_argument("--skip-quant", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        # the CPU oracle needs no process group: rank 0 alone runs, the other ranks exit 0
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

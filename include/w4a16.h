@@ -1,0 +1,153 @@
+/*
+ * w4a16.h -- C ABI of the B200 (sm_100a) W4A16 quantized-linear library, libw4a16.so.
+ *
+ * The operations are those of activation-aware weight quantization (AWQ) and of the
+ * dense-and-sparse decomposition of SqueezeLLM:
+ *   - awq_quantize_g128: per-input-channel activation-aware scaling, then asymmetric
+ *     uint4 round-to-nearest in groups of 128 along K, packed 8 codes per 32-bit word
+ *     [AWQ (MLSys 2024) translation, sections 2, 3.1 and 3.2; DeepCompressor README,
+ *     perplexity table row "W4A16 g128"; AWQ translation section 1 for TinyChat's
+ *     4-bit packing];
+ *   - w4a16_linear / w4a16_gemv / w4a16_gemm: y = x . dequant(Wq)^T (+ x . W_sparse^T)
+ *     with the weights dequantized on the fly [AWQ translation, section 1: TinyChat's
+ *     on-the-fly dequantization; SqueezeLLM article, sections 2.2 and 2.3: W x =
+ *     W_dense x + W_sparse x, the sparse part an fp16 matrix];
+ *   - w4a16_split_outliers: move the largest |w| * act_absmean entries into an fp16 CSR
+ *     W_sparse [SqueezeLLM article, section 2.2; ratio 0.0045 from section 5.3].
+ *
+ * Conventions for every entry point
+ *   - Tensor arguments are DEVICE pointers, allocated and owned by the caller.  The
+ *     library keeps no pointer after a call returns.  It allocates no device memory
+ *     except one static device status word per GPU, created when the library is loaded.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream).  The return value covers argument validation and the kernel launch.
+ *     Problems found while a kernel runs are reported later: the kernel records them in
+ *     the device status word, and w4a16_check_device_status() returns them.  These
+ *     problems are non-finite inputs, fp16 overflow, CSR indices out of range, and a
+ *     pipeline wait that ran out.  When a call fails, its outputs are unspecified.
+ *   - Element types are passed as raw bits: bf16 and fp16 as uint16_t, fp32 as float.
+ *   - Shapes: W is [N][K] (out x in), x is [M][K], y is [M][N], all row-major and dense.
+ *     K must be a positive multiple of 1024 (so a row's zero points fill whole words) and
+ *     N a positive multiple of 128.  Every pointer must be 16-byte aligned, except the
+ *     CSR arrays, which need only natural alignment.
+ *
+ * Packed weight format (shared with any reader of the quantized weights):
+ *   qweight[n][k/8]  uint32.  Nibble j (bits 4j..4j+3) holds the code of element
+ *                    k = 8*(k/8) + ORDER[j], ORDER = {0,2,4,6,1,3,5,7}.  Hence
+ *                    (word >> 4i) & 0x000F000F holds elements 2i and 2i+1 in its low
+ *                    and high 16-bit halves.
+ *   scales[n][g]     fp16 bits, g = k/128.
+ *   zeros[n][g/8]    uint32.  Nibble j holds the zero point of group 8*(g/8) + j.
+ *   Dequantized weight: w = (q - z) * scale.  This is exact in fp32.
+ *
+ * CSR outlier matrix (w4a16_csr), in the same scaled space as the packed weights:
+ *   row_ptr[N+1] int32, row_ptr[0] = 0, row_ptr[N] = nnz, non-decreasing;
+ *   col_idx[nnz] int32, strictly ascending within a row, each in [0, K);
+ *   values[nnz]  fp16 bits.
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4A16_OK = 0,
+    W4A16_ERR_NULL = 1,        /* a required pointer is NULL */
+    W4A16_ERR_SHAPE = 2,       /* bad size (M, N, K, nnz) or CSR structure */
+    W4A16_ERR_ALIGN = 3,       /* a pointer is not aligned as required */
+    W4A16_ERR_VALUE = 4,       /* non-finite input, negative act_absmean, fp16 overflow */
+    W4A16_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+    W4A16_ERR_TIMEOUT = 6,     /* a kernel's bounded pipeline wait ran out */
+    W4A16_ERR_UNSUPPORTED = 7  /* no sm_100 device, or a size beyond a documented limit */
+} w4a16_status;
+
+typedef struct {
+    const int32_t* row_ptr;  /* [N+1] device */
+    const int32_t* col_idx;  /* [nnz] device, ascending within each row */
+    const uint16_t* values;  /* [nnz] device, fp16 bits */
+    int64_t nnz;
+} w4a16_csr;
+
+/*
+ * awq_quantize_g128 -- activation-aware scaling + group-wise uint4 RTN + packing.
+ *   [AWQ translation, 3.2 (per-channel scaling); 2 (RTN); DeepCompressor "W4A16 g128"]
+ *
+ *   s_k      = max( float(pow(double(act_absmean[k]), double(alpha))), 1e-4 )
+ *   w'       = float(W[n][k] * s_k)
+ *   per group of 128 along K:
+ *     scale  = fp16_rne( max((max w' - min w') / 15, 1e-5) )
+ *     z      = clamp(rint(-min w' / scale), 0, 15)
+ *     q      = clamp(rint(w' / scale) + z, 0, 15)       (rint: ties to even)
+ *   Every float step is a single IEEE-754 operation with round-to-nearest-even.  The
+ *   outputs are therefore bit-reproducible by any correct implementation of these steps.
+ *
+ *   W            [N][K] fp32, device.
+ *   act_absmean  [K] fp32, device: mean |x| per input channel over calibration data.
+ *                Each value must be finite and >= 0.
+ *   alpha        finite exponent (AWQ searches it in [0, 1]).
+ *   qweight      [N][K/8] uint32, device, output.
+ *   scales       [N][K/128] fp16 bits, device, output.
+ *   zeros        [N][K/1024] uint32, device, output.
+ *   s_out        [K] fp32, device, output, may be NULL.  The caller divides the layer's
+ *                input by s (x' = x / s) before calling w4a16_linear.
+ *   Errors: NULL, SHAPE, ALIGN and VALUE (non-finite alpha) when called.  Later, through
+ *   w4a16_check_device_status: VALUE for a non-finite W, s or w', a negative
+ *   act_absmean, or a scale that overflows fp16.
+ */
+w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float alpha, int64_t N,
+                               int64_t K, uint32_t* qweight, uint16_t* scales, uint32_t* zeros,
+                               float* s_out, void* stream);
+
+/*
+ * w4a16_linear -- y = bf16_rne( x . dequant(Q)^T + x . W_sparse^T ), fp32 accumulation.
+ *   [AWQ translation, 1 (TinyChat on-the-fly dequantization); SqueezeLLM article 2.3]
+ *
+ *   x        [M][K] bf16 bits, device.  This is the layer input already divided by s.
+ *   qweight, scales, zeros: the packed weights, laid out as above.
+ *   outliers host pointer to a w4a16_csr whose arrays are on the device, or NULL when
+ *            there is no sparse term.  nnz may be 0.
+ *   y        [M][N] bf16 bits, device, output.  It must not overlap any input.
+ *   M >= 1.  M <= 16 runs the decode GEMV.  Larger M runs the tensor-core GEMM.
+ *   Errors: NULL, SHAPE, ALIGN and UNSUPPORTED when called.  Later: SHAPE if a CSR index
+ *   is out of range (that entry is skipped), TIMEOUT if a pipeline wait runs out.
+ */
+w4a16_status w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                          const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
+                          int64_t M, int64_t N, int64_t K, void* stream);
+
+/* w4a16_gemv -- the decode path of w4a16_linear, restricted to 1 <= M <= 16
+ * (W4A16_ERR_SHAPE otherwise).  Arguments and result are as for w4a16_linear. */
+w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                        const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
+                        int64_t M, int64_t N, int64_t K, void* stream);
+
+/* w4a16_gemm -- the tcgen05 tensor-core path of w4a16_linear, for any M >= 1.  Arguments
+ * and result are as for w4a16_linear.  Weights are dequantized to bf16 inside the kernel.
+ * When a CSR is given, its values are added to those weights before the bf16 rounding
+ * that feeds the tensor cores. */
+w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                        const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
+                        int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * w4a16_check_device_status -- synchronize `stream` and return the first problem that a
+ * kernel recorded since the last call, or W4A16_OK.  This clears the record.  The record
+ * is per device and shared by all streams of that device.
+ */
+w4a16_status w4a16_check_device_status(void* stream);
+
+/* Static, human-readable name of a status value. */
+const char* w4a16_status_string(w4a16_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int w4a16_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

@@ -1,0 +1,101 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry point that
+include/w4a16.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import w4a16_gemm_awq_b200 as w4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a16.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:w4a16_status|const char\s*\*|int)\s+(\w+)\s*\(", text, flags=re.M)
+
+
+@pytest.fixture(scope="module")
+def L():
+    w4.build()
+    return w4.lib()
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"awq_quantize_g128", "w4a16_linear", "w4a16_gemv", "w4a16_gemm", "w4a16_check_device_status",
+            "w4a16_status_string", "w4a16_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", w4.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_status_strings(L):
+    for code in range(8):
+        assert len(w4.status_string(code)) > 0
+    assert w4.status_string(99) == "unknown status"
+    assert w4.version() >= 100
+
+
+FAKE = 1 << 20  # a 16-byte-aligned address that is never dereferenced: validation fails first
+
+
+def _linear(L, name, x=FAKE, qw=FAKE, sc=FAKE, z=FAKE, csr=None, y=FAKE, M=1, N=128, K=1024):
+    fn = getattr(L, name)
+    return fn(ctypes.c_void_p(x), ctypes.c_void_p(qw), ctypes.c_void_p(sc), ctypes.c_void_p(z),
+              ctypes.byref(csr) if csr is not None else None, ctypes.c_void_p(y), M, N, K, None)
+
+
+@pytest.mark.parametrize("name", ["w4a16_linear", "w4a16_gemv", "w4a16_gemm"])
+def test_linear_validation(L, name):
+    assert _linear(L, name, x=0) == w4.ERR_NULL
+    assert _linear(L, name, y=0) == w4.ERR_NULL
+    assert _linear(L, name, K=1000) == w4.ERR_SHAPE
+    assert _linear(L, name, N=100) == w4.ERR_SHAPE
+    assert _linear(L, name, M=0) == w4.ERR_SHAPE
+    assert _linear(L, name, x=FAKE + 2) == w4.ERR_ALIGN
+    assert _linear(L, name, sc=FAKE + 8) == w4.ERR_ALIGN
+    bad = w4.Csr(None, None, None, 5)
+    assert _linear(L, name, csr=bad) == w4.ERR_NULL
+    neg = w4.Csr(FAKE, FAKE, FAKE, -1)
+    assert _linear(L, name, csr=neg) == w4.ERR_SHAPE
+    odd = w4.Csr(FAKE + 2, FAKE, FAKE, 3)
+    assert _linear(L, name, csr=odd) == w4.ERR_ALIGN
+
+
+def test_gemv_rejects_large_m(L):
+    assert _linear(L, "w4a16_gemv", M=17) == w4.ERR_SHAPE
+
+
+def test_quantize_validation(L):
+    def q(W=FAKE, a=FAKE, alpha=0.5, N=128, K=1024, qw=FAKE, sc=FAKE, z=FAKE, s=None):
+        return L.awq_quantize_g128(ctypes.c_void_p(W), ctypes.c_void_p(a), ctypes.c_float(alpha), N, K,
+                                   ctypes.c_void_p(qw), ctypes.c_void_p(sc), ctypes.c_void_p(z),
+                                   ctypes.c_void_p(s) if s else None, None)
+    assert q(W=0) == w4.ERR_NULL
+    assert q(z=0) == w4.ERR_NULL
+    assert q(K=1536) == w4.ERR_SHAPE
+    assert q(N=0) == w4.ERR_SHAPE
+    assert q(W=FAKE + 4) == w4.ERR_ALIGN
+    assert q(s=FAKE + 4) == w4.ERR_ALIGN
+    assert q(alpha=float("nan")) == w4.ERR_VALUE
+    assert q(alpha=float("inf")) == w4.ERR_VALUE
+
+
+def test_binding_has_no_cpu_path():
+    """The binding refuses CPU tensors instead of computing anything itself."""
+    import torch
+    x = torch.zeros(1, 1024, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        w4.w4a16_linear(x, torch.zeros(128, 128, dtype=torch.int32), torch.zeros(128, 8, dtype=torch.int16),
+                        torch.zeros(128, 1, dtype=torch.int32))

@@ -1,0 +1,109 @@
+"""GPU decode GEMV (1 <= M <= 16) against the oracle, with and without the CSR outlier term."""
+import numpy as np
+import pytest
+import torch
+
+import w4a16_gemm_awq_b200 as w4
+import workloads
+from parity import Case, check_close, dev_bits, dev_csr, host_bf16_as_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def gemv(case_dev, fn=None):
+    fn = fn or w4.w4a16_gemv
+    y = fn(case_dev["x"], case_dev["qweight"], case_dev["scales"], case_dev["zeros"], csr=case_dev["csr"])
+    w4.check_device_status()
+    return y
+
+
+def depth(K):
+    return K // 128 + 64
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 7, 8, 9, 15, 16])
+@pytest.mark.parametrize("csr", [False, True])
+def test_gemv_small_full_output(orc, M, csr):
+    c = Case(orc, seed=100 + M, K=2048, N=256, M=M, csr=csr)
+    y = host_bf16_as_f64(gemv(c.device()))
+    ref, ref_abs = c.reference(orc)
+    check_close(y, ref, ref_abs, 0.0, depth(c.K), f"M={M} csr={csr}")
+
+
+@pytest.mark.parametrize("K,N", [(1024, 128), (3072, 384), (8192, 128), (1024, 4096)])
+def test_gemv_odd_shapes(orc, K, N):
+    c = Case(orc, seed=K + N, K=K, N=N, M=5, csr=True)
+    y = host_bf16_as_f64(gemv(c.device()))
+    ref, ref_abs = c.reference(orc)
+    check_close(y, ref, ref_abs, 0.0, depth(K), f"{K}x{N}")
+
+
+def test_gemv_empty_csr_is_bit_identical(orc):
+    c = Case(orc, seed=7, K=2048, N=256, M=4)
+    d = c.device()
+    y0 = gemv(d)
+    d["csr"] = (torch.zeros(c.N + 1, dtype=torch.int32, device="cuda"), torch.zeros(0, dtype=torch.int32, device="cuda"),
+                torch.zeros(0, dtype=torch.int16, device="cuda"))
+    y1 = gemv(d)
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+
+
+def test_gemv_csr_only_and_dense_rows(orc):
+    """All-zero dense part; one CSR row fully dense, others empty or single."""
+    K, N, M = 1024, 128, 3
+    qw, sc, z, _ = orc.awq_quantize_g128(np.zeros((N, K), np.float32), np.ones(K, np.float32), 0.0)
+    rng = np.random.default_rng(8)
+    rows = [np.arange(K) if n == 5 else (np.array([n * 7 % K]) if n % 3 == 0 else np.array([], np.int64))
+            for n in range(N)]
+    rp = np.concatenate([[0], np.cumsum([len(r) for r in rows])]).astype(np.int32)
+    ci = np.concatenate(rows).astype(np.int32)
+    v = rng.standard_normal(ci.size).astype(np.float16).view(np.uint16)
+    x = workloads.uniform_bf16(9, (M, K))
+    d = dict(x=torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda(), qweight=dev_bits(qw, torch.int32),
+             scales=dev_bits(sc, torch.int16), zeros=dev_bits(z, torch.int32), csr=dev_csr((rp, ci, v)))
+    y = host_bf16_as_f64(gemv(d))
+    ref, ref_abs = orc.linear(x, qw, sc, z, N, csr=(rp, ci, v), with_abs=True)
+    check_close(y, ref, ref_abs, 0.0, K + 64, "csr only")
+
+
+def test_gemv_reports_bad_csr(orc):
+    c = Case(orc, seed=11, K=1024, N=128, M=2)
+    d = c.device()
+    rp = torch.zeros(c.N + 1, dtype=torch.int32, device="cuda")
+    rp[1:] = 1
+    d["csr"] = (rp, torch.tensor([c.K + 5], dtype=torch.int32, device="cuda"),
+                torch.tensor([0x3C00], dtype=torch.int16, device="cuda"))
+    w4.w4a16_gemv(d["x"], d["qweight"], d["scales"], d["zeros"], csr=d["csr"])
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.check_device_status()
+    assert e.value.code == w4.ERR_SHAPE
+
+
+def test_linear_dispatches_to_gemv(orc):
+    c = Case(orc, seed=12, K=2048, N=256, M=16, csr=True)
+    d = c.device()
+    a = gemv(d)
+    b = gemv(d, w4.w4a16_linear)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_gemv_config0_full(orc):
+    """4096 x 4096, M = 1, alpha = 0.5: the whole output against the oracle."""
+    c = Case(orc, seed=workloads.seed_of(0, 0), K=4096, N=4096, M=1)
+    y = host_bf16_as_f64(gemv(c.device()))
+    ref, ref_abs = c.reference(orc)
+    check_close(y, ref, ref_abs, 0.0, depth(c.K), "config 0")
+
+
+FULL = ([(1, i, K, N, M, False) for i, (_, K, N) in enumerate(workloads.LLAMA3_8B) for M in (1, 4, 8, 16)]
+        + [(3, i, K, N, M, True) for i, (_, K, N) in enumerate(workloads.LLAMA2_13B) for M in (1, 16)]
+        + [(4, i, K, N, 1, False) for i, (_, K, N) in enumerate(workloads.LLAMA2_70B)])
+
+
+@pytest.mark.parametrize("cfg,i,K,N,M,csr", FULL, ids=[f"c{c}_{K}x{N}_M{M}" for c, _, K, N, M, _ in FULL])
+def test_gemv_full_shapes_sampled(orc, cfg, i, K, N, M, csr):
+    c = Case(orc, seed=workloads.seed_of(cfg, i), K=K, N=N, M=M, csr=csr)
+    y = host_bf16_as_f64(gemv(c.device()))
+    m, n = c.sample(seed=cfg * 10 + i)
+    ref, ref_abs = c.reference_at(orc, m, n)
+    check_close(y[m, n], ref, ref_abs, 0.0, depth(K), f"{K}x{N} M={M}")

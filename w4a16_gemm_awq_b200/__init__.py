@@ -1,0 +1,160 @@
+"""Python binding of libw4a16.so (the B200 W4A16 quantized-linear library).
+
+Argument marshalling only: every step of the computation runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current stream.  The entry points
+mirror the C ABI in include/w4a16.h:
+
+  awq_quantize_g128(W, act_absmean, alpha)      -> (qweight, scales, zeros, s)
+  w4a16_linear(x, qweight, scales, zeros, csr)  -> y      (any M)
+  w4a16_gemv(...)                               -> y      (1 <= M <= 16)
+  w4a16_gemm(...)                               -> y      (tcgen05 path, any M)
+  check_device_status()                         -> raises W4A16Error on a recorded problem
+
+Bit containers: qweight and zeros are int32 tensors holding uint32 words, scales is an
+int16 tensor holding fp16 bits, x and y are bfloat16 tensors.  A CSR is a tuple
+(row_ptr int32 [N+1], col_idx int32 [nnz], values int16 fp16-bits [nnz]) of CUDA tensors.
+
+There is no fallback: if the library is not built, or there is no sm_100 GPU, the calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw4a16.so")
+
+STATUS = {0: "W4A16_OK", 1: "W4A16_ERR_NULL", 2: "W4A16_ERR_SHAPE", 3: "W4A16_ERR_ALIGN",
+          4: "W4A16_ERR_VALUE", 5: "W4A16_ERR_CUDA", 6: "W4A16_ERR_TIMEOUT", 7: "W4A16_ERR_UNSUPPORTED"}
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_VALUE, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = range(8)
+
+
+class W4A16Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Csr(ctypes.Structure):
+    _fields_ = [("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p), ("values", ctypes.c_void_p),
+                ("nnz", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    from . import buildlib
+    return buildlib.build(force=force)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libw4a16.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with w4a16_gemm_awq_b200.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
+        L.awq_quantize_g128.argtypes = [P, P, F, I64, I64, P, P, P, P, P]
+        for name in ("w4a16_linear", "w4a16_gemv", "w4a16_gemm"):
+            fn = getattr(L, name)
+            fn.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P]
+        L.w4a16_check_device_status.argtypes = [P]
+        L.w4a16_status_string.argtypes = [ctypes.c_int]
+        L.w4a16_status_string.restype = ctypes.c_char_p
+        L.w4a16_version.argtypes = []
+        for name in ("awq_quantize_g128", "w4a16_linear", "w4a16_gemv", "w4a16_gemm", "w4a16_check_device_status",
+                     "w4a16_version"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise W4A16Error(code, what)
+
+
+def _need(t, dtype, ndim, name):
+    if not (t.is_cuda and t.dtype == dtype and t.dim() == ndim and t.is_contiguous()):
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor of rank {ndim}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def awq_quantize_g128(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, out=None):
+    """W fp32 [N][K], act_absmean fp32 [K] -> (qweight int32 [N][K/8], scales int16 [N][K/128],
+    zeros int32 [N][K/1024], s fp32 [K])."""
+    _need(W, torch.float32, 2, "W")
+    _need(act_absmean, torch.float32, 1, "act_absmean")
+    N, K = W.shape
+    dev = W.device
+    if out is None:
+        out = (torch.empty(N, K // 8, dtype=torch.int32, device=dev),
+               torch.empty(N, max(K // 128, 1), dtype=torch.int16, device=dev),
+               torch.empty(N, max(K // 1024, 1), dtype=torch.int32, device=dev),
+               torch.empty(K, dtype=torch.float32, device=dev))
+    qw, sc, z, s = out
+    code = lib().awq_quantize_g128(_ptr(W), _ptr(act_absmean), ctypes.c_float(alpha), N, K, _ptr(qw), _ptr(sc),
+                                   _ptr(z), _ptr(s), _stream(dev))
+    _check(code, "awq_quantize_g128")
+    return qw, sc, z, s
+
+
+def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None):
+    _need(x, torch.bfloat16, 2, "x")
+    _need(qweight, torch.int32, 2, "qweight")
+    _need(scales, torch.int16, 2, "scales")
+    _need(zeros, torch.int32, 2, "zeros")
+    M, K = x.shape
+    N = qweight.shape[0]
+    if qweight.shape[1] * 8 != K:
+        raise ValueError(f"qweight {tuple(qweight.shape)} does not match K = {K}")
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    cs = None
+    if csr is not None:
+        rp, ci, v = csr
+        _need(rp, torch.int32, 1, "row_ptr")
+        cs = Csr(rp.data_ptr(), ci.data_ptr() if ci.numel() else None, v.data_ptr() if v.numel() else None,
+                 int(ci.numel()))
+    code = getattr(lib(), name)(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros),
+                                ctypes.byref(cs) if cs is not None else None, _ptr(y), M, N, K, _stream(x.device))
+    _check(code, name)
+    return y
+
+
+def w4a16_linear(x, qweight, scales, zeros, csr=None, out=None):
+    return _linear("w4a16_linear", x, qweight, scales, zeros, csr, out)
+
+
+def w4a16_gemv(x, qweight, scales, zeros, csr=None, out=None):
+    return _linear("w4a16_gemv", x, qweight, scales, zeros, csr, out)
+
+
+def w4a16_gemm(x, qweight, scales, zeros, csr=None, out=None):
+    return _linear("w4a16_gemm", x, qweight, scales, zeros, csr, out)
+
+
+def check_device_status(stream=None):
+    """Synchronize and raise W4A16Error if a kernel recorded a problem since the last check."""
+    s = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream(torch.device("cuda"))
+    _check(lib().w4a16_check_device_status(s), "device status")
+
+
+def status_string(code: int) -> str:
+    return lib().w4a16_status_string(code).decode()
+
+
+def version() -> int:
+    return lib().w4a16_version()

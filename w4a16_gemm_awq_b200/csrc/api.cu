@@ -1,0 +1,250 @@
+// api.cu -- the extern "C" entry points of libw4a16.so: argument validation, dispatch on M,
+// TMA tensor-map encoding and the per-device status word.  The operations and formats are
+// documented in include/w4a16.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "internal.h"
+#include "w4a16.h"
+
+namespace w4a16 {
+
+// Problems found by kernels while they run (bit set of kErrValue / kErrShape / kErrTimeout).
+__device__ unsigned g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxN = int64_t(1) << 22;
+constexpr int64_t kMaxK = int64_t(1) << 20;
+constexpr int64_t kMaxM = int64_t(1) << 24;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool sm100 = false;
+    int num_sms = 0;
+    unsigned* status = nullptr;  // device address of g_device_status
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+w4a16_status device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return W4A16_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return W4A16_ERR_CUDA;
+        d.sm100 = prop.major == 10 && prop.minor == 0;
+        d.num_sms = prop.multiProcessorCount;
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return W4A16_ERR_CUDA;
+        d.status = static_cast<unsigned*>(addr);
+        d.ready = true;
+    }
+    *out = &d;
+    return d.sm100 ? W4A16_OK : W4A16_ERR_UNSUPPORTED;
+}
+
+w4a16_status encoder(EncodeTiledFn* out) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return W4A16_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    *out = g_encode;
+    return W4A16_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline w4a16_status from_cuda(cudaError_t e) { return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA; }
+
+struct LinearArgs {
+    const uint16_t* x;
+    const uint32_t* qweight;
+    const uint16_t* scales;
+    const uint32_t* zeros;
+    const int32_t* row_ptr = nullptr;
+    const int32_t* col_idx = nullptr;
+    const uint16_t* vals = nullptr;
+    long long nnz = 0;
+    uint16_t* y;
+    int64_t M, N, K;
+};
+
+w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                             const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N,
+                             int64_t K, LinearArgs* a) {
+    if (!x || !qweight || !scales || !zeros || !y) return W4A16_ERR_NULL;
+    if (M < 1 || M > kMaxM || N < 128 || N % 128 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK)
+        return W4A16_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(zeros, 16) || !aligned(y, 16))
+        return W4A16_ERR_ALIGN;
+    *a = LinearArgs{x, qweight, scales, zeros};
+    a->y = y;
+    a->M = M;
+    a->N = N;
+    a->K = K;
+    if (outliers != nullptr) {
+        if (outliers->nnz < 0 || outliers->nnz > INT_MAX) return W4A16_ERR_SHAPE;
+        if (outliers->nnz > 0 || outliers->row_ptr != nullptr) {
+            if (!outliers->row_ptr) return W4A16_ERR_NULL;
+            if (outliers->nnz > 0 && (!outliers->col_idx || !outliers->values)) return W4A16_ERR_NULL;
+            if (!aligned(outliers->row_ptr, 4) || (outliers->col_idx && !aligned(outliers->col_idx, 4)) ||
+                (outliers->values && !aligned(outliers->values, 2)))
+                return W4A16_ERR_ALIGN;
+            a->row_ptr = outliers->row_ptr;
+            a->col_idx = outliers->col_idx;
+            a->vals = outliers->values;
+            a->nnz = outliers->nnz;
+        }
+    }
+    return W4A16_OK;
+}
+
+w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream) {
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    return from_cuda(launch_gemv(a.x, a.qweight, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
+                                 (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status, stream));
+}
+
+int pick_bn(int64_t M) {
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+w4a16_status run_gemm(const LinearArgs& a, cudaStream_t stream) {
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    EncodeTiledFn enc = nullptr;
+    st = encoder(&enc);
+    if (st != W4A16_OK) return st;
+    const int bn = pick_bn(a.M);
+    GemmMaps maps;
+    {   // x: bf16 [M][K]; box 64 k (128 bytes) x bn tokens; 128-byte swizzle
+        cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
+        cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)bn};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4A16_ERR_CUDA;
+    }
+    {   // qweight: uint32 [N][K/8]; box 8 words (64 k) x 128 rows; 32-byte swizzle
+        cuuint64_t dims[2] = {(cuuint64_t)(a.K / 8), (cuuint64_t)a.N};
+        cuuint64_t strides[1] = {(cuuint64_t)(a.K / 8) * 4};
+        cuuint32_t box[2] = {8, 128};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&maps.qw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(a.qweight), dims, strides, box,
+                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4A16_ERR_CUDA;
+    }
+    return from_cuda(launch_gemm(maps, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y, (int)a.M,
+                                 (int)a.N, (int)a.K, bn, d->num_sms, d->status, stream));
+}
+
+}  // namespace
+}  // namespace w4a16
+
+using namespace w4a16;
+
+extern "C" {
+
+w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                               uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, void* stream) {
+    if (!W || !act_absmean || !qweight || !scales || !zeros) return W4A16_ERR_NULL;
+    if (N < 1 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK) return W4A16_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(act_absmean, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
+        !aligned(zeros, 16) || (s_out && !aligned(s_out, 16)))
+        return W4A16_ERR_ALIGN;
+    if (!std::isfinite(alpha)) return W4A16_ERR_VALUE;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    return from_cuda(launch_awq_quantize(W, act_absmean, alpha, (int)N, (int)K, qweight, scales, zeros, s_out,
+                                         d->status, static_cast<cudaStream_t>(stream)));
+}
+
+w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
+                        const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+    LinearArgs a;
+    w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
+    if (st != W4A16_OK) return st;
+    if (M > 16) return W4A16_ERR_SHAPE;
+    return run_gemv(a, static_cast<cudaStream_t>(stream));
+}
+
+w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
+                        const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+    LinearArgs a;
+    w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
+    if (st != W4A16_OK) return st;
+    return run_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
+w4a16_status w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                          const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N,
+                          int64_t K, void* stream) {
+    LinearArgs a;
+    w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
+    if (st != W4A16_OK) return st;
+    return M <= 16 ? run_gemv(a, static_cast<cudaStream_t>(stream)) : run_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
+w4a16_status w4a16_check_device_status(void* stream) {
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A16_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, d->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return W4A16_ERR_CUDA;
+    if (v != 0 && cudaMemset(d->status, 0, sizeof(v)) != cudaSuccess) return W4A16_ERR_CUDA;
+    if (v & kErrTimeout) return W4A16_ERR_TIMEOUT;
+    if (v & kErrShape) return W4A16_ERR_SHAPE;
+    if (v & kErrValue) return W4A16_ERR_VALUE;
+    return W4A16_OK;
+}
+
+const char* w4a16_status_string(w4a16_status status) {
+    switch (status) {
+        case W4A16_OK: return "ok";
+        case W4A16_ERR_NULL: return "null pointer";
+        case W4A16_ERR_SHAPE: return "bad shape or CSR structure";
+        case W4A16_ERR_ALIGN: return "misaligned pointer";
+        case W4A16_ERR_VALUE: return "non-finite or out-of-range value";
+        case W4A16_ERR_CUDA: return "CUDA runtime error";
+        case W4A16_ERR_TIMEOUT: return "kernel pipeline wait timed out";
+        case W4A16_ERR_UNSUPPORTED: return "unsupported device or size";
+    }
+    return "unknown status";
+}
+
+int w4a16_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,358 @@
+// gemm_tc.cu -- prefill W4A16 GEMM on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// y[m][n] = bf16( sum_k x[m][k] * w~[n][k] ),  w~ = bf16((q - z) * scale) (+ CSR value)
+//
+// [AWQ (MLSys 2024) translation, section 1: TinyChat dequantizes the packed 4-bit weights on
+//  the fly inside the linear-layer kernel; SqueezeLLM article, section 2.3: W x = W_dense x +
+//  W_sparse x.  At prefill sizes the layer is a dense contraction and runs on tensor cores.]
+//
+// Design (B200, one CTA per SM, one 128-channel x BN-token output tile per CTA):
+//   - Swap-AB.  MMA M = 128 output channels, MMA N = BN tokens, both operands K-major.
+//     D[channel][token] accumulates in TMEM (fp32, BN columns).
+//   - The A operand (the weights) lives in TMEM.  Four dequant warps each own 32 TMEM lanes,
+//     one channel row per thread.  Each thread reads its row's 8 packed words per 64-k
+//     stage from shared memory and dequantizes them in registers: LOP3 magic-number unpack
+//     to bf16 (128 + q), exact subtraction of (128 + z), multiplication by the bf16 group
+//     scale.  The thread then writes the 32 bf16x2 columns into a TMEM A-stage with
+//     tcgen05.st.  The dequantized weights never pass through shared memory, so shared
+//     memory bandwidth serves only the TMA fills and the MMA's reads of x.
+//   - The B operand (x) is TMA-staged: a 64-k x BN-token box, 128-byte swizzle, matching the
+//     canonical K-major SW128 UMMA layout.  The packed weights of the stage (128 rows x 32
+//     bytes) arrive on the same mbarrier.
+//   - Warp roles: warp 0 issues the TMA, warp 1 issues tcgen05.mma from one thread, and
+//     warps 2..5 dequantize and then run the epilogue.  There are four smem stages and
+//     four TMEM A-stages, linked by mbarriers; tcgen05.commit releases the stages.
+//   - CSR outlier term: each dequant thread walks its row of the CSR.  It adds each value
+//     (fp32) to the dequantized weight at that column before the bf16 rounding.  The
+//     sparse product therefore rides on the same tensor-core contraction, with no gather
+//     of x and no extra pass.
+//   - Every mbarrier wait is bounded.  On timeout the CTA records kErrTimeout, stops its
+//     loops, drains its own TMA and MMA work with bounded waits, and frees its TMEM.
+#include "common.cuh"
+#include "internal.h"
+
+namespace w4a16 {
+
+constexpr int kGemmThreads = 192;
+constexpr int kStages = 4;
+constexpr int kAStages = 4;
+constexpr int kBK = 64;                          // k per pipeline stage
+constexpr int kWStageBytes = 128 * kBK / 2;      // 128 rows x 32 bytes of packed weights
+constexpr uint32_t kACols = kBK / 2;             // TMEM columns per A-stage (bf16 pairs)
+
+struct GemmArgs {
+    const uint16_t* scales;
+    const uint32_t* zeros;
+    const int32_t* row_ptr;
+    const int32_t* col_idx;
+    const uint16_t* vals;
+    long long nnz;
+    uint16_t* y;
+    int M, N, K;
+    unsigned* err;
+};
+
+template <int BN>
+struct GemmSmem {
+    static constexpr int kXStageBytes = BN * kBK * 2;
+    static constexpr int kXOff = 0;
+    static constexpr int kWOff = kStages * kXStageBytes;
+    static constexpr int kBarOff = kWOff + kStages * kWStageBytes;
+    static constexpr int kBytes = kBarOff + 256;
+    static constexpr uint32_t kTmemCols = (BN + kAStages * kACols) <= 256 ? 256u : 512u;
+};
+
+// UMMA shared-memory descriptor: K-major, 128-byte swizzle, rows of 128 bytes, 8-row
+// groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;            // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset
+    d |= (uint64_t)1 << 46;            // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;            // SWIZZLE_128B
+    return d;
+}
+
+// kind::f16 instruction descriptor: D fp32, A bf16, B bf16, both K-major, M = 128, N = BN.
+template <int BN>
+__device__ __forceinline__ constexpr uint32_t idesc_bf16_m128() {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t patch_bf16x2(uint32_t v, int hi, float add) {
+    const float old = __uint_as_float(hi ? (v & 0xFFFF0000u) : (v << 16));
+    const uint32_t nb = float_to_bf16_bits(old + add);
+    return hi ? ((v & 0x0000FFFFu) | (nb << 16)) : ((v & 0xFFFF0000u) | nb);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                     const GemmArgs p) {
+    using L = GemmSmem<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+    uint64_t* empty = full + kStages;
+    uint64_t* afull = empty + kStages;
+    uint64_t* aempty = afull + kAStages;
+    uint64_t* accfull = aempty + kAStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN;
+    const int nK = p.K / kBK;
+    const int G = p.K >> 7;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1 + 4);  // the MMA commit + one arrive per dequant warp
+        }
+        for (int i = 0; i < kAStages; ++i) {
+            mbar_init(&afull[i], 4);
+            mbar_init(&aempty[i], 1);
+        }
+        mbar_init(accfull, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, L::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&map_x);
+        prefetch_tensormap(&map_w);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t a_col0 = (uint32_t)BN;  // A-stages follow the accumulator columns
+
+    auto fail = [&]() {
+        record_error(p.err, kErrTimeout);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int s = 0; s < nK; ++s) {
+                const int slot = s % kStages;
+                if (*abort_flag) break;
+                if (s >= kStages && !mbar_wait_bounded(&empty[slot], ((s / kStages) - 1) & 1)) {
+                    fail();
+                    break;
+                }
+                mbar_arrive_expect_tx(&full[slot], (uint32_t)(L::kXStageBytes + kWStageBytes));
+                tma_load_2d(smem + L::kXOff + slot * L::kXStageBytes, &map_x, &full[slot], s * kBK, m0);
+                tma_load_2d(smem + L::kWOff + slot * kWStageBytes, &map_w, &full[slot], s * (kBK / 8), n0);
+                ++issued;
+            }
+            // the copies this CTA started must land before it may exit
+            for (int s = issued > kStages ? issued - kStages : 0; s < issued; ++s)
+                (void)mbar_wait_bounded(&full[s % kStages], (s / kStages) & 1);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_m128<BN>();
+            for (int s = 0; s < nK; ++s) {
+                const int slot = s % kStages, as = s % kAStages;
+                if (*abort_flag) break;
+                if (!mbar_wait_bounded(&full[slot], (s / kStages) & 1) ||
+                    !mbar_wait_bounded(&afull[as], (s / kAStages) & 1)) {
+                    fail();
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t xs = smem_u32(smem + L::kXOff + slot * L::kXStageBytes);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk) {
+                    tc_mma_ts(tmem, tmem + a_col0 + (uint32_t)as * kACols + (uint32_t)kk * 8u,
+                              desc_k_sw128(xs + kk * 32), idesc, (s | kk) != 0 ? 1u : 0u);
+                }
+                tc_commit(&empty[slot]);
+                tc_commit(&aempty[as]);
+            }
+            tc_commit(accfull);
+            if (*abort_flag) (void)mbar_wait_bounded(accfull, 0);  // MMAs in flight finish first
+        }
+    } else {
+        // ---------------------------------------------------------------- dequant + epilogue
+        const int quarter = warp & 3;             // TMEM lanes 32*quarter .. +31
+        const int row = 32 * quarter + lane;      // channel within the tile == TMEM lane
+        const int n = n0 + row;
+        const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
+        const uint4* sc_row = reinterpret_cast<const uint4*>(p.scales + (size_t)n * G);
+        const uint32_t* z_row = p.zeros + (size_t)n * (G >> 3);
+
+        // scales and zeros come 8 groups (1024 k, 16 stages) at a time; prefetch one ahead
+        uint4 sc_cur = __ldg(sc_row), sc_nxt = make_uint4(0, 0, 0, 0);
+        uint32_t z_cur = __ldg(z_row), z_nxt = 0;
+        if (G > 8) {
+            sc_nxt = __ldg(sc_row + 1);
+            z_nxt = __ldg(z_row + 1);
+        }
+        uint32_t sb = 0, zb = 0;
+
+        // CSR walk for this row: next entry's column and value
+        int jc = 0, jend = 0, ccol = 0x7FFFFFFF;
+        float cval = 0.0f;
+        if (p.row_ptr != nullptr) {
+            jc = p.row_ptr[n];
+            jend = p.row_ptr[n + 1];
+            if (jc < 0 || jend < jc || (long long)jend > p.nnz) {
+                record_error(p.err, kErrShape);
+                jend = jc;
+            }
+            if (jc < jend) {
+                ccol = p.col_idx[jc];
+                cval = fp16_bits_to_float(p.vals[jc]);
+            }
+        }
+
+        // waits and abort checks are made warp-uniform: tcgen05.st/ld are .sync.aligned
+        auto warp_wait = [&](uint64_t* bar, uint32_t parity) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+            if (!ok && lane == 0) fail();
+            return ok;
+        };
+        auto warp_abort = [&]() { return __any_sync(0xffffffffu, *abort_flag != 0); };
+
+        for (int s = 0; s < nK; ++s) {
+            const int slot = s % kStages, as = s % kAStages;
+            if (warp_abort()) break;
+            if (!warp_wait(&full[slot], (s / kStages) & 1)) break;
+            // the row's 32 bytes in the 32-byte-swizzled W stage: chunk c at c ^ ((row >> 2) & 1)
+            const uint8_t* wrow = smem + L::kWOff + slot * kWStageBytes + row * 32;
+            const int sw = (row >> 2) & 1;
+            const uint4 wa = *reinterpret_cast<const uint4*>(wrow + ((0 ^ sw) << 4));
+            const uint4 wb = *reinterpret_cast<const uint4*>(wrow + ((1 ^ sw) << 4));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+
+            if ((s & 1) == 0) {  // a new group of 128 k
+                const int g = s >> 1;
+                if ((g & 7) == 0 && g > 0) {
+                    sc_cur = sc_nxt;
+                    z_cur = z_nxt;
+                    if ((g >> 3) + 1 < (G >> 3)) {
+                        sc_nxt = __ldg(sc_row + (g >> 3) + 1);
+                        z_nxt = __ldg(z_row + (g >> 3) + 1);
+                    }
+                }
+                const int gi = g & 7;
+                const uint32_t sw2 = u4_get(sc_cur, gi >> 1);
+                const uint16_t sbits = (uint16_t)((gi & 1) ? (sw2 >> 16) : (sw2 & 0xFFFFu));
+                const uint32_t sbf = float_to_bf16_bits(fp16_bits_to_float(sbits));
+                sb = sbf | (sbf << 16);
+                const uint32_t z = (z_cur >> (4 * gi)) & 15u;
+                zb = 0x43004300u | z | (z << 16);
+            }
+
+            uint32_t v[32];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                const uint32_t word = w < 4 ? u4_get(wa, w) : u4_get(wb, w - 4);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    uint32_t t;
+                    asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(t) : "r"(word >> (4 * i)), "r"(0x000F000Fu),
+                        "r"(0x43004300u));
+                    v[4 * w + i] = bf16x2_mul(bf16x2_sub(t, zb), sb);
+                }
+            }
+
+            // CSR values of this row that fall in the stage's 64 columns
+            const int kend = (s + 1) * kBK;
+            while (ccol < kend) {
+                const int pos = ccol - s * kBK;
+                if (pos >= 0 && ccol < p.K) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (c == (pos >> 1)) v[c] = patch_bf16x2(v[c], pos & 1, cval);
+                } else {
+                    record_error(p.err, kErrShape);  // unsorted or out-of-range column
+                }
+                ++jc;
+                if (jc < jend) {
+                    ccol = p.col_idx[jc];
+                    cval = fp16_bits_to_float(p.vals[jc]);
+                } else {
+                    ccol = 0x7FFFFFFF;
+                }
+            }
+
+            if (s >= kAStages && !warp_wait(&aempty[as], ((s / kAStages) - 1) & 1)) break;
+            tc_fence_after();
+            tmem_st_32x32b_x32(tmem + t_lane + a_col0 + (uint32_t)as * kACols, v);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[as]);
+        }
+        const bool aborted = warp_abort();
+        if (jc < jend && !aborted) record_error(p.err, kErrShape);  // entries past column K
+
+        // epilogue: TMEM -> registers -> bf16 -> y[m][n]
+        if (!aborted) {
+            if (warp_wait(accfull, 0)) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c0, r);
+                    tmem_ld_wait();
+                    if (m0 + c0 >= p.M) break;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = m0 + c0 + j;
+                        if (m < p.M) p.y[(size_t)m * p.N + n] = float_to_bf16_bits(__uint_as_float(r[j]));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+    }
+}
+
+template <int BN>
+static cudaError_t launch_bn(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream) {
+    using L = GemmSmem<BN>;
+    // At most 512 / kTmemCols CTAs may share an SM, or a tcgen05.alloc would have to wait for
+    // another CTA's TMEM: the shared-memory request enforces that bound.
+    constexpr int kMinSmem = L::kTmemCols == 512u ? 120 * 1024 : 80 * 1024;
+    const int smem = (L::kBytes + 1024) > kMinSmem ? (L::kBytes + 1024) : kMinSmem;
+    cudaError_t e = cudaFuncSetAttribute(gemm_w4a16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.N / 128, (a.M + BN - 1) / BN);
+    gemm_w4a16_tc_kernel<BN><<<grid, kGemmThreads, smem, stream>>>(maps.x, maps.qw, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const GemmMaps& maps, const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
+                        const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, int M, int N,
+                        int K, int bn, int /*num_sms*/, unsigned* err, cudaStream_t stream) {
+    GemmArgs a{scales, zeros, row_ptr, col_idx, vals, nnz, y, M, N, K, err};
+    switch (bn) {
+        case 32: return launch_bn<32>(maps, a, stream);
+        case 64: return launch_bn<64>(maps, a, stream);
+        case 128: return launch_bn<128>(maps, a, stream);
+        case 256: return launch_bn<256>(maps, a, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace w4a16

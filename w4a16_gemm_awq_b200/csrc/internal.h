@@ -1,0 +1,31 @@
+// internal.h -- launchers behind the C ABI (not part of the public interface).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace w4a16 {
+
+// Bits of the per-device status word that kernels set when they find a problem.
+enum : unsigned { kErrValue = 1u, kErrShape = 2u, kErrTimeout = 4u };
+
+cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, uint32_t* qweight,
+                                uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
+                                cudaStream_t stream);
+
+cudaError_t launch_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
+                        const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
+                        uint16_t* y, int M, int N, int K, int num_sms, unsigned* err, cudaStream_t stream);
+
+// Tensor maps the GEMM needs, encoded by the caller (api.cu) with the driver's encoder.
+struct GemmMaps {
+    CUtensorMap x;   // bf16 [M][K], box 64 (k) x BN (tokens), 128-byte swizzle
+    CUtensorMap qw;  // uint32 [N][K/8], box 16 words (one group) x 128 rows, 64-byte swizzle
+};
+
+cudaError_t launch_gemm(const GemmMaps& maps, const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
+                        const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, int M, int N,
+                        int K, int bn, int num_sms, unsigned* err, cudaStream_t stream);
+
+}  // namespace w4a16

@@ -1,0 +1,132 @@
+// quantize.cu -- AWQ activation-aware scaling + group-wise asymmetric uint4 RTN + packing.
+//
+// [AWQ (MLSys 2024) translation, section 3.2: per-input-channel scaling of the weights by a
+//  factor derived from the activation magnitude; section 2: round-to-nearest; DeepCompressor
+//  README, perplexity table row "W4A16 g128": groups of 128 along K; AWQ translation
+//  section 1: TinyChat's 4-bit packing, 8 codes per 32-bit word.]
+//
+// Work decomposition.  A CTA of 8 warps owns a tile of kRowsPerCta rows x 1024 columns
+// (one zero-point word per row).  It first computes the 1024 per-channel scales s_k into
+// shared memory (double pow, as the definition states).  Then each warp quantizes one row
+// of the tile at a time: 32 lanes x 16 bytes is exactly one group of 128 fp32 weights,
+// so the row's 8 groups arrive as 8 coalesced 128-bit loads per lane, all issued before
+// the first group is processed.  The group's min/max is a 5-step warp-shuffle reduction.
+// Each lane quantizes its 4 weights.  Lane pairs (2i, 2i+1) merge their nibbles into
+// packed word i with one shuffle.
+//
+// Bit-exactness: every float step is a single IEEE operation with round-to-nearest-even
+// (__fmul_rn, __fsub_rn, __fdiv_rn, __fadd_rn, rintf, __float2half_rn).  The build does
+// not use fast-math or flush-to-zero, so any correct implementation of the same steps
+// gives the same bits.
+#include "common.cuh"
+#include "internal.h"
+
+namespace w4a16 {
+
+constexpr int kQuantThreads = 256;
+constexpr int kRowsPerCta = 64;
+
+// Nibble position of each of a lane's 4 elements inside the packed word.  Element e of an
+// 8-wide block sits in nibble j with ORDER[j] = e, ORDER = {0,2,4,6,1,3,5,7}.  The even
+// lane holds elements 0..3, which go to nibbles 0,4,1,5.  The odd lane holds elements
+// 4..7, which go to nibbles 2,6,3,7.
+__device__ __forceinline__ uint32_t place_nibbles(const float q[4], bool odd) {
+    const uint32_t q0 = (uint32_t)q[0], q1 = (uint32_t)q[1], q2 = (uint32_t)q[2], q3 = (uint32_t)q[3];
+    if (!odd) return q0 | (q1 << 16) | (q2 << 4) | (q3 << 20);
+    return (q0 << 8) | (q1 << 24) | (q2 << 12) | (q3 << 28);
+}
+
+__global__ void __launch_bounds__(kQuantThreads)
+awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, float alpha, int N, int K,
+                    uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
+                    uint32_t* __restrict__ zeros, float* __restrict__ s_out, unsigned* err) {
+    __shared__ __align__(16) float s_sm[1024];
+    const int kc = blockIdx.x;                 // 1024-column chunk
+    const int row0 = blockIdx.y * kRowsPerCta;
+    const int G = K >> 7;
+
+    for (int i = threadIdx.x; i < 1024; i += kQuantThreads) {
+        const float a = act[(size_t)kc * 1024 + i];
+        const float p = (float)pow((double)a, (double)alpha);
+        if (!(a >= 0.0f) || isinf(a) || !isfinite(p)) record_error(err, kErrValue);
+        const float s = p > 1e-4f ? p : 1e-4f;
+        s_sm[i] = s;
+        if (s_out != nullptr && blockIdx.y == 0) s_out[(size_t)kc * 1024 + i] = s;
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool odd = lane & 1;
+    for (int r = warp; r < kRowsPerCta; r += kQuantThreads / 32) {
+        const int n = row0 + r;
+        if (n >= N) break;
+        const float* wrow = W + (size_t)n * K + (size_t)kc * 1024 + 4 * lane;
+        float4 v[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            uint4 u = ldg_stream(wrow + g * 128);
+            v[g] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
+                               __uint_as_float(u.w));
+        }
+        uint32_t zword = 0;
+        uint32_t sbits[8];
+        bool bad = false;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            const float4 sv = *reinterpret_cast<const float4*>(&s_sm[g * 128 + 4 * lane]);
+            float w[4] = {__fmul_rn(v[g].x, sv.x), __fmul_rn(v[g].y, sv.y), __fmul_rn(v[g].z, sv.z),
+                          __fmul_rn(v[g].w, sv.w)};
+            float mx = w[0], mn = w[0];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                bad |= !isfinite(w[i]);
+                mx = fmaxf(mx, w[i]);
+                mn = fminf(mn, w[i]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            }
+            float scale32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+            if (scale32 < 1e-5f) scale32 = 1e-5f;
+            const __half h = __float2half_rn(scale32);
+            const float sf = __half2float(h);
+            bad |= isinf(scale32) || isinf(sf);
+            float zf = rintf(__fdiv_rn(-mn, sf));
+            zf = fminf(fmaxf(zf, 0.0f), 15.0f);
+            float q[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float t = __fadd_rn(rintf(__fdiv_rn(w[i], sf)), zf);
+                q[i] = fminf(fmaxf(t, 0.0f), 15.0f);
+            }
+            uint32_t part = place_nibbles(q, odd);
+            part |= __shfl_xor_sync(0xffffffffu, part, 1);
+            if (!odd) qweight[(size_t)n * (K >> 3) + (size_t)kc * 128 + g * 16 + (lane >> 1)] = part;
+            zword |= (uint32_t)zf << (4 * g);
+            sbits[g] = __half_as_ushort(h);
+        }
+        if (bad) record_error(err, kErrValue);
+        if (lane == 0) {
+            zeros[(size_t)n * (K >> 10) + kc] = zword;
+            uint4 sv;
+            sv.x = sbits[0] | (sbits[1] << 16);
+            sv.y = sbits[2] | (sbits[3] << 16);
+            sv.z = sbits[4] | (sbits[5] << 16);
+            sv.w = sbits[6] | (sbits[7] << 16);
+            *reinterpret_cast<uint4*>(scales + (size_t)n * G + (size_t)kc * 8) = sv;
+        }
+    }
+}
+
+cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, uint32_t* qweight,
+                                uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
+                                cudaStream_t stream) {
+    dim3 grid(K / 1024, (N + kRowsPerCta - 1) / kRowsPerCta);
+    awq_quantize_kernel<<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out,
+                                                            err);
+    return cudaGetLastError();
+}
+
+}  // namespace w4a16
