@@ -133,21 +133,21 @@ def quantize_with_scales(W, s):
     s = _c(s, np.float32)
     N, K = W.shape
     qw = np.zeros((N, K // 8), np.uint32)
-    sc = np.zeros((N, K // 128), np.uint16)
-    z = np.zeros((N, max(K // 1024, 1)), np.uint32)
+    sc = np.zeros((K // 128, N), np.uint16)
+    z = np.zeros((K // 128, max(N // 8, 1)), np.uint32)
     _check(_L().oracle_quantize_with_scales(_p(W), _p(s), N, K, _p(qw), _p(sc), _p(z)),
            "quantize_with_scales")
     return qw, sc, z
 
 
 def awq_quantize_g128(W, act_absmean, alpha: float):
-    """-> (qweight u32 [N][K/8], scales fp16 bits u16 [N][K/128], zeros u32 [N][K/1024], s f32 [K])"""
+    """-> (qweight u32 [N][K/8], scales fp16 bits u16 [K/128][N], zeros u32 [K/128][N/8], s f32 [K])"""
     W = _c(W, np.float32)
     a = _c(act_absmean, np.float32)
     N, K = W.shape
     qw = np.zeros((N, K // 8), np.uint32)
-    sc = np.zeros((N, K // 128), np.uint16)
-    z = np.zeros((N, max(K // 1024, 1)), np.uint32)
+    sc = np.zeros((K // 128, N), np.uint16)
+    z = np.zeros((K // 128, max(N // 8, 1)), np.uint32)
     s = np.zeros(K, np.float32)
     _check(_L().oracle_awq_quantize_g128(_p(W), _p(a), ctypes.c_float(alpha), N, K, _p(qw), _p(sc),
                                          _p(z), _p(s)), "awq_quantize_g128")

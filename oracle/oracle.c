@@ -116,8 +116,8 @@ float oracle_bf16_to_f32(uint16_t h) {
  * Packed format (the interface shared with the CUDA library, restated here):
  *   qweight[n][k/8]  uint32; nibble j (bits 4j..4j+3) holds element k = 8*(k/8) + ORDER[j]
  *                    with ORDER = {0,2,4,6,1,3,5,7};
- *   scales[n][g]     fp16 bits, g = k/128;
- *   zeros[n][g/8]    uint32; nibble j holds the zero point of group 8*(g/8) + j.
+ *   scales[g][n]     fp16 bits, g = k/128 (group-major);
+ *   zeros[g][n/8]    uint32; nibble j holds the zero point of row 8*(n/8) + j in group g.
  * ---------------------------------------------------------------------------------- */
 static const int ORACLE_ORDER[8] = {0, 2, 4, 6, 1, 3, 5, 7};
 
@@ -194,8 +194,12 @@ static int quantize_group(const float* wp, uint16_t* s16_out, uint8_t* z_out, ui
 }
 
 static int check_qshape(int64_t N, int64_t K) {
-    if (N <= 0 || K <= 0 || K % 1024 != 0) return ORACLE_ERR_SHAPE;
+    if (N <= 0 || N % 8 != 0 || K <= 0 || K % 1024 != 0) return ORACLE_ERR_SHAPE;
     return ORACLE_OK;
+}
+
+static int zero_of(const uint32_t* zeros, int64_t N, int64_t n, int64_t g) {
+    return (int)((zeros[g * (N / 8) + n / 8] >> (4 * (n % 8))) & 15u);
 }
 
 /* Quantize W (fp32 [N][K]) with a given per-channel scale s ([K]):
@@ -207,6 +211,8 @@ int oracle_quantize_with_scales(const float* W, const float* s, int64_t N, int64
     if (st) return st;
     const int64_t G = K / GROUP;
     int err = ORACLE_OK;
+    uint8_t* zcode = (uint8_t*)malloc((size_t)(N * G));
+    if (!zcode) return ORACLE_ERR_VALUE;
 #pragma omp parallel for schedule(dynamic, 4)
     for (int64_t n = 0; n < N; ++n) {
         float wp[GROUP];
@@ -221,9 +227,8 @@ int oracle_quantize_with_scales(const float* W, const float* s, int64_t N, int64
                 err = e;
                 continue;
             }
-            scales[n * G + g] = s16;
-            if (g % 8 == 0) zeros[n * (G / 8) + g / 8] = 0;
-            zeros[n * (G / 8) + g / 8] |= (uint32_t)z << (4 * (g % 8));
+            scales[g * N + n] = s16;
+            zcode[n * G + g] = z;
             for (int w = 0; w < GROUP / 8; ++w) {
                 uint32_t word;
                 oracle_pack8(&q[8 * w], &word);
@@ -231,6 +236,14 @@ int oracle_quantize_with_scales(const float* W, const float* s, int64_t N, int64
             }
         }
     }
+    /* zero points packed along n: nibble j of zeros[g][n/8] is row 8*(n/8) + j */
+    for (int64_t g = 0; g < G; ++g)
+        for (int64_t n8 = 0; n8 < N / 8; ++n8) {
+            uint32_t word = 0;
+            for (int j = 0; j < 8; ++j) word |= (uint32_t)(zcode[(n8 * 8 + j) * G + g] & 15u) << (4 * j);
+            zeros[g * (N / 8) + n8] = word;
+        }
+    free(zcode);
     return err;
 }
 
@@ -264,8 +277,8 @@ int oracle_dequant(const uint32_t* qweight, const uint16_t* scales, const uint32
             uint8_t codes[8];
             oracle_unpack8(qweight[n * (K / 8) + k / 8], codes);
             int q = codes[k % 8];
-            int z = (int)((zeros[n * (G / 8) + g / 8] >> (4 * (g % 8))) & 15u);
-            float sf = oracle_f16_to_f32(scales[n * G + g]);
+            int z = zero_of(zeros, N, n, g);
+            float sf = oracle_f16_to_f32(scales[g * N + n]);
             deq[n * K + k] = (float)(q - z) * sf;
         }
     }
@@ -291,19 +304,18 @@ static int check_csr(const int32_t* row_ptr, const int32_t* col_idx, const uint1
 /* One output y[m][n] = sum_k x[m][k] deq[n][k] + sum_{j in row n} x[m][col_j] val_j, summed
  * in double (each product of a bf16 and a dequantized weight or fp16 value is exact in
  * double), plus the sum of the absolute products, which bounds any rounding error. */
-static void one_output(const uint16_t* x, int64_t K, const uint32_t* qweight,
+static void one_output(const uint16_t* x, int64_t K, int64_t N, const uint32_t* qweight,
                        const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
                        const int32_t* col_idx, const uint16_t* values, int64_t m, int64_t n,
                        double* y, double* yabs) {
-    const int64_t G = K / GROUP;
     double acc = 0.0, aacc = 0.0;
     for (int64_t k = 0; k < K; ++k) {
         int64_t g = k / GROUP;
         uint8_t codes[8];
         oracle_unpack8(qweight[n * (K / 8) + k / 8], codes);
         int q = codes[k % 8];
-        int z = (int)((zeros[n * (G / 8) + g / 8] >> (4 * (g % 8))) & 15u);
-        double w = (double)((float)(q - z) * oracle_f16_to_f32(scales[n * G + g]));
+        int z = zero_of(zeros, N, n, g);
+        double w = (double)((float)(q - z) * oracle_f16_to_f32(scales[g * N + n]));
         double p = (double)oracle_bf16_to_f32(x[m * K + k]) * w;
         acc += p;
         aacc += fabs(p);
@@ -336,7 +348,7 @@ int oracle_linear(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweig
 #pragma omp parallel for collapse(2) schedule(dynamic, 16)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n)
-            one_output(x, K, qweight, scales, zeros, row_ptr, col_idx, values, m, n,
+            one_output(x, K, N, qweight, scales, zeros, row_ptr, col_idx, values, m, n,
                        &y[m * N + n], yabs ? &yabs[m * N + n] : NULL);
     return ORACLE_OK;
 }
@@ -357,7 +369,7 @@ int oracle_linear_at(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qw
         if (m_idx[p] < 0 || m_idx[p] >= M || n_idx[p] < 0 || n_idx[p] >= N) return ORACLE_ERR_SHAPE;
 #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t p = 0; p < P; ++p)
-        one_output(x, K, qweight, scales, zeros, row_ptr, col_idx, values, m_idx[p], n_idx[p],
+        one_output(x, K, N, qweight, scales, zeros, row_ptr, col_idx, values, m_idx[p], n_idx[p],
                    &y[p], yabs ? &yabs[p] : NULL);
     return ORACLE_OK;
 }

@@ -47,8 +47,28 @@ def host_bf16_as_f64(y: torch.Tensor) -> np.ndarray:
     return bits.view(np.float32).astype(np.float64)
 
 
-def check_close(y: np.ndarray, ref: np.ndarray, ref_abs: np.ndarray, c_w: float, depth: int, what: str = ""):
-    """y, ref, ref_abs: float64 arrays of the same shape ([M][N] or sampled [P])."""
+# The decode GEMV feeds the MMA the exact biased codes (128 + q) and removes the bias per
+# group in fp32: s * (sum (128+q) x - (128+z) X_g).  Its rounding error is then relative to
+# 143 * sum_k |x_k| s_g, not to sum |x w|: with <= 24 sequential fp32 adds in the MMA chain
+# (2^-23 each, truncating accumulation assumed) and <= 130 in X_g and the correction (2^-24):
+GEMV_XS_COEF = 143.0 * (24 * 2.0 ** -23 + 130 * 2.0 ** -24)
+
+
+def xs_abs(x_bits: np.ndarray, scales: np.ndarray, m_idx=None, n_idx=None) -> np.ndarray:
+    """sum_k |x[m][k]| * scale[n][k // 128] for all (m, n) or at the sampled positions."""
+    x = (x_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    M, K = x.shape
+    xa = np.abs(x).reshape(M, K // 128, 128).sum(-1)              # [M][G]
+    sc = scales.view(np.float16).astype(np.float64).T               # stored [G][N] -> [N][G]
+    if m_idx is None:
+        return xa @ sc.T
+    return np.einsum("pg,pg->p", xa[m_idx], sc[n_idx])
+
+
+def check_close(y: np.ndarray, ref: np.ndarray, ref_abs: np.ndarray, c_w: float, depth: int, what: str = "",
+                xsabs: np.ndarray | None = None):
+    """y, ref, ref_abs: float64 arrays of the same shape ([M][N] or sampled [P]).  xsabs, when
+    given, adds GEMV_XS_COEF * xsabs to the per-element bound (the decode GEMV's arithmetic)."""
     assert y.shape == ref.shape
     assert np.all(np.isfinite(y)), f"{what}: non-finite output"
     err = np.abs(y - ref)
@@ -58,6 +78,8 @@ def check_close(y: np.ndarray, ref: np.ndarray, ref_abs: np.ndarray, c_w: float,
         rel = np.array([err.max() / max(np.abs(ref).max(), 1e-30)])
     assert rel.max() <= NORTH_STAR_REL, f"{what}: max relative error {rel.max():.3e} > {NORTH_STAR_REL}"
     bound = 2.0 ** -8 * np.abs(ref) + (c_w + depth * 2.0 ** -22) * ref_abs + 1e-30
+    if xsabs is not None:
+        bound = bound + GEMV_XS_COEF * xsabs
     bad = err > bound
     assert not bad.any(), (f"{what}: {bad.sum()} outputs beyond the per-element bound; worst "
                            f"err/bound = {(err / bound).max():.3f}")

@@ -122,16 +122,17 @@ def test_pack_rejects_out_of_range_code(orc):
 # ------------------------------------------------------------------ helpers --------------
 
 def unpack_all(qw, sc, z, N, K):
-    """Format definition restated with numpy: codes [N][K], zero [N][G], scale f32 [N][G]."""
+    """Format definition restated with numpy: codes [N][K], zero [N][G], scale f32 [N][G].
+    scales are stored [G][N]; zeros [G][N/8] with nibble j of word n/8 for row 8*(n/8) + j."""
     codes = np.zeros((N, K), np.int64)
     for j in range(8):
         codes[:, ORDER[j]::8] = (qw >> np.uint32(4 * j)) & np.uint32(15)
     G = K // 128
-    zz = np.zeros((N, G), np.int64)
+    zz = np.zeros((G, N), np.int64)
     for j in range(8):
         zz[:, j::8] = (z >> np.uint32(4 * j)) & np.uint32(15)
     s = sc.view(np.float16).astype(np.float32)
-    return codes, zz, s
+    return codes, zz.T.copy(), s.T.copy()
 
 
 def closed_form_group(z0, scale=2.0 ** -6):
@@ -161,20 +162,22 @@ def test_closed_form_golden(orc):
         else:
             W = np.tile(closed_form_group(int(z0)), K // 128)[None, :]
             want_codes = np.arange(K) % 16
+        W = np.repeat(W, 8, axis=0)   # 8 identical rows: one whole word of zero points
         qw, sc, z, s = orc.awq_quantize_g128(W, np.ones(K, np.float32), 0.0)
         assert np.all(s == 1.0)
-        codes, zz, scale = unpack_all(qw, sc, z, 1, K)
+        codes, zz, scale = unpack_all(qw, sc, z, 8, K)
         assert np.all(sc == int(sbits, 16)), name
         assert np.all(zz == int(zero)), name
-        assert np.array_equal(codes[0], want_codes), name
-        deq = orc.dequant(qw, sc, z, 1, K)
+        assert np.all(z == int(zero) * 0x11111111), name   # the zero point in all 8 nibbles
+        assert np.array_equal(codes[0], want_codes) and np.all(codes == codes[0]), name
+        deq = orc.dequant(qw, sc, z, 8, K)
         if name == "Z":
             assert np.all(deq == 0.0)
         else:
             want = W.copy()
             if name == "T":   # the tied weights reconstruct to (q - z) * 2^-6
                 for i, c in enumerate(head):
-                    want[0, i::128] = (int(c) - int(zero)) * 2.0 ** -6
+                    want[:, i::128] = (int(c) - int(zero)) * 2.0 ** -6
             assert np.array_equal(deq, want)  # zero reconstruction error off the ties
 
 
@@ -248,7 +251,7 @@ def test_power_of_two_scales_commute(orc):
     assert np.array_equal(s, np.repeat(2.0 ** j, 128).astype(np.float32))
     qw0, sc0, z0 = orc.quantize_with_scales(W, np.ones(K, np.float32))
     assert np.array_equal(qw, qw0) and np.array_equal(z, z0)
-    want = (sc0.view(np.float16).astype(np.float64) * (2.0 ** j)[None, :]).astype(np.float16)
+    want = (sc0.view(np.float16).astype(np.float64) * (2.0 ** j)[:, None]).astype(np.float16)
     assert np.array_equal(sc, want.view(np.uint16))
 
 
@@ -264,18 +267,21 @@ def test_scale_vector(orc):
 
 def test_value_errors(orc):
     K = 1024
-    W = np.zeros((2, K), np.float32)
+    W = np.zeros((8, K), np.float32)
     W[1, 7] = np.nan
     with pytest.raises(orc.OracleError) as e:
         orc.awq_quantize_g128(W, np.ones(K, np.float32), 0.5)
     assert e.value.code == orc.ERR_VALUE
-    W = np.zeros((2, K), np.float32)
+    W = np.zeros((8, K), np.float32)
     W[0, :64] = 1e6   # (max - min)/15 = 66667 > 65504: the fp16 scale overflows
     with pytest.raises(orc.OracleError) as e:
         orc.awq_quantize_g128(W, np.ones(K, np.float32), 0.5)
     assert e.value.code == orc.ERR_VALUE
     with pytest.raises(orc.OracleError) as e:
-        orc.awq_quantize_g128(np.zeros((2, 1000), np.float32), np.ones(1000, np.float32), 0.5)
+        orc.awq_quantize_g128(np.zeros((8, 1000), np.float32), np.ones(1000, np.float32), 0.5)
+    assert e.value.code == orc.ERR_SHAPE
+    with pytest.raises(orc.OracleError) as e:   # zero points pack 8 rows per word
+        orc.awq_quantize_g128(np.zeros((12, 1024), np.float32), np.ones(1024, np.float32), 0.5)
     assert e.value.code == orc.ERR_SHAPE
     with pytest.raises(orc.OracleError) as e:
         orc.awq_scales(np.array([-1.0], np.float32), 0.5)
@@ -377,14 +383,14 @@ def test_csr_empty_equals_dense_only(orc):
 
 
 def test_csr_validation(orc):
-    N, K = 4, 1024
+    N, K = 8, 1024
     qw, sc, z, _ = orc.awq_quantize_g128(np.zeros((N, K), np.float32), np.ones(K, np.float32), 0.0)
     x = workloads.uniform_bf16(20, (1, K))
-    bad_sorted = (np.array([0, 2, 2, 2, 2], np.int32), np.array([5, 3], np.int32),
+    bad_sorted = (np.array([0, 2] + [2] * 7, np.int32), np.array([5, 3], np.int32),
                   np.array([0x3C00, 0x3C00], np.uint16))
     with pytest.raises(orc.OracleError):
         orc.linear(x, qw, sc, z, N, csr=bad_sorted)
-    bad_col = (np.array([0, 1, 1, 1, 1], np.int32), np.array([K], np.int32), np.array([0], np.uint16))
+    bad_col = (np.array([0] + [1] * 8, np.int32), np.array([K], np.int32), np.array([0], np.uint16))
     with pytest.raises(orc.OracleError):
         orc.linear(x, qw, sc, z, N, csr=bad_col)
 
