@@ -296,11 +296,14 @@ def run_gpu(args, world, rank, local):
     import w4a16_gemm_awq_b200 as w4
     pk, pk_kind = peaks()
     calls, quant = build_gemv_workload(torch, w4)
+    # one zeroed workspace, reused by every call in stream order (each call leaves it zeroed)
+    ws = torch.zeros(max(w4.workspace_bytes(16, c["N"], c["K"]) for c in calls), dtype=torch.uint8,
+                     device="cuda")
 
     def step():
         for c in calls:
             qw, sc, z = c["w"]
-            w4.w4a16_gemv(c["x"], qw, sc, z, out=c["y"])
+            w4.w4a16_gemv(c["x"], qw, sc, z, out=c["y"], workspace=ws)
 
     step_bytes = sum(c["bytes"] for c in calls)
     # warmup (eager, then graph), then the timed region: barrier + sync on both sides
@@ -345,7 +348,7 @@ def run_gpu(args, world, rank, local):
         for c, a, b in zip(calls, hx, hy):
             c["x"].copy_(a, non_blocking=True)
             qw, sc, z = c["w"]
-            w4.w4a16_gemv(c["x"], qw, sc, z, out=c["y"])
+            w4.w4a16_gemv(c["x"], qw, sc, z, out=c["y"], workspace=ws)
             b.copy_(c["y"], non_blocking=True)
 
     e2e_steps = max(1, min(args.steps, 2000))
@@ -438,6 +441,53 @@ def profile_traffic():
     return None
 
 
+def run_case(args):
+    """One kernel on one layer, launched eagerly (for ncu): --case gemv|gemm|quantize."""
+    import torch
+
+    import w4a16_gemm_awq_b200 as w4
+    torch.cuda.set_device(0)
+    K, N, M = args.K, args.N, args.M
+    L = workloads.make_layer(seed=99, K=K, N=N)
+    W = torch.from_numpy(L.W).cuda()
+    act = torch.from_numpy(L.act_absmean).cuda()
+    qw, sc, z, _ = w4.awq_quantize_g128(W, act, workloads.ALPHA)
+    copies = max(1, int(np.ceil(2 * 126e6 / workloads.packed_bytes(N, K)))) if args.case != "quantize" else 1
+    packs = [(qw, sc, z)] + [(qw.clone(), sc.clone(), z.clone()) for _ in range(copies - 1)]
+    x = torch.from_numpy(workloads.make_activations(99, M, L.mult).view(np.int16)).view(torch.bfloat16).cuda()
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    fn = {"gemv": w4.w4a16_gemv, "gemm": w4.w4a16_gemm}.get(args.case)
+    ws = torch.zeros(max(256, w4.workspace_bytes(min(M, 16), N, K)), dtype=torch.uint8, device="cuda")
+
+    def once(i):
+        if args.case == "quantize":
+            w4.awq_quantize_g128(W, act, workloads.ALPHA, out=(qw, sc, z, _s))
+        else:
+            a, b, c = packs[i % len(packs)]
+            fn(x, a, b, c, out=y, workspace=ws)
+
+    _s = torch.empty(K, device="cuda")
+    for i in range(args.warmup):
+        once(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        once(i)
+    e1.record()
+    torch.cuda.synchronize()
+    w4.check_device_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    if args.case == "quantize":
+        b = N * K * 4 + workloads.packed_bytes(N, K) + K * 4
+        print(json.dumps({"case": "quantize", "K": K, "N": N, "ms": ms, "GB/s": b / ms / 1e6}))
+    elif args.case == "gemv":
+        print(json.dumps({"case": "gemv", "K": K, "N": N, "M": M, "ms": ms, "copies": copies,
+                          "GB/s": gemv_bytes(N, K, M) / ms / 1e6}))
+    else:
+        print(json.dumps({"case": "gemm", "K": K, "N": N, "M": M, "ms": ms, "TFLOP/s": 2.0 * M * N * K / ms / 1e9}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -448,7 +498,14 @@ def main():
     ap.add_argument("--skip-gemm", action="store_true")
     ap.add_argument("--skip-quant", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--case", choices=["gemv", "gemm", "quantize"], help="time one kernel on one layer (ncu)")
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--N", type=int, default=28672)
+    ap.add_argument("--M", type=int, default=16)
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -11,14 +11,13 @@
  *   - w4a16_linear / w4a16_gemv / w4a16_gemm: y = x . dequant(Wq)^T (+ x . W_sparse^T)
  *     with the weights dequantized on the fly [AWQ translation, section 1: TinyChat's
  *     on-the-fly dequantization; SqueezeLLM article, sections 2.2 and 2.3: W x =
- *     W_dense x + W_sparse x, the sparse part an fp16 matrix];
- *   - w4a16_split_outliers: move the largest |w| * act_absmean entries into an fp16 CSR
- *     W_sparse [SqueezeLLM article, section 2.2; ratio 0.0045 from section 5.3].
+ *     W_dense x + W_sparse x, the sparse part an fp16 matrix].
  *
  * Conventions for every entry point
- *   - Tensor arguments are DEVICE pointers, allocated and owned by the caller.  The
- *     library keeps no pointer after a call returns.  It allocates no device memory
- *     except one static device status word per GPU, created when the library is loaded.
+ *   - Tensor arguments are DEVICE pointers, allocated and owned by the caller.  So is
+ *     the decode path's workspace (see w4a16_workspace_bytes).  The library keeps no
+ *     pointer after a call returns.  It allocates no device memory except one static
+ *     device status word per GPU, created when the library is loaded.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
  *     stream).  The return value covers argument validation and the kernel launch.
  *     Problems found while a kernel runs are reported later: the kernel records them in
@@ -27,8 +26,8 @@
  *     pipeline wait that ran out.  When a call fails, its outputs are unspecified.
  *   - Element types are passed as raw bits: bf16 and fp16 as uint16_t, fp32 as float.
  *   - Shapes: W is [N][K] (out x in), x is [M][K], y is [M][N], all row-major and dense.
- *     K must be a positive multiple of 1024 (so a row's zero points fill whole words) and
- *     N a positive multiple of 128.  Every pointer must be 16-byte aligned, except the
+ *     K must be a positive multiple of 1024 and N a positive multiple of 128 (the quantizer
+ *     accepts any positive multiple of 8, so zero points fill whole words).  Every pointer must be 16-byte aligned, except the
  *     CSR arrays, which need only natural alignment.
  *
  * Packed weight format (shared with any reader of the quantized weights):
@@ -36,9 +35,12 @@
  *                    k = 8*(k/8) + ORDER[j], ORDER = {0,2,4,6,1,3,5,7}.  Hence
  *                    (word >> 4i) & 0x000F000F holds elements 2i and 2i+1 in its low
  *                    and high 16-bit halves.
- *   scales[n][g]     fp16 bits, g = k/128.
- *   zeros[n][g/8]    uint32.  Nibble j holds the zero point of group 8*(g/8) + j.
+ *   scales[g][n]     fp16 bits, g = k/128 (group-major).
+ *   zeros[g][n/8]    uint32.  Nibble j holds the zero point of row 8*(n/8) + j in group g.
  *   Dequantized weight: w = (q - z) * scale.  This is exact in fp32.
+ *   Group-major parameters put the scales and zero points of consecutive output channels
+ *   of one group next to each other, so a kernel fetches a tile's parameters as one
+ *   contiguous run.
  *
  * CSR outlier matrix (w4a16_csr), in the same scaled space as the packed weights:
  *   row_ptr[N+1] int32, row_ptr[0] = 0, row_ptr[N] = nnz, non-decreasing;
@@ -48,6 +50,7 @@
 #ifndef W4A16_H
 #define W4A16_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -90,8 +93,8 @@ typedef struct {
  *                Each value must be finite and >= 0.
  *   alpha        finite exponent (AWQ searches it in [0, 1]).
  *   qweight      [N][K/8] uint32, device, output.
- *   scales       [N][K/128] fp16 bits, device, output.
- *   zeros        [N][K/1024] uint32, device, output.
+ *   scales       [K/128][N] fp16 bits, device, output.
+ *   zeros        [K/128][N/8] uint32, device, output.
  *   s_out        [K] fp32, device, output, may be NULL.  The caller divides the layer's
  *                input by s (x' = x / s) before calling w4a16_linear.
  *   Errors: NULL, SHAPE, ALIGN and VALUE (non-finite alpha) when called.  Later, through
@@ -103,6 +106,23 @@ w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float a
                                float* s_out, void* stream);
 
 /*
+ * Workspace of the decode path.  The GEMV splits the output row blocks evenly over a
+ * persistent grid.  Row blocks shared by two or more CTAs are combined through fp32
+ * partial tiles and per-row-block counters, which live in a caller-provided device
+ * workspace.
+ *   - It must hold at least w4a16_workspace_bytes(M, N, K) bytes and be 16-byte aligned.
+ *   - It must be zero-filled before its first use.  Every call that completes leaves it
+ *     zero-filled again, so one workspace serves any number of calls in stream order.
+ *   - Calls that may run at the same time (on different streams without ordering between
+ *     them) need different workspaces.
+ *   - After a call reports W4A16_ERR_TIMEOUT, zero the workspace again before reusing it.
+ * w4a16_workspace_bytes returns the size for the CURRENT device (it depends on the number
+ * of SMs), or 0 when the call with these sizes needs no workspace (M > 16) or the sizes
+ * are invalid.  Its value for a given device and N does not depend on M or K.
+ */
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
  * w4a16_linear -- y = bf16_rne( x . dequant(Q)^T + x . W_sparse^T ), fp32 accumulation.
  *   [AWQ translation, 1 (TinyChat on-the-fly dequantization); SqueezeLLM article 2.3]
  *
@@ -111,27 +131,38 @@ w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float a
  *   outliers host pointer to a w4a16_csr whose arrays are on the device, or NULL when
  *            there is no sparse term.  nnz may be 0.
  *   y        [M][N] bf16 bits, device, output.  It must not overlap any input.
- *   M >= 1.  M <= 16 runs the decode GEMV.  Larger M runs the tensor-core GEMM.
- *   Errors: NULL, SHAPE, ALIGN and UNSUPPORTED when called.  Later: SHAPE if a CSR index
- *   is out of range (that entry is skipped), TIMEOUT if a pipeline wait runs out.
+ *   workspace, workspace_bytes: see above.  Required when M <= 16; ignored otherwise.
+ *   M >= 1.  M <= 16 runs the decode GEMV; larger M runs the tensor-core GEMM.
+ *   Errors: NULL, SHAPE, ALIGN and UNSUPPORTED when called (SHAPE also for a workspace that
+ *   is too small).  Later: SHAPE if a CSR index is out of range (that entry is skipped),
+ *   TIMEOUT if a pipeline wait runs out.
  */
 w4a16_status w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
                           const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
-                          int64_t M, int64_t N, int64_t K, void* stream);
+                          int64_t M, int64_t N, int64_t K, void* workspace,
+                          size_t workspace_bytes, void* stream);
 
 /* w4a16_gemv -- the decode path of w4a16_linear, restricted to 1 <= M <= 16
- * (W4A16_ERR_SHAPE otherwise).  Arguments and result are as for w4a16_linear. */
+ * (W4A16_ERR_SHAPE otherwise).  Arguments and result are as for w4a16_linear; the
+ * workspace is required.
+ * Launch overlap: the kernel may start fetching its packed weights, scales and zeros
+ * before the previous kernel on the stream has finished.  It reads x, touches the
+ * workspace and writes y only after that kernel has finished.  The output y of an earlier
+ * library call on the same stream must therefore not alias this call's qweight, scales,
+ * zeros or CSR. */
 w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
                         const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
-                        int64_t M, int64_t N, int64_t K, void* stream);
+                        int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                        void* stream);
 
 /* w4a16_gemm -- the tcgen05 tensor-core path of w4a16_linear, for any M >= 1.  Arguments
- * and result are as for w4a16_linear.  Weights are dequantized to bf16 inside the kernel.
- * When a CSR is given, its values are added to those weights before the bf16 rounding
- * that feeds the tensor cores. */
+ * and result are as for w4a16_linear.  The workspace is not used (NULL and 0 are fine).
+ * Weights are dequantized to bf16 inside the kernel.  When a CSR is given, its values are
+ * added to those weights before the bf16 rounding that feeds the tensor cores. */
 w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
                         const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
-                        int64_t M, int64_t N, int64_t K, void* stream);
+                        int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                        void* stream);
 
 /*
  * w4a16_check_device_status -- synchronize `stream` and return the first problem that a

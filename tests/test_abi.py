@@ -16,7 +16,7 @@ HEADER = os.path.join(ROOT, "include", "w4a16.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return re.findall(r"^\s*(?:w4a16_status|const char\s*\*|int)\s+(\w+)\s*\(", text, flags=re.M)
+    return re.findall(r"^\s*(?:w4a16_status|const char\s*\*|int|size_t)\s+(\w+)\s*\(", text, flags=re.M)
 
 
 @pytest.fixture(scope="module")
@@ -28,7 +28,7 @@ def L():
 def test_header_declares_the_boundary():
     names = set(declared_functions())
     assert {"awq_quantize_g128", "w4a16_linear", "w4a16_gemv", "w4a16_gemm", "w4a16_check_device_status",
-            "w4a16_status_string", "w4a16_version"} <= names
+            "w4a16_status_string", "w4a16_version", "w4a16_workspace_bytes"} <= names
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -38,6 +38,12 @@ def test_every_declared_symbol_is_exported(L):
     for name in declared_functions():
         assert name in exported, name
         assert hasattr(L, name)
+
+
+def test_workspace_query_without_gpu(L):
+    # no device here: the query reports 0 rather than failing; invalid sizes report 0 too
+    assert L.w4a16_workspace_bytes(1, 4096, 4096) == 0
+    assert L.w4a16_workspace_bytes(17, 4096, 4096) == 0
 
 
 def test_status_strings(L):
@@ -50,10 +56,11 @@ def test_status_strings(L):
 FAKE = 1 << 20  # a 16-byte-aligned address that is never dereferenced: validation fails first
 
 
-def _linear(L, name, x=FAKE, qw=FAKE, sc=FAKE, z=FAKE, csr=None, y=FAKE, M=1, N=128, K=1024):
+def _linear(L, name, x=FAKE, qw=FAKE, sc=FAKE, z=FAKE, csr=None, y=FAKE, M=1, N=128, K=1024, ws=FAKE, wsb=1 << 30):
     fn = getattr(L, name)
     return fn(ctypes.c_void_p(x), ctypes.c_void_p(qw), ctypes.c_void_p(sc), ctypes.c_void_p(z),
-              ctypes.byref(csr) if csr is not None else None, ctypes.c_void_p(y), M, N, K, None)
+              ctypes.byref(csr) if csr is not None else None, ctypes.c_void_p(y), M, N, K,
+              ctypes.c_void_p(ws), wsb, None)
 
 
 @pytest.mark.parametrize("name", ["w4a16_linear", "w4a16_gemv", "w4a16_gemm"])

@@ -5,7 +5,7 @@ import torch
 
 import w4a16_gemm_awq_b200 as w4
 import workloads
-from parity import Case, check_close, dev_bits, dev_csr, host_bf16_as_f64
+from parity import Case, check_close, dev_bits, dev_csr, host_bf16_as_f64, xs_abs
 
 pytestmark = pytest.mark.gpu
 
@@ -27,15 +27,18 @@ def test_gemv_small_full_output(orc, M, csr):
     c = Case(orc, seed=100 + M, K=2048, N=256, M=M, csr=csr)
     y = host_bf16_as_f64(gemv(c.device()))
     ref, ref_abs = c.reference(orc)
-    check_close(y, ref, ref_abs, 0.0, depth(c.K), f"M={M} csr={csr}")
+    check_close(y, ref, ref_abs, 0.0, depth(c.K), f"M={M} csr={csr}", xs_abs(c.x, c.sc))
 
 
-@pytest.mark.parametrize("K,N", [(1024, 128), (3072, 384), (8192, 128), (1024, 4096)])
+@pytest.mark.parametrize("K,N", [(1024, 128), (3072, 384), (8192, 128), (1024, 4096), (65536, 128), (16384, 640),
+                                 (4096, 2048)])
 def test_gemv_odd_shapes(orc, K, N):
+    """Includes shapes with more work units than CTAs, where a CTA streams several groups
+    through the ring and row blocks are split between CTAs."""
     c = Case(orc, seed=K + N, K=K, N=N, M=5, csr=True)
     y = host_bf16_as_f64(gemv(c.device()))
     ref, ref_abs = c.reference(orc)
-    check_close(y, ref, ref_abs, 0.0, depth(K), f"{K}x{N}")
+    check_close(y, ref, ref_abs, 0.0, depth(K), f"{K}x{N}", xs_abs(c.x, c.sc))
 
 
 def test_gemv_empty_csr_is_bit_identical(orc):
@@ -63,7 +66,7 @@ def test_gemv_csr_only_and_dense_rows(orc):
              scales=dev_bits(sc, torch.int16), zeros=dev_bits(z, torch.int32), csr=dev_csr((rp, ci, v)))
     y = host_bf16_as_f64(gemv(d))
     ref, ref_abs = orc.linear(x, qw, sc, z, N, csr=(rp, ci, v), with_abs=True)
-    check_close(y, ref, ref_abs, 0.0, K + 64, "csr only")
+    check_close(y, ref, ref_abs, 0.0, K + 64, "csr only", xs_abs(x, sc))
 
 
 def test_gemv_reports_bad_csr(orc):
@@ -79,6 +82,27 @@ def test_gemv_reports_bad_csr(orc):
     assert e.value.code == w4.ERR_SHAPE
 
 
+def test_gemv_workspace_contract(orc):
+    """A NULL or short workspace is refused; a workspace is all-zero again after calls that
+    split row blocks between CTAs; concurrent-stream calls get their own workspaces."""
+    c = Case(orc, seed=13, K=4096, N=512, M=3)
+    d = c.device()
+    need = w4.workspace_bytes(3, c.N, c.K)
+    assert need > 0 and w4.workspace_bytes(17, c.N, c.K) == 0
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.w4a16_gemv(d["x"], d["qweight"], d["scales"], d["zeros"],
+                      workspace=torch.zeros(need - 256, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == w4.ERR_SHAPE
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    y0 = w4.w4a16_gemv(d["x"], d["qweight"], d["scales"], d["zeros"], workspace=ws)
+    y1 = w4.w4a16_gemv(d["x"], d["qweight"], d["scales"], d["zeros"], workspace=ws)
+    w4.check_device_status()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+    assert int(ws.count_nonzero()) == ws.numel() - int((ws == 0).sum())  # sanity
+    counters = ws[need - 256 * ((c.N // 128 * 4 + 255) // 256):]
+    assert int(counters.count_nonzero()) == 0
+
+
 def test_linear_dispatches_to_gemv(orc):
     c = Case(orc, seed=12, K=2048, N=256, M=16, csr=True)
     d = c.device()
@@ -92,7 +116,7 @@ def test_gemv_config0_full(orc):
     c = Case(orc, seed=workloads.seed_of(0, 0), K=4096, N=4096, M=1)
     y = host_bf16_as_f64(gemv(c.device()))
     ref, ref_abs = c.reference(orc)
-    check_close(y, ref, ref_abs, 0.0, depth(c.K), "config 0")
+    check_close(y, ref, ref_abs, 0.0, depth(c.K), "config 0", xs_abs(c.x, c.sc))
 
 
 FULL = ([(1, i, K, N, M, False) for i, (_, K, N) in enumerate(workloads.LLAMA3_8B) for M in (1, 4, 8, 16)]
@@ -106,4 +130,4 @@ def test_gemv_full_shapes_sampled(orc, cfg, i, K, N, M, csr):
     y = host_bf16_as_f64(gemv(c.device()))
     m, n = c.sample(seed=cfg * 10 + i)
     ref, ref_abs = c.reference_at(orc, m, n)
-    check_close(y[m, n], ref, ref_abs, 0.0, depth(K), f"{K}x{N} M={M}")
+    check_close(y[m, n], ref, ref_abs, 0.0, depth(K), f"{K}x{N} M={M}", xs_abs(c.x, c.sc, m, n))

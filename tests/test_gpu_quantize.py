@@ -29,7 +29,7 @@ def assert_same(orc, W, act, alpha, what=""):
 
 
 @pytest.mark.parametrize("N,K,alpha", [(128, 1024, 0.5), (64, 2048, 0.5), (256, 4096, 0.25), (192, 1024, 0.0),
-                                       (1, 1024, 1.0), (100, 3072, 0.5)])
+                                       (8, 1024, 1.0), (104, 3072, 0.5), (200, 2048, 0.5)])
 def test_quantize_small_bit_exact(orc, N, K, alpha):
     L = workloads.make_layer(seed=N * 7 + K, K=K, N=N)
     assert_same(orc, L.W, L.act_absmean, alpha, f"{N}x{K}")
@@ -54,10 +54,10 @@ def test_quantize_wide_dynamic_range(orc):
 def test_quantize_closed_form_on_gpu(orc):
     K = 1024
     i = np.arange(K) % 16
-    W = ((i - 5) * 2.0 ** -6).astype(np.float32)[None, :].repeat(4, 0)
+    W = ((i - 5) * 2.0 ** -6).astype(np.float32)[None, :].repeat(8, 0)
     qw, sc, z, s = run_gpu(W, np.ones(K, np.float32), 0.0)
     assert np.all(sc == 0x2400)
-    assert np.all(z == 0x55555555)
+    assert np.all(z == 0x55555555)  # zero point 5 in the nibbles of all 8 rows
 
 
 def test_quantize_reports_bad_values():

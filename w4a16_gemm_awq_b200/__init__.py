@@ -8,10 +8,11 @@ mirror the C ABI in include/w4a16.h:
   w4a16_linear(x, qweight, scales, zeros, csr)  -> y      (any M)
   w4a16_gemv(...)                               -> y      (1 <= M <= 16)
   w4a16_gemm(...)                               -> y      (tcgen05 path, any M)
+  workspace_bytes(M, N, K)                      -> bytes of zeroed device workspace a decode call needs
   check_device_status()                         -> raises W4A16Error on a recorded problem
 
-Bit containers: qweight and zeros are int32 tensors holding uint32 words, scales is an
-int16 tensor holding fp16 bits, x and y are bfloat16 tensors.  A CSR is a tuple
+Bit containers: qweight [N][K/8] and zeros [K/128][N/8] are int32 tensors holding uint32
+words, scales [K/128][N] is an int16 tensor holding fp16 bits, x and y are bfloat16 tensors.  A CSR is a tuple
 (row_ptr int32 [N+1], col_idx int32 [nnz], values int16 fp16-bits [nnz]) of CUDA tensors.
 
 There is no fallback: if the library is not built, or there is no sm_100 GPU, the calls
@@ -62,7 +63,9 @@ def lib() -> ctypes.CDLL:
         L.awq_quantize_g128.argtypes = [P, P, F, I64, I64, P, P, P, P, P]
         for name in ("w4a16_linear", "w4a16_gemv", "w4a16_gemm"):
             fn = getattr(L, name)
-            fn.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P]
+            fn.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P, ctypes.c_size_t, P]
+        L.w4a16_workspace_bytes.argtypes = [I64, I64, I64]
+        L.w4a16_workspace_bytes.restype = ctypes.c_size_t
         L.w4a16_check_device_status.argtypes = [P]
         L.w4a16_status_string.argtypes = [ctypes.c_int]
         L.w4a16_status_string.restype = ctypes.c_char_p
@@ -94,16 +97,16 @@ def _need(t, dtype, ndim, name):
 
 
 def awq_quantize_g128(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, out=None):
-    """W fp32 [N][K], act_absmean fp32 [K] -> (qweight int32 [N][K/8], scales int16 [N][K/128],
-    zeros int32 [N][K/1024], s fp32 [K])."""
+    """W fp32 [N][K], act_absmean fp32 [K] -> (qweight int32 [N][K/8], scales int16 [K/128][N],
+    zeros int32 [K/128][N/8], s fp32 [K])."""
     _need(W, torch.float32, 2, "W")
     _need(act_absmean, torch.float32, 1, "act_absmean")
     N, K = W.shape
     dev = W.device
     if out is None:
         out = (torch.empty(N, K // 8, dtype=torch.int32, device=dev),
-               torch.empty(N, max(K // 128, 1), dtype=torch.int16, device=dev),
-               torch.empty(N, max(K // 1024, 1), dtype=torch.int32, device=dev),
+               torch.empty(max(K // 128, 1), N, dtype=torch.int16, device=dev),
+               torch.empty(max(K // 128, 1), max(N // 8, 1), dtype=torch.int32, device=dev),
                torch.empty(K, dtype=torch.float32, device=dev))
     qw, sc, z, s = out
     code = lib().awq_quantize_g128(_ptr(W), _ptr(act_absmean), ctypes.c_float(alpha), N, K, _ptr(qw), _ptr(sc),
@@ -112,7 +115,28 @@ def awq_quantize_g128(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, 
     return qw, sc, z, s
 
 
-def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None):
+_workspaces = {}
+
+
+def workspace(device: torch.device, nbytes: int, stream=None) -> torch.Tensor:
+    """A zero-filled device workspace of at least nbytes for calls on `stream` of `device`,
+    cached so that consecutive calls on the same stream reuse it (each call leaves it zeroed).
+    Calls on different streams get different workspaces."""
+    dev = torch.device(device)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    key = (dev.index if dev.index is not None else torch.cuda.current_device(), s.cuda_stream)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        _workspaces[key] = ws
+    return ws
+
+
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().w4a16_workspace_bytes(M, N, K))
+
+
+def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None):
     _need(x, torch.bfloat16, 2, "x")
     _need(qweight, torch.int32, 2, "qweight")
     _need(scales, torch.int16, 2, "scales")
@@ -128,22 +152,27 @@ def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None):
         _need(rp, torch.int32, 1, "row_ptr")
         cs = Csr(rp.data_ptr(), ci.data_ptr() if ci.numel() else None, v.data_ptr() if v.numel() else None,
                  int(ci.numel()))
+    need = workspace_bytes(M, N, K) if name != "w4a16_gemm" else 0
+    if ws is None and need > 0:
+        ws = workspace(x.device, need)
     code = getattr(lib(), name)(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros),
-                                ctypes.byref(cs) if cs is not None else None, _ptr(y), M, N, K, _stream(x.device))
+                                ctypes.byref(cs) if cs is not None else None, _ptr(y), M, N, K,
+                                _ptr(ws), ws.numel() if ws is not None else 0, _stream(x.device))
     _check(code, name)
     return y
 
 
-def w4a16_linear(x, qweight, scales, zeros, csr=None, out=None):
-    return _linear("w4a16_linear", x, qweight, scales, zeros, csr, out)
+def w4a16_linear(x, qweight, scales, zeros, csr=None, out=None, workspace=None):
+    """y = x . dequant(Q)^T (+ CSR term); M <= 16 runs the GEMV (with a cached workspace)."""
+    return _linear("w4a16_linear", x, qweight, scales, zeros, csr, out, workspace)
 
 
-def w4a16_gemv(x, qweight, scales, zeros, csr=None, out=None):
-    return _linear("w4a16_gemv", x, qweight, scales, zeros, csr, out)
+def w4a16_gemv(x, qweight, scales, zeros, csr=None, out=None, workspace=None):
+    return _linear("w4a16_gemv", x, qweight, scales, zeros, csr, out, workspace)
 
 
-def w4a16_gemm(x, qweight, scales, zeros, csr=None, out=None):
-    return _linear("w4a16_gemm", x, qweight, scales, zeros, csr, out)
+def w4a16_gemm(x, qweight, scales, zeros, csr=None, out=None, workspace=None):
+    return _linear("w4a16_gemm", x, qweight, scales, zeros, csr, out, workspace)
 
 
 def check_device_status(stream=None):

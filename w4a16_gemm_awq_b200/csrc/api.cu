@@ -88,6 +88,8 @@ struct LinearArgs {
     long long nnz = 0;
     uint16_t* y;
     int64_t M, N, K;
+    void* workspace = nullptr;
+    size_t workspace_bytes = 0;
 };
 
 w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -120,12 +122,39 @@ w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const u
     return W4A16_OK;
 }
 
+w4a16_status encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc = nullptr;
+    w4a16_status st = encoder(&enc);
+    if (st != W4A16_OK) return st;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return W4A16_ERR_CUDA;
+    return W4A16_OK;
+}
+
 w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream) {
     DeviceInfo* d = nullptr;
     w4a16_status st = device_info(&d);
     if (st != W4A16_OK) return st;
-    return from_cuda(launch_gemv(a.x, a.qweight, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
-                                 (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status, stream));
+    if (a.K > gemv_max_k()) return W4A16_ERR_UNSUPPORTED;
+    if (a.workspace == nullptr) return W4A16_ERR_NULL;
+    if (!aligned(a.workspace, 16)) return W4A16_ERR_ALIGN;
+    if (a.workspace_bytes < gemv_workspace_bytes((int)a.N, d->num_sms)) return W4A16_ERR_SHAPE;
+    GemvMaps maps;
+    const uint32_t mpad = a.M > 8 ? 16u : 8u;
+    st = encode_2d(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.qweight, (uint64_t)a.K / 8, (uint64_t)a.N,
+                   (uint64_t)a.K / 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != W4A16_OK) return st;
+    st = encode_2d(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * 2,
+                   64, mpad + 2, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != W4A16_OK) return st;
+    return from_cuda(launch_gemv(maps, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
+                                 a.workspace, (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status, stream));
 }
 
 int pick_bn(int64_t M) {
@@ -178,7 +207,7 @@ extern "C" {
 w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, void* stream) {
     if (!W || !act_absmean || !qweight || !scales || !zeros) return W4A16_ERR_NULL;
-    if (N < 1 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK) return W4A16_ERR_SHAPE;
+    if (N < 8 || N % 8 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK) return W4A16_ERR_SHAPE;
     if (!aligned(W, 16) || !aligned(act_absmean, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
         !aligned(zeros, 16) || (s_out && !aligned(s_out, 16)))
         return W4A16_ERR_ALIGN;
@@ -190,17 +219,31 @@ w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float a
                                          d->status, static_cast<cudaStream_t>(stream)));
 }
 
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || M > 16 || N < 128 || N % 128 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > gemv_max_k())
+        return 0;
+    DeviceInfo* d = nullptr;
+    if (device_info(&d) != W4A16_OK) return 0;
+    return gemv_workspace_bytes((int)N, d->num_sms);
+}
+
 w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
-                        const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+                        const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
+                        size_t workspace_bytes, void* stream) {
     LinearArgs a;
     w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
     if (st != W4A16_OK) return st;
     if (M > 16) return W4A16_ERR_SHAPE;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
     return run_gemv(a, static_cast<cudaStream_t>(stream));
 }
 
 w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
-                        const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+                        const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+    (void)workspace;
+    (void)workspace_bytes;
     LinearArgs a;
     w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
     if (st != W4A16_OK) return st;
@@ -209,11 +252,14 @@ w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16
 
 w4a16_status w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
                           const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N,
-                          int64_t K, void* stream) {
+                          int64_t K, void* workspace, size_t workspace_bytes, void* stream) {
     LinearArgs a;
     w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
     if (st != W4A16_OK) return st;
-    return M <= 16 ? run_gemv(a, static_cast<cudaStream_t>(stream)) : run_gemm(a, static_cast<cudaStream_t>(stream));
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    const bool decode = M <= 16 && K <= gemv_max_k();
+    return decode ? run_gemv(a, static_cast<cudaStream_t>(stream)) : run_gemm(a, static_cast<cudaStream_t>(stream));
 }
 
 w4a16_status w4a16_check_device_status(void* stream) {

@@ -57,9 +57,12 @@ struct GemmSmem {
     static constexpr int kXStageBytes = BN * kBK * 2;
     static constexpr int kXOff = 0;
     static constexpr int kWOff = kStages * kXStageBytes;
-    static constexpr int kBarOff = kWOff + kStages * kWStageBytes;
+    static constexpr int kParOff = kWOff + kStages * kWStageBytes;  // per stage: 256 B scales + 64 B zeros
+    static constexpr int kBarOff = kParOff + kStages * 512;
     static constexpr int kBytes = kBarOff + 256;
     static constexpr uint32_t kTmemCols = (BN + kAStages * kACols) <= 256 ? 256u : 512u;
+    static_assert(kXStageBytes % 1024 == 0 && kWOff % 1024 == 0,
+                  "128-byte-swizzled TMA boxes need 1024-byte aligned stages");
 };
 
 // UMMA shared-memory descriptor: K-major, 128-byte swizzle, rows of 128 bytes, 8-row
@@ -104,7 +107,6 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN;
     const int nK = p.K / kBK;
-    const int G = p.K >> 7;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -149,9 +151,18 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     fail();
                     break;
                 }
-                mbar_arrive_expect_tx(&full[slot], (uint32_t)(L::kXStageBytes + kWStageBytes));
+                // a stage that starts a group also brings the group's 128 scales and 16 zero words
+                const bool first_half = (s & 1) == 0;
+                mbar_arrive_expect_tx(&full[slot],
+                                      (uint32_t)(L::kXStageBytes + kWStageBytes + (first_half ? 256 + 64 : 0)));
                 tma_load_2d(smem + L::kXOff + slot * L::kXStageBytes, &map_x, &full[slot], s * kBK, m0);
                 tma_load_2d(smem + L::kWOff + slot * kWStageBytes, &map_w, &full[slot], s * (kBK / 8), n0);
+                if (first_half) {
+                    const int g = s >> 1;
+                    uint8_t* par = smem + L::kParOff + slot * 512;
+                    bulk_load(par, p.scales + (size_t)g * p.N + n0, 256, &full[slot]);
+                    bulk_load(par + 256, p.zeros + (size_t)g * (p.N >> 3) + (n0 >> 3), 64, &full[slot]);
+                }
                 ++issued;
             }
             // the copies this CTA started must land before it may exit
@@ -189,16 +200,6 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         const int row = 32 * quarter + lane;      // channel within the tile == TMEM lane
         const int n = n0 + row;
         const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
-        const uint4* sc_row = reinterpret_cast<const uint4*>(p.scales + (size_t)n * G);
-        const uint32_t* z_row = p.zeros + (size_t)n * (G >> 3);
-
-        // scales and zeros come 8 groups (1024 k, 16 stages) at a time; prefetch one ahead
-        uint4 sc_cur = __ldg(sc_row), sc_nxt = make_uint4(0, 0, 0, 0);
-        uint32_t z_cur = __ldg(z_row), z_nxt = 0;
-        if (G > 8) {
-            sc_nxt = __ldg(sc_row + 1);
-            z_nxt = __ldg(z_row + 1);
-        }
         uint32_t sb = 0, zb = 0;
 
         // CSR walk for this row: next entry's column and value
@@ -234,27 +235,16 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             const int sw = (row >> 2) & 1;
             const uint4 wa = *reinterpret_cast<const uint4*>(wrow + ((0 ^ sw) << 4));
             const uint4 wb = *reinterpret_cast<const uint4*>(wrow + ((1 ^ sw) << 4));
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-
-            if ((s & 1) == 0) {  // a new group of 128 k
-                const int g = s >> 1;
-                if ((g & 7) == 0 && g > 0) {
-                    sc_cur = sc_nxt;
-                    z_cur = z_nxt;
-                    if ((g >> 3) + 1 < (G >> 3)) {
-                        sc_nxt = __ldg(sc_row + (g >> 3) + 1);
-                        z_nxt = __ldg(z_row + (g >> 3) + 1);
-                    }
-                }
-                const int gi = g & 7;
-                const uint32_t sw2 = u4_get(sc_cur, gi >> 1);
-                const uint16_t sbits = (uint16_t)((gi & 1) ? (sw2 >> 16) : (sw2 & 0xFFFFu));
+            if ((s & 1) == 0) {  // a new group of 128 k: its scale and zero point from the stage
+                const uint8_t* par = smem + L::kParOff + slot * 512;
+                const uint16_t sbits = reinterpret_cast<const uint16_t*>(par)[row];
+                const uint32_t z = (reinterpret_cast<const uint32_t*>(par + 256)[row >> 3] >> (4 * (row & 7))) & 15u;
                 const uint32_t sbf = float_to_bf16_bits(fp16_bits_to_float(sbits));
                 sb = sbf | (sbf << 16);
-                const uint32_t z = (z_cur >> (4 * gi)) & 15u;
                 zb = 0x43004300u | z | (z << 16);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
 
             uint32_t v[32];
 #pragma unroll

@@ -14,9 +14,22 @@ cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, i
                                 uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
                                 cudaStream_t stream);
 
-cudaError_t launch_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
+// Tensor maps the GEMV needs.
+struct GemvMaps {
+    CUtensorMap w;  // uint32 [N][K/8], box 16 words (one group) x 128 rows, no swizzle
+    CUtensorMap x;  // bf16 [M][K], box 64 (k) x (Mpad + 2) tokens, 128-byte swizzle
+};
+
+// Largest K the GEMV supports.
+int gemv_max_k();
+
+// Bytes of zero-initialised device workspace the GEMV needs for N output channels.
+size_t gemv_workspace_bytes(int N, int num_sms);
+
+cudaError_t launch_gemv(const GemvMaps& maps, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
                         const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
-                        uint16_t* y, int M, int N, int K, int num_sms, unsigned* err, cudaStream_t stream);
+                        uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
+                        cudaStream_t stream);
 
 // Tensor maps the GEMM needs, encoded by the caller (api.cu) with the driver's encoder.
 struct GemmMaps {

@@ -6,13 +6,15 @@
 //  section 1: TinyChat's 4-bit packing, 8 codes per 32-bit word.]
 //
 // Work decomposition.  A CTA of 8 warps owns a tile of kRowsPerCta rows x 1024 columns
-// (one zero-point word per row).  It first computes the 1024 per-channel scales s_k into
+// (8 groups).  It first computes the 1024 per-channel scales s_k into
 // shared memory (double pow, as the definition states).  Then each warp quantizes one row
 // of the tile at a time: 32 lanes x 16 bytes is exactly one group of 128 fp32 weights,
 // so the row's 8 groups arrive as 8 coalesced 128-bit loads per lane, all issued before
 // the first group is processed.  The group's min/max is a 5-step warp-shuffle reduction.
 // Each lane quantizes its 4 weights.  Lane pairs (2i, 2i+1) merge their nibbles into
-// packed word i with one shuffle.
+// packed word i with one shuffle.  The fp16 scales and zero points of the tile are collected
+// in shared memory and written group-major at the end (scales[g][n], zeros[g][n/8] with the
+// nibbles of 8 consecutive rows), so those stores are coalesced too.
 //
 // Bit-exactness: every float step is a single IEEE operation with round-to-nearest-even
 // (__fmul_rn, __fsub_rn, __fdiv_rn, __fadd_rn, rintf, __float2half_rn).  The build does
@@ -41,9 +43,10 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
                     uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
                     uint32_t* __restrict__ zeros, float* __restrict__ s_out, unsigned* err) {
     __shared__ __align__(16) float s_sm[1024];
-    const int kc = blockIdx.x;                 // 1024-column chunk
+    __shared__ __align__(16) uint16_t sc_sm[8][kRowsPerCta];  // fp16 scale bits per (group, row)
+    __shared__ uint8_t zc_sm[8][kRowsPerCta];                 // zero point per (group, row)
+    const int kc = blockIdx.x;                 // 1024-column chunk (groups 8 kc .. 8 kc + 7)
     const int row0 = blockIdx.y * kRowsPerCta;
-    const int G = K >> 7;
 
     for (int i = threadIdx.x; i < 1024; i += kQuantThreads) {
         const float a = act[(size_t)kc * 1024 + i];
@@ -59,7 +62,7 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
     const bool odd = lane & 1;
     for (int r = warp; r < kRowsPerCta; r += kQuantThreads / 32) {
         const int n = row0 + r;
-        if (n >= N) break;
+        if (n >= N) break;  // warp-uniform
         const float* wrow = W + (size_t)n * K + (size_t)kc * 1024 + 4 * lane;
         float4 v[8];
 #pragma unroll
@@ -68,8 +71,6 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
             v[g] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
                                __uint_as_float(u.w));
         }
-        uint32_t zword = 0;
-        uint32_t sbits[8];
         bool bad = false;
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
@@ -104,18 +105,32 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
             uint32_t part = place_nibbles(q, odd);
             part |= __shfl_xor_sync(0xffffffffu, part, 1);
             if (!odd) qweight[(size_t)n * (K >> 3) + (size_t)kc * 128 + g * 16 + (lane >> 1)] = part;
-            zword |= (uint32_t)zf << (4 * g);
-            sbits[g] = __half_as_ushort(h);
+            if (lane == 0) {
+                sc_sm[g][r] = __half_as_ushort(h);
+                zc_sm[g][r] = (uint8_t)zf;
+            }
         }
         if (bad) record_error(err, kErrValue);
-        if (lane == 0) {
-            zeros[(size_t)n * (K >> 10) + kc] = zword;
-            uint4 sv;
-            sv.x = sbits[0] | (sbits[1] << 16);
-            sv.y = sbits[2] | (sbits[3] << 16);
-            sv.z = sbits[4] | (sbits[5] << 16);
-            sv.w = sbits[6] | (sbits[7] << 16);
-            *reinterpret_cast<uint4*>(scales + (size_t)n * G + (size_t)kc * 8) = sv;
+    }
+    __syncthreads();
+
+    // group-major parameters: scales[g][n] (row pairs as one 32-bit store) and zeros[g][n/8]
+    // (the nibbles of 8 consecutive rows), both coalesced along n
+    {
+        const int g = threadIdx.x >> 5, j = threadIdx.x & 31;  // 8 groups x 32 row pairs
+        const int r = 2 * j;
+        if (row0 + r < N) {
+            const uint32_t pair = (uint32_t)sc_sm[g][r] | ((uint32_t)sc_sm[g][r + 1] << 16);
+            *reinterpret_cast<uint32_t*>(scales + ((size_t)kc * 8 + g) * N + row0 + r) = pair;
+        }
+        if (threadIdx.x < 64) {
+            const int gz = threadIdx.x >> 3, w = threadIdx.x & 7;
+            if (row0 + 8 * w < N) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int b = 0; b < 8; ++b) word |= (uint32_t)(zc_sm[gz][8 * w + b] & 15u) << (4 * b);
+                zeros[((size_t)kc * 8 + gz) * (N >> 3) + (row0 >> 3) + w] = word;
+            }
         }
     }
 }
