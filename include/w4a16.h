@@ -165,6 +165,30 @@ w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16
                         void* stream);
 
 /*
+ * w4a16_gemv_noalloc -- the decode GEMV of w4a16_gemv without a caller workspace.  The
+ * paper has no counterpart; this entry point exists for callers that cannot allocate
+ * device memory around the call.  Examples are a plugin of an inference engine that is
+ * handed only its input and output buffers (the engine plans all memory ahead and forbids
+ * allocations while it executes), and code that runs inside an allocator or memory-pool
+ * callback, where calling cudaMalloc would re-enter the allocator.
+ *   - Arguments, result and limits are those of w4a16_gemv, minus the workspace.
+ *     N <= 131072 and at most 160 SMs on the device; otherwise W4A16_ERR_UNSUPPORTED.
+ *   - Its scratch is a static device array of about 5 MiB inside the library.  Every GPU
+ *     that loads the library holds one until the process exits.  The call allocates
+ *     nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress).  Make that first call before any stream capture.
+ *   - Each call clears the scratch's counters with cudaMemsetAsync on `stream`, and then
+ *     runs the GEMV.
+ *   - All calls on a device share the one array, which keeps the last call's contents.
+ *     Calls that overlap on the GPU (different streams without ordering) race on it and
+ *     give wrong results.
+ */
+w4a16_status w4a16_gemv_noalloc(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                                const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
+                                int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
  * w4a16_check_device_status -- synchronize `stream` and return the first problem that a
  * kernel recorded since the last call, or W4A16_OK.  This clears the record.  The record
  * is per device and shared by all streams of that device.

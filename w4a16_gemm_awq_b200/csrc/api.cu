@@ -17,6 +17,16 @@ namespace w4a16 {
 // Problems found by kernels while they run (bit set of kErrValue / kErrShape / kErrTimeout).
 __device__ unsigned g_device_status;
 
+// Scratch of w4a16_gemv_noalloc: the decode GEMV's workspace (fp32 partial tiles, then the
+// per-row-block counters) for devices with up to kNoallocMaxSms SMs and N up to
+// kNoallocMaxN.  It is part of the loaded module: every GPU that loads the library holds
+// it until the process exits, and every call of w4a16_gemv_noalloc on that GPU uses it.
+constexpr int kNoallocMaxSms = 160;
+constexpr int kNoallocMaxN = 131072;
+constexpr size_t kNoallocScratchBytes =
+    (size_t)2 * 2 * kNoallocMaxSms * 128 * 16 * sizeof(float) + (size_t)(kNoallocMaxN / 128) * sizeof(unsigned);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -57,6 +67,24 @@ w4a16_status device_info(DeviceInfo** out) {
     }
     *out = &d;
     return d.sm100 ? W4A16_OK : W4A16_ERR_UNSUPPORTED;
+}
+
+// Device address of g_noalloc_scratch for the current device.  In host code the array's
+// name only stands in for the symbol; the address comes from cudaGetSymbolAddress, taken
+// once per device with that device current.
+w4a16_status noalloc_scratch(void** out) {
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return W4A16_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return W4A16_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return W4A16_OK;
 }
 
 w4a16_status encoder(EncodeTiledFn* out) {
@@ -260,6 +288,35 @@ w4a16_status w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint
     a.workspace_bytes = workspace_bytes;
     const bool decode = M <= 16 && K <= gemv_max_k();
     return decode ? run_gemv(a, static_cast<cudaStream_t>(stream)) : run_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
+w4a16_status w4a16_gemv_noalloc(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                                const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y, int64_t M,
+                                int64_t N, int64_t K, void* stream) {
+    LinearArgs a;
+    w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
+    if (st != W4A16_OK) return st;
+    if (M > 16) return W4A16_ERR_SHAPE;
+    if (N > kNoallocMaxN) return W4A16_ERR_UNSUPPORTED;
+    DeviceInfo* d = nullptr;
+    st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    if (d->num_sms > kNoallocMaxSms) return W4A16_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != W4A16_OK) return st;
+    const size_t need = gemv_workspace_bytes((int)N, d->num_sms);
+    if (need > kNoallocScratchBytes) return W4A16_ERR_UNSUPPORTED;
+    // The row-block counters sit at the end of the workspace and must start at zero.  A
+    // completed call leaves them zero, but one that failed may not have, so clear them.
+    const size_t counter_bytes = (((size_t)(N / 128) * sizeof(unsigned)) + 255) / 256 * 256;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + (need - counter_bytes), 0, counter_bytes, s) !=
+        cudaSuccess)
+        return W4A16_ERR_CUDA;
+    a.workspace = scratch;
+    a.workspace_bytes = kNoallocScratchBytes;
+    return run_gemv(a, s);
 }
 
 w4a16_status w4a16_check_device_status(void* stream) {
