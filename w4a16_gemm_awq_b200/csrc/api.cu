@@ -150,20 +150,6 @@ w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const u
     return W4A16_OK;
 }
 
-w4a16_status encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
-                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
-    EncodeTiledFn enc = nullptr;
-    w4a16_status st = encoder(&enc);
-    if (st != W4A16_OK) return st;
-    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
-    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    if (enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return W4A16_ERR_CUDA;
-    return W4A16_OK;
-}
 
 w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream) {
     DeviceInfo* d = nullptr;
@@ -174,13 +160,19 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream) {
     if (!aligned(a.workspace, 16)) return W4A16_ERR_ALIGN;
     if (a.workspace_bytes < gemv_workspace_bytes((int)a.N, d->num_sms)) return W4A16_ERR_SHAPE;
     GemvMaps maps;
-    const uint32_t mpad = a.M > 8 ? 16u : 8u;
-    st = encode_2d(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.qweight, (uint64_t)a.K / 8, (uint64_t)a.N,
-                   (uint64_t)a.K / 2, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (st != W4A16_OK) return st;
-    st = encode_2d(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * 2,
-                   64, mpad + 2, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != W4A16_OK) return st;
+    {
+        EncodeTiledFn enc = nullptr;
+        st = encoder(&enc);
+        if (st != W4A16_OK) return st;
+        cuuint64_t dims[3] = {16, (cuuint64_t)a.N, (cuuint64_t)(a.K / 128)};
+        cuuint64_t strides[2] = {(cuuint64_t)(a.K / 2), 64};
+        cuuint32_t box[3] = {16, 128, 4};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (enc(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(a.qweight), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4A16_ERR_CUDA;
+    }
     return from_cuda(launch_gemv(maps, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
                                  a.workspace, (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status, stream));
 }

@@ -5,63 +5,68 @@
 //  bandwidth (section 2: weight-only quantization relieves the memory bottleneck).
 //  SqueezeLLM article, section 2.3: the fp16 sparse term is added to the dense product.]
 //
-// Design (B200).  Each packed weight byte is streamed once from HBM through a TMA pipeline
-// by a persistent, evenly balanced grid.
-//   - Work units are (128-channel row block, quantization group of 128 k), ordered row block
-//     by row block.  The grid has P = min(2 x SMs, units) CTAs; CTA p takes the contiguous
-//     unit range [p*T/P, (p+1)*T/P), so every CTA streams the same number of bytes and the
-//     GPU runs one balanced wave (stream-K).  Two resident CTAs per SM keep enough TMA
-//     traffic in flight to saturate HBM.
-//   - A row block processed whole by one CTA is written straight to y.  A row block split
+// Design (B200).  Each packed weight byte is streamed once from HBM by a persistent grid of
+// one CTA per SM.
+//   - Work units are (128-channel row block, block of 4 quantization groups = 512 k): 32 KB
+//     of packed weights, brought in by ONE TMA copy.  A CTA's TMA copies are served nearly
+//     one after another, so the bytes per copy set the streaming rate of a CTA: 8 KB copies
+//     stream at ~16 GB/s per CTA, 32 KB copies at ~40 GB/s, enough for one CTA per SM to
+//     saturate HBM.  The copy uses a 3-D view of qweight (16 words of a group, rows, groups;
+//     strides K/2 and 64 bytes), so it lands as [4 groups][128 rows][64 bytes] and the
+//     consumers' 128-bit loads of one group are free of bank conflicts.
+//   - Stream-K: CTA p takes the contiguous unit range [p*T/P, (p+1)*T/P), ordered row block
+//     by row block, so every CTA streams the same number of bytes in one balanced wave.  A
+//     row block processed whole by one CTA is written straight to y.  A row block split
 //     between CTAs leaves fp32 partial tiles in the caller's workspace.  Each contributing
 //     CTA then increments the row block's counter.  The CTA that completes the count sums
 //     the partials once its own stream has ended, writes y and resets the counter to zero.
 //     No CTA waits for another, and the workspace is all-zero again after every call.
-//   - CTA = 4 consumer warps (32 channels each, two m16 tiles), 1 TMA producer warp, 1 sum
-//     warp and 1 epilogue warp.  At the end of each row-block segment the consumers drop
-//     their accumulators into one of two shared-memory partial tiles and go on streaming;
-//     the epilogue warp does the workspace exchange, the CSR term and the stores of y.  One pipeline stage holds one unit: the packed weights of the 128 channels
-//     (TMA box 16 words x 128 rows, 8 KB) and the group's activations (two TMA boxes of
-//     64 k x (Mpad + 2) tokens, 128-byte swizzle).  The second box is loaded from token -2.
-//     Its rows therefore sit two swizzle phases after the first box's rows, which makes
-//     every B-fragment load below free of shared-memory bank conflicts.
-//   - On B200 the CUDA cores cannot do one FMA per weight per token at HBM rate, so the
-//     multiply-adds go to the tensor cores (mma.sync m16n8k16) with the operands swapped.
-//     The MMA rows are 16 channels, the columns are 8 tokens (two tiles when M > 8), and
-//     the depth is 16 input channels.  The A operand (the weights) goes from shared memory
-//     to registers.  One LOP3 per nibble pair makes the bf16 pair (128 + q_lo, 128 + q_hi)
-//     (exponent bits 0x43), and those exact values feed the MMA unchanged.  The zero point
-//     and the scale are applied once per group in fp32:
-//         y += s * ( sum_k (128 + q_k) x_k  -  (128 + z) * X_g ),   X_g = sum_{k in g} x_k.
-//     The sum warp computes X_g for every staged group from the x tile, so the per-weight
-//     work is one shift and one LOP3 per two weights plus the MMA.
+//   - Warps: 8 consumers, 1 TMA producer (weights), 2 helpers, 1 epilogue.  Everything
+//     except the weights comes in through the helpers with ordinary loads, so the weights
+//     are the only TMA traffic.  For their 2 groups of each unit the helpers
+//       * copy the activations from global memory (L2-resident) into shared memory, already
+//         in the order of the MMA B fragments;
+//       * compute the group sums X_g of every token with tensor-core MMAs against an
+//         all-ones A operand;
+//       * decode the scales and zero points of the unit's 128 rows into fp32 pairs
+//         (s, -(128 + z)).
+//   - Consumer warp c owns rows 32 (c % 4) .. +31 and groups 2 (c / 4), +1 of every unit
+//     (two m16 tiles x two groups).  The MMA is the legacy mma.sync m16n8k16 with swapped
+//     operands: rows are 16 channels, columns 8 tokens (two tiles when M > 8), depth 16 input
+//     channels.  The A operand (weights) goes from shared memory to registers.  One LOP3 per
+//     nibble pair makes the bf16 pair (128 + q_lo, 128 + q_hi) (exponent bits 0x43), and
+//     those exact values feed the MMA unchanged.  The zero point and the scale are applied
+//     once per group in fp32:
+//         acc += s * ( sum_k (128 + q_k) x_k  -  (128 + z) * X_g ).
 //   - Which physical k feeds which MMA slot.  Thread t (= lane % 4) takes words 4t..4t+3 of
 //     a row's group, i.e. k in [32t, 32t+32).  MMA pair w (0..3) uses word w: nibble pairs
 //     (0,1) in the first MMA and (2,3) in the second.  Pair p of word w holds
-//     k = 32t + 8w + 2p + {0,1}.  The B fragment of thread (token g, t) is then one
-//     128-bit load of x[g][32t + 8w .. +8], whose four 32-bit parts are the same pairs.
-//   - Scales and zero points are stored group-major, so a unit's parameters (128 fp16 scales
-//     and 16 words of zero points) are two contiguous runs that 1D bulk copies bring into the
-//     same stage.
-//   - Programmatic dependent launch.  The weights of the first stages may be fetched before
-//     the previous kernel on the stream has finished.  The producer waits for that kernel
-//     before it loads x.  The epilogue warp waits before it touches the workspace, gathers x
-//     for the CSR term, or writes y.
+//     k = 32t + 8w + 2p + {0,1}.  The B fragment of thread (token g, t) is then the 16 bytes
+//     x[g][32t + 8w .. +8], whose four 32-bit parts are the same pairs.
+//   - At the end of a row-block segment the consumers drop their accumulators into a
+//     shared-memory partial tile (one half per group pair) and go on streaming; the
+//     epilogue warp adds the halves and does the workspace exchange, the CSR term and the
+//     stores of y.
+//   - Programmatic dependent launch.  The weights may be fetched before the previous kernel
+//     on the stream has finished.  The helpers wait for it before they load x; the
+//     epilogue and the completion phase wait before they touch the workspace or y.
 #include "common.cuh"
 #include "internal.h"
 
 namespace w4a16 {
 
-constexpr int kGemvRows = 128;
-constexpr int kGemvConsumers = 4;                         // warps 0..3
-constexpr int kGemvProducer = kGemvConsumers;             // warp 4: TMA
-constexpr int kGemvSummer = kGemvConsumers + 1;           // warp 5: per-group token sums X_g
-constexpr int kGemvEpilogue = kGemvConsumers + 2;         // warp 6: partial exchange, CSR, y
-constexpr int kGemvThreads = 32 * (kGemvConsumers + 3);
-constexpr int kGemvStages = 6;
-constexpr int kGemvWBytes = kGemvRows * 64;  // one group of packed weights for 128 rows
-constexpr int kGemvCtasPerSm = 2;
-constexpr int kGemvSlotFloats = kGemvRows * 16;  // one partial tile [128][16] fp32
+constexpr int kGemvRows = 128;                                  // output channels per row block
+constexpr int kGemvUnitGroups = 4;                              // groups of 128 k per work unit
+constexpr int kGemvGroupBytes = kGemvRows * 64;                 // one group of packed weights, 128 rows
+constexpr int kGemvWBytes = kGemvUnitGroups * kGemvGroupBytes;  // 32 KB per unit
+constexpr int kGemvConsumers = 8;                               // warps 0..7
+constexpr int kGemvProducer = 8;                                // warp 8
+constexpr int kGemvHelper0 = 9;                                 // warps 9, 10
+constexpr int kGemvHelpers = 2;
+constexpr int kGemvEpilogue = 11;                               // warp 11
+constexpr int kGemvThreads = 32 * 12;
+constexpr int kGemvStages = 4;
+constexpr int kGemvSlotFloats = kGemvRows * 16;                 // one partial tile in the workspace
 
 struct GemvArgs {
     const uint16_t* x;
@@ -75,25 +80,25 @@ struct GemvArgs {
     float* partials;     // workspace: [2P][128][16] fp32
     unsigned* counters;  // workspace: [N/128], zero between calls
     int M, N, K;
-    long long T;         // work units = (N/128) * (K/128)
+    long long T;         // work units = (N/128) * (K/512)
     int P;               // CTAs
     unsigned* err;
 };
 
 template <int NT>
 struct GemvSmem {
-    static constexpr int kMpad = 8 * NT;
-    static constexpr int kXRows = kMpad + 2;                       // tokens -2 .. Mpad-1 (box 1)
-    static constexpr int kXTx = kXRows * 128;                        // bytes one x box brings
-    static constexpr int kXBox = ((kXTx + 1023) / 1024) * 1024;      // 1024-aligned slot
-    static constexpr int kStage = kGemvWBytes + 2 * kXBox;   // 1024-aligned: the x boxes are swizzled
-    static constexpr int kParOff = kGemvStages * kStage;       // [stage]: scales 256 B + zeros 64 B
-    static constexpr int kPartOff = kParOff + kGemvStages * 512;
-    static constexpr int kXsumOff = kPartOff + 2 * kGemvSlotFloats * 4;  // [stage][16] fp32
-    static constexpr int kBarOff = kXsumOff + kGemvStages * 16 * 4;
-    static constexpr int kListOff = kBarOff + (4 * kGemvStages + 4) * 8;  // row blocks this CTA completes
+    static constexpr int kCols = 8 * NT;                                    // token columns
+    static constexpr int kXBytes = kGemvUnitGroups * NT * 4 * 32 * 16;      // B fragments of a unit
+    static constexpr int kParBytes = kGemvUnitGroups * kGemvRows * 8;       // (s, -(128+z)) per group, row
+    static constexpr int kSumBytes = kGemvUnitGroups * 16 * 4;              // X_g per group, token
+    static constexpr int kXOff = kGemvStages * kGemvWBytes;
+    static constexpr int kParOff = kXOff + kGemvStages * kXBytes;
+    static constexpr int kSumOff = kParOff + kGemvStages * kParBytes;
+    static constexpr int kPartOff = kSumOff + kGemvStages * kSumBytes;      // [2 halves][128 rows][kCols]
+    static constexpr int kBarOff = kPartOff + 2 * kGemvRows * kCols * 4;
+    static constexpr int kListOff = kBarOff + (4 * kGemvStages + 2) * 8;    // row blocks this CTA completes
     static constexpr int kBytes = kListOff + 16 * 4;
-    static_assert(kStage % 1024 == 0, "128-byte-swizzled TMA boxes need 1024-byte aligned stages");
+    static_assert(kBytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -101,34 +106,11 @@ __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-__device__ __forceinline__ uint4 lds128(const uint8_t* p) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(smem_u32(p)));
-    return v;
-}
-
 // bf16 pairs (128 + q_lo, 128 + q_hi) of the 4 nibble pairs of a packed word.
 __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t out[4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(out[i]) : "r"(w >> (4 * i)), "r"(0x000F000Fu), "r"(0x43004300u));
-}
-
-// fp32 sum of the 64 bf16 values of one 128-byte row of an x box (the order within the row
-// does not matter, so the swizzle does not either).
-__device__ __forceinline__ float row_sum_128b(const uint8_t* row) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const uint4 v = lds128(row + 16 * c);
-        a0 += __uint_as_float(v.x << 16) + __uint_as_float(v.x & 0xFFFF0000u);
-        a1 += __uint_as_float(v.y << 16) + __uint_as_float(v.y & 0xFFFF0000u);
-        a2 += __uint_as_float(v.z << 16) + __uint_as_float(v.z & 0xFFFF0000u);
-        a3 += __uint_as_float(v.w << 16) + __uint_as_float(v.w & 0xFFFF0000u);
-    }
-    return (a0 + a1) + (a2 + a3);
 }
 
 __device__ __forceinline__ long long unit_begin(int p, long long T, int P) { return T * p / P; }
@@ -164,128 +146,159 @@ __device__ __forceinline__ void write_row(const GemvArgs& p, int n, float v[16])
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
-gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
-                  const GemvArgs p) {
+__global__ void __launch_bounds__(kGemvThreads, 1)
+gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
     using L = GemvSmem<NT>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-    uint64_t* empty = full + kGemvStages;
-    uint64_t* xfull = empty + kGemvStages;
-    uint64_t* xempty = xfull + kGemvStages;
-    uint64_t* pfull = xempty + kGemvStages;   // [2] a partial tile is ready for the epilogue
-    uint64_t* pempty = pfull + 2;             // [2] the epilogue is done with a partial tile
-    float* part = reinterpret_cast<float*>(smem + L::kPartOff);     // [2][row][token]
-    float* xsum = reinterpret_cast<float*>(smem + L::kXsumOff);     // [stage][token]
+    constexpr int S = kGemvStages;
+    constexpr int C = L::kCols;
+    // Pointers into shared memory derive from the array itself (no integer round trip), so the
+    // compiler keeps the shared address space and issues shared-memory loads and stores.
+    extern __shared__ __align__(128) uint8_t smem[];
+    if (smem_u32(smem) & 127u) {  // the TMA destinations need 128-byte alignment
+        if (threadIdx.x == 0) record_error(p.err, kErrShape);
+        return;
+    }
+    uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+    uint64_t* wempty = wfull + S;   // the consumers have read the weights of a stage
+    uint64_t* xfull = wempty + S;   // the helpers have filled a stage's activations and parameters
+    uint64_t* xempty = xfull + S;   // the consumers are done with them
+    uint64_t* pfull = xempty + S;   // the partial tile holds a finished segment
+    uint64_t* pempty = pfull + 1;   // the epilogue is done with it
+    float* part = reinterpret_cast<float*>(smem + L::kPartOff);
     int* reduce_list = reinterpret_cast<int*>(smem + L::kListOff);  // [0] = count, then row blocks
 
-    const int G = p.K >> 7;
+    const int GB = p.K >> 9;  // units per row block
     const long long u0 = unit_begin(blockIdx.x, p.T, p.P);
     const int n = (int)(unit_begin(blockIdx.x + 1, p.T, p.P) - u0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kGemvStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kGemvConsumers + 1);  // consumers + the sum warp read the stage
-            mbar_init(&xfull[i], 1);
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&wfull[i], 1);
+            mbar_init(&wempty[i], kGemvConsumers);
+            mbar_init(&xfull[i], kGemvHelpers);
             mbar_init(&xempty[i], kGemvConsumers);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&pfull[i], kGemvConsumers);
-            mbar_init(&pempty[i], 1);
-        }
+        mbar_init(pfull, kGemvConsumers);
+        mbar_init(pempty, 1);
         reduce_list[0] = 0;
         fence_mbarrier_init();
     }
     __syncthreads();
 
-    if (warp == kGemvSummer) {
-        // ------------------------------------------------------------------ sum warp
-        // lane l sums token l/2, half l%2 (k 0..63 from box 0, k 64..127 from box 1 at row +2)
-        const int tok = lane >> 1, half = lane & 1;
-        for (int s = 0; s < n; ++s) {
-            const int slot = s % kGemvStages;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], (s / kGemvStages) & 1) &&
-                                                        (s < kGemvStages ||
-                                                         mbar_wait_bounded(&xempty[slot], ((s / kGemvStages) - 1) & 1)));
-            if (!ok) {
-                if (lane == 0) record_error(p.err, kErrTimeout);
-                break;
-            }
-            float v = 0.0f;
-            if (tok < L::kMpad) {
-                const uint8_t* xs = smem + slot * L::kStage + kGemvWBytes + half * L::kXBox;
-                v = row_sum_128b(xs + (tok + 2 * half) * 128);
-            }
-            v += __shfl_xor_sync(0xffffffffu, v, 1);
-            if (half == 0 && tok < L::kMpad) xsum[slot * 16 + tok] = v;
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&empty[slot]);
-                mbar_arrive(&xfull[slot]);
-            }
-        }
-    } else if (warp == kGemvProducer) {
+    if (warp == kGemvProducer) {
         // ------------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tensormap(&map_w);
-            prefetch_tensormap(&map_x);
-            const uint32_t tx = (uint32_t)(kGemvWBytes + 2 * L::kXTx + 256 + 64);
-            // the unit's scales (128 fp16 of row block rb, group g) and zero points (16 words)
-            auto load_params = [&](int slot, int rb, int g, uint64_t* bar) {
-                uint8_t* par = smem + L::kParOff + slot * 512;
-                bulk_load(par, p.scales + (size_t)g * p.N + (size_t)rb * kGemvRows, 256, bar);
-                bulk_load(par + 256, p.zeros + (size_t)g * (p.N >> 3) + (size_t)rb * (kGemvRows / 8), 64, bar);
-            };
-            auto coords = [&](int s, int& rb, int& g) {
-                const long long u = u0 + s;
-                rb = (int)(u / G);
-                g = (int)(u - (long long)rb * G);
-            };
-            const int pre = n < kGemvStages ? n : kGemvStages;
-            for (int s = 0; s < pre; ++s) {   // weights do not depend on the previous kernel
-                int rb, g;
-                coords(s, rb, g);
-                mbar_arrive_expect_tx(&full[s], tx);
-                tma_load_2d(smem + s * L::kStage, &map_w, &full[s], g * 16, rb * kGemvRows);
-                load_params(s, rb, g, &full[s]);
-            }
-            griddep_wait();
-            for (int s = 0; s < pre; ++s) {
-                int rb, g;
-                coords(s, rb, g);
-                uint8_t* xs = smem + s * L::kStage + kGemvWBytes;
-                tma_load_2d(xs, &map_x, &full[s], g * 128, 0);
-                tma_load_2d(xs + L::kXBox, &map_x, &full[s], g * 128 + 64, -2);
-            }
-            int issued = pre;
-            for (int s = pre; s < n; ++s) {
-                const int slot = s % kGemvStages;
-                if (!mbar_wait_bounded(&empty[slot], ((s / kGemvStages) - 1) & 1)) {
+            int issued = 0;
+            for (int s = 0; s < n; ++s) {
+                const int slot = s % S;
+                if (s >= S && !mbar_wait_bounded(&wempty[slot], ((s / S) - 1) & 1)) {
                     record_error(p.err, kErrTimeout);
                     break;
                 }
-                int rb, g;
-                coords(s, rb, g);
-                uint8_t* st = smem + slot * L::kStage;
-                mbar_arrive_expect_tx(&full[slot], tx);
-                tma_load_2d(st, &map_w, &full[slot], g * 16, rb * kGemvRows);
-                load_params(slot, rb, g, &full[slot]);
-                tma_load_2d(st + kGemvWBytes, &map_x, &full[slot], g * 128, 0);
-                tma_load_2d(st + kGemvWBytes + L::kXBox, &map_x, &full[slot], g * 128 + 64, -2);
+                const long long u = u0 + s;
+                const int rb = (int)(u / GB), gb = (int)(u - (long long)rb * GB);
+                mbar_arrive_expect_tx(&wfull[slot], (uint32_t)kGemvWBytes);
+                tma_load_3d(smem + slot * kGemvWBytes, &map_w, &wfull[slot], 0, rb * kGemvRows, gb * kGemvUnitGroups);
                 ++issued;
             }
             // the copies this CTA started must land before it may exit
-            for (int s = issued > kGemvStages ? issued - kGemvStages : 0; s < issued; ++s)
-                (void)mbar_wait_bounded(&full[s % kGemvStages], (s / kGemvStages) & 1);
+            for (int s = issued > S ? issued - S : 0; s < issued; ++s)
+                (void)mbar_wait_bounded(&wfull[s % S], (s / S) & 1);
+        }
+    } else if (warp >= kGemvHelper0 && warp < kGemvHelper0 + kGemvHelpers) {
+        // ------------------------------------------------------------------ helpers
+        // Helper h serves groups 2h, 2h+1 of every unit.  Lane (gq, t) loads the B fragments
+        // of token tile j: x[8j + gq][k0 + 32t + 8w .. +8] for w = 0..3, and the parameters of
+        // rows 4 lane .. 4 lane + 3.
+        const int h = warp - kGemvHelper0;
+        const int gq = lane >> 2, t = lane & 3;
+        const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};  // bf16 1.0 pairs
+        griddep_wait();  // x belongs to the stream order
+        for (int s = 0; s < n; ++s) {
+            const int slot = s % S;
+            const long long u = u0 + s;
+            const int rb = (int)(u / GB), gb = (int)(u - (long long)rb * GB);
+            // global loads first: they do not touch the ring and overlap the wait below
+            uint4 xv[2][NT][4];
+            uint2 scv[2];
+            uint32_t zw[2];
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg) {
+                const int g = gb * kGemvUnitGroups + 2 * h + gg;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    const int m = 8 * j + gq;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        xv[gg][j][w] = m < p.M ? ldg_cached(p.x + (size_t)m * p.K + ((size_t)g << 7) + 32 * t + 8 * w)
+                                               : make_uint4(0u, 0u, 0u, 0u);
+                }
+                scv[gg] = __ldg(reinterpret_cast<const uint2*>(p.scales + (size_t)g * p.N + (size_t)rb * kGemvRows) + lane);
+                zw[gg] = __ldg(p.zeros + (size_t)g * (p.N >> 3) + (size_t)rb * (kGemvRows / 8) + (lane >> 1));
+            }
+            if (s >= S && !__all_sync(0xffffffffu, mbar_wait_bounded(&xempty[slot], ((s / S) - 1) & 1))) {
+                if (lane == 0) record_error(p.err, kErrTimeout);
+                break;
+            }
+            uint8_t* xs = smem + L::kXOff + slot * L::kXBytes;
+            float4* par = reinterpret_cast<float4*>(smem + L::kParOff + slot * L::kParBytes);
+            float* sum = reinterpret_cast<float*>(smem + L::kSumOff + slot * L::kSumBytes);
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg)
+#pragma unroll
+                for (int j = 0; j < NT; ++j)
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        *reinterpret_cast<uint4*>(xs + (((((2 * h + gg) * NT + j) * 4 + w) * 32) + lane) * 16) =
+                            xv[gg][j][w];
+            // X_g of tokens 8j + 2t, 8j + 2t + 1: column sums of B against all-ones rows, in
+            // 4 NT independent chains of 4 MMAs
+            float dx[2][NT][2][4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+#pragma unroll
+                for (int gg = 0; gg < 2; ++gg)
+#pragma unroll
+                    for (int j = 0; j < NT; ++j)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t B[2] = {u4_get(xv[gg][j][w], 2 * hh), u4_get(xv[gg][j][w], 2 * hh + 1)};
+                            if (w == 0)
+                                mma_16816_bf16_zero_nv(dx[gg][j][hh], ones, B);
+                            else
+                                mma_16816_bf16_nv(dx[gg][j][hh], ones, B);
+                        }
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg) {
+                const int gp = 2 * h + gg;  // group within the unit
+#pragma unroll
+                for (int j = 0; j < NT; ++j)
+                    if (gq == 0)
+                        *reinterpret_cast<float2*>(&sum[gp * 16 + 8 * j + 2 * t]) =
+                            make_float2(dx[gg][j][0][0] + dx[gg][j][1][0], dx[gg][j][0][1] + dx[gg][j][1][1]);
+                // rows 4 lane + i: scale bits in scv, zero point in nibble (4 lane + i) % 8 of zw
+                const uint32_t zsh = 16u * (lane & 1);
+                float sv[4], bv[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t bits = (i < 2 ? scv[gg].x : scv[gg].y) >> (16 * (i & 1));
+                    sv[i] = fp16_bits_to_float((uint16_t)(bits & 0xFFFFu));
+                    bv[i] = -(float)(128u + ((zw[gg] >> (zsh + 4 * i)) & 15u));
+                }
+                par[gp * (kGemvRows / 2) + 2 * lane] = make_float4(sv[0], bv[0], sv[1], bv[1]);
+                par[gp * (kGemvRows / 2) + 2 * lane + 1] = make_float4(sv[2], bv[2], sv[3], bv[3]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xfull[slot]);
         }
     } else if (warp < kGemvConsumers) {
         // ------------------------------------------------------------------ consumers
         const int gq = lane >> 2, t = lane & 3;
-        const int rbase = 32 * warp + gq;  // this thread's rows: rbase + 16 i + 8 h
-        int seg = 0;                       // segments handed to the epilogue so far
+        const int half = warp >> 2;                  // groups 2 half, 2 half + 1 of each unit
+        const int rbase = 32 * (warp & 3) + gq;      // rows rbase + 16 i + 8 hh
+        int seg = 0;
         float acc[2][NT][4];
 #pragma unroll
         for (int i = 0; i < 2; ++i)
@@ -294,137 +307,116 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0f;
 
-        int rb = (int)(u0 / G), g = (int)(u0 - (long long)rb * G);  // coordinates of unit u0 + s
-        for (int s = 0; s < n; ++s, (g + 1 == G ? (g = 0, ++rb) : ++g)) {
-            const int slot = s % kGemvStages;
-
-            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], (s / kGemvStages) & 1));
-            if (!ok) {
+        int rb = (int)(u0 / GB), gb = (int)(u0 - (long long)rb * GB);  // coordinates of unit u0 + s
+        for (int s = 0; s < n; ++s, (gb + 1 == GB ? (gb = 0, ++rb) : ++gb)) {
+            const int slot = s % S;
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&wfull[slot], (s / S) & 1))) {
                 if (lane == 0) record_error(p.err, kErrTimeout);
                 break;
             }
-            const uint8_t* ws = smem + slot * L::kStage;
-            const uint8_t* xs = ws + kGemvWBytes;
-            uint4 wv[2][2];
+            const uint8_t* ws = smem + slot * kGemvWBytes;
+            uint4 wv[2][2][2];  // [group][tile i][row half hh]
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
+            for (int gg = 0; gg < 2; ++gg)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) wv[i][h] = lds128(ws + (rbase + 16 * i + 8 * h) * 64 + t * 16);
-            uint4 xv[NT][4];
+                for (int i = 0; i < 2; ++i)
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const int b = t >> 1, c = 4 * (t & 1) + w;
-                    const int row = 8 * j + gq + 2 * b;
-                    xv[j][w] = lds128(xs + b * L::kXBox + row * 128 + ((c ^ (row & 7)) << 4));
-                }
-            }
-            uint32_t sz4[4];  // rows rbase + 0, 8, 16, 24: scale bits | zero << 16
-            {
-                const uint8_t* par = smem + L::kParOff + slot * 512;
-                const uint16_t* sc = reinterpret_cast<const uint16_t*>(par);
-                const uint32_t* zw = reinterpret_cast<const uint32_t*>(par + 256);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int row = rbase + 8 * k;
-                    sz4[k] = (uint32_t)sc[row] | (((zw[row >> 3] >> (4 * (row & 7))) & 15u) << 16);
-                }
-            }
+                    for (int hh = 0; hh < 2; ++hh)
+                        wv[gg][i][hh] = *reinterpret_cast<const uint4*>(
+                            ws + (2 * half + gg) * kGemvGroupBytes + (rbase + 16 * i + 8 * hh) * 64 + 16 * t);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-
-            // MMA chains: kParts independent partial accumulators per (tile, token tile), one per
-            // packed word (M <= 8) or per pair of words (M <= 16), so that the dependent
-            // mma.sync chains are short and the tensor pipe sees several in flight.
-            constexpr int kParts = NT == 1 ? 4 : 2;
-            float d[2][NT][4];
-            {
-                float dp[kParts][2][NT][4];
+            if (lane == 0) mbar_arrive(&wempty[slot]);
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&xfull[slot], (s / S) & 1))) {
+                if (lane == 0) record_error(p.err, kErrTimeout);
+                break;
+            }
+            const uint8_t* xs = smem + L::kXOff + slot * L::kXBytes;
+            const float2* par = reinterpret_cast<const float2*>(smem + L::kParOff + slot * L::kParBytes);
+            const float* sum = reinterpret_cast<const float*>(smem + L::kSumOff + slot * L::kSumBytes);
+            // GI groups at a time: both for M <= 8 (4 independent MMA chains per warp), one for
+            // M > 8 (already 4 chains: 2 tiles x 2 token tiles), which keeps the registers in bounds
+            constexpr int GI = NT == 1 ? 2 : 1;
+#pragma unroll
+            for (int pass = 0; pass < 2 / GI; ++pass) {
+                uint4 xv[GI][NT][4];
+#pragma unroll
+                for (int g2 = 0; g2 < GI; ++g2)
+#pragma unroll
+                    for (int j = 0; j < NT; ++j)
+#pragma unroll
+                        for (int w = 0; w < 4; ++w)
+                            xv[g2][j][w] = *reinterpret_cast<const uint4*>(
+                                xs + (((((2 * half + pass * GI + g2) * NT + j) * 4 + w) * 32) + lane) * 16);
+                float d[GI][2][NT][4];
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
-                    const int part_i = w % kParts;
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        uint32_t pa0[4], pa1[4];
-                        unpack_word(u4_get(wv[i][0], w), pa0);
-                        unpack_word(u4_get(wv[i][1], w), pa1);
+                    for (int g2 = 0; g2 < GI; ++g2) {
 #pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const uint32_t A[4] = {pa0[2 * hh], pa1[2 * hh], pa0[2 * hh + 1], pa1[2 * hh + 1]};
+                        for (int i = 0; i < 2; ++i) {
+                            uint32_t pa0[4], pa1[4];
+                            unpack_word(u4_get(wv[pass * GI + g2][i][0], w), pa0);
+                            unpack_word(u4_get(wv[pass * GI + g2][i][1], w), pa1);
 #pragma unroll
-                            for (int j = 0; j < NT; ++j) {
-                                const uint32_t B[2] = {u4_get(xv[j][w], 2 * hh), u4_get(xv[j][w], 2 * hh + 1)};
-                                if (w < kParts && hh == 0)
-                                    mma_16816_bf16_zero(dp[part_i][i][j], A, B);
-                                else
-                                    mma_16816_bf16(dp[part_i][i][j], A, B);
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const uint32_t A[4] = {pa0[2 * hh], pa1[2 * hh], pa0[2 * hh + 1], pa1[2 * hh + 1]};
+#pragma unroll
+                                for (int j = 0; j < NT; ++j) {
+                                    const uint32_t B[2] = {u4_get(xv[g2][j][w], 2 * hh), u4_get(xv[g2][j][w], 2 * hh + 1)};
+                                    if (w == 0 && hh == 0)
+                                        mma_16816_bf16_zero_nv(d[g2][i][j], A, B);
+                                    else
+                                        mma_16816_bf16_nv(d[g2][i][j], A, B);
+                                }
                             }
                         }
                     }
                 }
+                // the group's zero point and scale, applied in fp32: acc += s (d - (128 + z) X_g)
 #pragma unroll
-                for (int i = 0; i < 2; ++i)
+                for (int g2 = 0; g2 < GI; ++g2) {
+                    const int gp = 2 * half + pass * GI + g2;
+                    float2 sp[4];  // rows rbase + 8k, k = 2i + hh
 #pragma unroll
-                    for (int j = 0; j < NT; ++j)
+                    for (int k = 0; k < 4; ++k) sp[k] = par[gp * kGemvRows + rbase + 8 * k];
+                    float2 X[NT];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float v = dp[0][i][j][e];
+                    for (int j = 0; j < NT; ++j) X[j] = *reinterpret_cast<const float2*>(&sum[gp * 16 + 8 * j + 2 * t]);
 #pragma unroll
-                            for (int q = 1; q < kParts; ++q) v += dp[q][i][j][e];
-                            d[i][j][e] = v;
+                    for (int i = 0; i < 2; ++i)
+#pragma unroll
+                        for (int j = 0; j < NT; ++j) {
+                            const float2 a = sp[2 * i], b = sp[2 * i + 1];
+                            acc[i][j][0] = fmaf(a.x, fmaf(a.y, X[j].x, d[g2][i][j][0]), acc[i][j][0]);
+                            acc[i][j][1] = fmaf(a.x, fmaf(a.y, X[j].y, d[g2][i][j][1]), acc[i][j][1]);
+                            acc[i][j][2] = fmaf(b.x, fmaf(b.y, X[j].x, d[g2][i][j][2]), acc[i][j][2]);
+                            acc[i][j][3] = fmaf(b.x, fmaf(b.y, X[j].y, d[g2][i][j][3]), acc[i][j][3]);
                         }
-            }
-            // the group's zero point and scale, applied in fp32:
-            //   acc += s * d - s * (128 + z) * X_g
-            const bool xok = __all_sync(0xffffffffu, mbar_wait_bounded(&xfull[slot], (s / kGemvStages) & 1));
-            if (!xok) {
-                if (lane == 0) record_error(p.err, kErrTimeout);
-                break;
-            }
-            float2 X[NT];
-#pragma unroll
-            for (int j = 0; j < NT; ++j) X[j] = *reinterpret_cast<const float2*>(&xsum[slot * 16 + 8 * j + 2 * t]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xempty[slot]);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                // rows rbase + 16 i (index 2i) and rbase + 16 i + 8 (index 2i + 1)
-                const float sc0 = fp16_bits_to_float((uint16_t)(sz4[2 * i] & 0xFFFFu));
-                const float sc1 = fp16_bits_to_float((uint16_t)(sz4[2 * i + 1] & 0xFFFFu));
-                const float b0 = -(float)(128u + (sz4[2 * i] >> 16)), b1 = -(float)(128u + (sz4[2 * i + 1] >> 16));
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    acc[i][j][0] = fmaf(sc0, fmaf(b0, X[j].x, d[i][j][0]), acc[i][j][0]);
-                    acc[i][j][1] = fmaf(sc0, fmaf(b0, X[j].y, d[i][j][1]), acc[i][j][1]);
-                    acc[i][j][2] = fmaf(sc1, fmaf(b1, X[j].x, d[i][j][2]), acc[i][j][2]);
-                    acc[i][j][3] = fmaf(sc1, fmaf(b1, X[j].y, d[i][j][3]), acc[i][j][3]);
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xempty[slot]);
 
-            if (g == G - 1 || s == n - 1) {
+            if (gb == GB - 1 || s == n - 1) {
                 // ---------------------------------------------------------- segment end
-                // hand the accumulators to the epilogue warp through partial tile `buf`
-                const int buf = seg & 1;
-                const bool ok2 = seg < 2 || __all_sync(0xffffffffu, mbar_wait_bounded(&pempty[buf], ((seg >> 1) - 1) & 1));
-                if (!ok2) {
+                if (seg > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(pempty, (seg - 1) & 1))) {
                     if (lane == 0) record_error(p.err, kErrTimeout);
                     break;
                 }
-                float* pt = part + buf * kGemvSlotFloats;
+                float* pt = part + half * (kGemvRows * C);
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const int c0 = rbase + 16 * i, c1 = c0 + 8;
 #pragma unroll
                     for (int j = 0; j < NT; ++j) {
                         const int tk = 8 * j + 2 * t;
-                        *reinterpret_cast<float2*>(&pt[c0 * 16 + tk]) = make_float2(acc[i][j][0], acc[i][j][1]);
-                        *reinterpret_cast<float2*>(&pt[c1 * 16 + tk]) = make_float2(acc[i][j][2], acc[i][j][3]);
+                        *reinterpret_cast<float2*>(&pt[c0 * C + tk]) = make_float2(acc[i][j][0], acc[i][j][1]);
+                        *reinterpret_cast<float2*>(&pt[c1 * C + tk]) = make_float2(acc[i][j][2], acc[i][j][3]);
                         acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.0f;
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&pfull[buf]);
+                if (lane == 0) mbar_arrive(pfull);
                 ++seg;
             }
         }
@@ -433,16 +425,14 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
         // Walks the same segments as the consumers.  Lane l owns rows l, l+32, l+64, l+96.
         bool waited = false;
         int seg = 0;
-        int seg_g0 = (int)(u0 % G);
+        long long seg_first = u0;  // first unit of the current segment
         for (int s = 0; s < n; ++s) {
             const long long u = u0 + s;
-            const int rb = (int)(u / G), g = (int)(u - (long long)rb * G);
-            if (!(g == G - 1 || s == n - 1)) continue;
-            const bool whole = seg_g0 == 0 && g == G - 1;
-            seg_g0 = 0;
-            const int buf = seg & 1;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&pfull[buf], (seg >> 1) & 1));
-            if (!ok) {
+            const int rb = (int)(u / GB), gb = (int)(u - (long long)rb * GB);
+            if (!(gb == GB - 1 || s == n - 1)) continue;
+            const bool whole = seg_first == (long long)rb * GB && gb == GB - 1;
+            seg_first = u + 1;
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(pfull, seg & 1))) {
                 if (lane == 0) record_error(p.err, kErrTimeout);
                 break;
             }
@@ -450,27 +440,35 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
                 griddep_wait();  // the workspace, x and y belong to the stream order
                 waited = true;
             }
-            const float* pt = part + buf * kGemvSlotFloats;
+            const float* p0 = part;
+            const float* p1 = part + kGemvRows * C;
             if (whole) {
                 for (int r = lane; r < kGemvRows; r += 32) {
                     float v[16];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const float4 a = *reinterpret_cast<const float4*>(&pt[r * 16 + 4 * c]);
-                        v[4 * c] = a.x;
-                        v[4 * c + 1] = a.y;
-                        v[4 * c + 2] = a.z;
-                        v[4 * c + 3] = a.w;
+                    for (int c = 0; c < 16; ++c) v[c] = 0.0f;
+#pragma unroll
+                    for (int c = 0; c < C; c += 4) {
+                        const float4 a = *reinterpret_cast<const float4*>(&p0[r * C + c]);
+                        const float4 b = *reinterpret_cast<const float4*>(&p1[r * C + c]);
+                        v[c] = a.x + b.x;
+                        v[c + 1] = a.y + b.y;
+                        v[c + 2] = a.z + b.z;
+                        v[c + 3] = a.w + b.w;
                     }
                     write_row(p, rb * kGemvRows + r, v);
                 }
             } else {
-                const int pf = cta_of_unit((long long)rb * G, p.T, p.P);
-                const int pl = cta_of_unit((long long)rb * G + G - 1, p.T, p.P);
-                const int mine = 2 * (int)blockIdx.x + (u0 >= (long long)rb * G ? 0 : 1);
+                const int pf = cta_of_unit((long long)rb * GB, p.T, p.P);
+                const int pl = cta_of_unit((long long)rb * GB + GB - 1, p.T, p.P);
+                const int mine = 2 * (int)blockIdx.x + (u0 >= (long long)rb * GB ? 0 : 1);
                 float4* dst = reinterpret_cast<float4*>(p.partials + (size_t)mine * kGemvSlotFloats);
-                const float4* srcp = reinterpret_cast<const float4*>(pt);
-                for (int q = lane; q < kGemvSlotFloats / 4; q += 32) __stcg(dst + q, srcp[q]);
+                const float4* a4 = reinterpret_cast<const float4*>(p0);
+                const float4* b4 = reinterpret_cast<const float4*>(p1);
+                for (int q = lane; q < kGemvRows * C / 4; q += 32) {
+                    const float4 a = a4[q], b = b4[q];
+                    __stcg(dst + q, make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w));
+                }
                 // release the partial tile to the completing CTA: the warp's stores, then a fence
                 // and the counter increment by lane 0; the completing CTA fences after it
                 __syncwarp();
@@ -486,7 +484,7 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
                     reduce_list[1 + reduce_list[0]++] = rb;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&pempty[buf]);
+            if (lane == 0) mbar_arrive(pempty);
             ++seg;
         }
     }
@@ -497,34 +495,37 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
     // CTA completed: thread r (< 128) owns row r, loads of several slots are in flight at once.
     if (warp < kGemvConsumers || warp == kGemvEpilogue) {
         asm volatile("bar.sync 2, %0;" ::"r"(32 * (kGemvConsumers + 1)) : "memory");
-        const int r = warp < kGemvConsumers ? (int)threadIdx.x : -1;
         const int count = reduce_list[0];
-        if (count > 0) __threadfence();  // acquire: every other contributor's partial is visible
+        const int r = threadIdx.x < kGemvRows ? (int)threadIdx.x : -1;
+        if (count > 0) {
+            griddep_wait();
+            __threadfence();  // acquire: every other contributor's partial is visible
+        }
         for (int e = 0; e < count && r >= 0; ++e) {
             const int rb = reduce_list[1 + e];
-            const int pf = cta_of_unit((long long)rb * G, p.T, p.P);
-            const int pl = cta_of_unit((long long)rb * G + G - 1, p.T, p.P);
+            const int pf = cta_of_unit((long long)rb * GB, p.T, p.P);
+            const int pl = cta_of_unit((long long)rb * GB + GB - 1, p.T, p.P);
             float v[16];
 #pragma unroll
             for (int m = 0; m < 16; ++m) v[m] = 0.0f;
             for (int q0 = pf; q0 <= pl; q0 += 2) {
-                float4 a[2][4];
+                float4 a[2][C / 4];
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
                     const int q = q0 + qq;
                     if (q <= pl) {
-                        const int slotq = 2 * q + (unit_begin(q, p.T, p.P) >= (long long)rb * G ? 0 : 1);
-                        const float4* sp = reinterpret_cast<const float4*>(p.partials +
-                                                                           (size_t)slotq * kGemvSlotFloats + r * 16);
+                        const int slotq = 2 * q + (unit_begin(q, p.T, p.P) >= (long long)rb * GB ? 0 : 1);
+                        const float4* sp =
+                            reinterpret_cast<const float4*>(p.partials + (size_t)slotq * kGemvSlotFloats + r * C);
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) a[qq][c] = __ldcg(sp + c);
+                        for (int c = 0; c < C / 4; ++c) a[qq][c] = __ldcg(sp + c);
                     }
                 }
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq) {
                     if (q0 + qq <= pl) {
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
+                        for (int c = 0; c < C / 4; ++c) {
                             v[4 * c] += a[qq][c].x;
                             v[4 * c + 1] += a[qq][c].y;
                             v[4 * c + 2] += a[qq][c].z;
@@ -544,13 +545,12 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
 int gemv_max_k() { return 1 << 20; }
 
 int gemv_ctas(int N, int K, int num_sms) {
-    const long long T = (long long)(N / kGemvRows) * (K / 128);
-    const long long P = (long long)kGemvCtasPerSm * num_sms;
-    return (int)(T < P ? T : P);
+    const long long T = (long long)(N / kGemvRows) * (K / (128 * kGemvUnitGroups));
+    return (int)(T < num_sms ? T : num_sms);
 }
 
 size_t gemv_workspace_bytes(int N, int num_sms) {
-    const size_t partials = (size_t)2 * kGemvCtasPerSm * num_sms * kGemvSlotFloats * sizeof(float);
+    const size_t partials = (size_t)2 * num_sms * kGemvSlotFloats * sizeof(float);
     const size_t counters = (size_t)(N / kGemvRows) * sizeof(unsigned);
     return partials + ((counters + 255) / 256) * 256;
 }
@@ -571,15 +571,15 @@ cudaError_t launch_gemv(const GemvMaps& maps, const uint16_t* x, const uint16_t*
     a.M = M;
     a.N = N;
     a.K = K;
-    a.T = (long long)(N / kGemvRows) * (K / 128);
+    a.T = (long long)(N / kGemvRows) * (K / (128 * kGemvUnitGroups));
     a.P = gemv_ctas(N, K, num_sms);
     a.err = err;
-    const size_t partial_bytes = (size_t)2 * kGemvCtasPerSm * num_sms * kGemvSlotFloats * sizeof(float);
+    const size_t partial_bytes = (size_t)2 * num_sms * kGemvSlotFloats * sizeof(float);
     a.partials = static_cast<float*>(workspace);
     a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + partial_bytes);
 
     const bool two = M > 8;
-    const int smem = (two ? GemvSmem<2>::kBytes : GemvSmem<1>::kBytes) + 1024;
+    const int smem = two ? GemvSmem<2>::kBytes : GemvSmem<1>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(two ? gemv_w4a16_kernel<2> : gemv_w4a16_kernel<1>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -593,8 +593,8 @@ cudaError_t launch_gemv(const GemvMaps& maps, const uint16_t* x, const uint16_t*
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (two) return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<2>, maps.w, maps.x, a);
-    return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<1>, maps.w, maps.x, a);
+    if (two) return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<2>, maps.w, a);
+    return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<1>, maps.w, a);
 }
 
 }  // namespace w4a16

@@ -14,10 +14,11 @@ cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, i
                                 uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
                                 cudaStream_t stream);
 
-// Tensor maps the GEMV needs.
+// Tensor map the GEMV needs: qweight uint32 [N][K/8] seen as 3-D (16 words of a group,
+// N rows, K/128 groups; strides K/2 and 64 bytes), box 16 x 128 x 4, no swizzle.  One copy
+// brings 4 groups of 128 rows and lays them out group by group: [4][128 rows][64 bytes].
 struct GemvMaps {
-    CUtensorMap w;  // uint32 [N][K/8], box 16 words (one group) x 128 rows, no swizzle
-    CUtensorMap x;  // bf16 [M][K], box 64 (k) x (Mpad + 2) tokens, 128-byte swizzle
+    CUtensorMap w;
 };
 
 // Largest K the GEMV supports.
