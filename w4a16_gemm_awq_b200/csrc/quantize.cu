@@ -17,9 +17,15 @@
 // nibbles of 8 consecutive rows), so those stores are coalesced too.
 //
 // Bit-exactness: every float step is a single IEEE operation with round-to-nearest-even
-// (__fmul_rn, __fsub_rn, __fdiv_rn, __fadd_rn, rintf, __float2half_rn).  The build does
-// not use fast-math or flush-to-zero, so any correct implementation of the same steps
-// gives the same bits.
+// (__fmul_rn, __fsub_rn, __fdiv_rn, __fadd_rn, __float2half_rn) or an exact equivalent of
+// one.  The build does not use fast-math or flush-to-zero, so any correct implementation of
+// the same steps gives the same bits.
+//
+// Throughput: the quarter-rate XU pipe (reciprocal, rounding, float-to-integer conversion)
+// is the limiting unit, so only the division stays there.  rint(v) is computed as
+// (v + 1.5 * 2^23) - 1.5 * 2^23 on the FMA pipe: for |v| < 2^22 this is exactly
+// round-to-nearest-even, and larger magnitudes end up clamped to 0 or 15 either way.  The
+// integer code of an integral float c in [0, 15] is the low mantissa bits of c + 2^23.
 #include "common.cuh"
 #include "internal.h"
 
@@ -28,12 +34,21 @@ namespace w4a16 {
 constexpr int kQuantThreads = 256;
 constexpr int kRowsPerCta = 64;
 
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr float kIntMagic = 8388608.0f;      // 2^23
+
+// round-to-nearest-even to an integral float; exact for |v| < 2^22 (see above)
+__device__ __forceinline__ float round_rne(float v) { return __fsub_rn(__fadd_rn(v, kRoundMagic), kRoundMagic); }
+
+// the integer value of an integral float in [0, 2^22)
+__device__ __forceinline__ uint32_t int_bits(float c) { return __float_as_uint(__fadd_rn(c, kIntMagic)) & 0x3FFFFFu; }
+
 // Nibble position of each of a lane's 4 elements inside the packed word.  Element e of an
 // 8-wide block sits in nibble j with ORDER[j] = e, ORDER = {0,2,4,6,1,3,5,7}.  The even
 // lane holds elements 0..3, which go to nibbles 0,4,1,5.  The odd lane holds elements
 // 4..7, which go to nibbles 2,6,3,7.
 __device__ __forceinline__ uint32_t place_nibbles(const float q[4], bool odd) {
-    const uint32_t q0 = (uint32_t)q[0], q1 = (uint32_t)q[1], q2 = (uint32_t)q[2], q3 = (uint32_t)q[3];
+    const uint32_t q0 = int_bits(q[0]), q1 = int_bits(q[1]), q2 = int_bits(q[2]), q3 = int_bits(q[3]);
     if (!odd) return q0 | (q1 << 16) | (q2 << 4) | (q3 << 20);
     return (q0 << 8) | (q1 << 24) | (q2 << 12) | (q3 << 28);
 }
@@ -99,7 +114,7 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
             float q[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float t = __fadd_rn(rintf(__fdiv_rn(w[i], sf)), zf);
+                const float t = __fadd_rn(round_rne(__fdiv_rn(w[i], sf)), zf);
                 q[i] = fminf(fmaxf(t, 0.0f), 15.0f);
             }
             uint32_t part = place_nibbles(q, odd);
@@ -107,7 +122,7 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
             if (!odd) qweight[(size_t)n * (K >> 3) + (size_t)kc * 128 + g * 16 + (lane >> 1)] = part;
             if (lane == 0) {
                 sc_sm[g][r] = __half_as_ushort(h);
-                zc_sm[g][r] = (uint8_t)zf;
+                zc_sm[g][r] = (uint8_t)int_bits(zf);
             }
         }
         if (bad) record_error(err, kErrValue);
