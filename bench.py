@@ -222,7 +222,7 @@ def run_reference(args, world, rank):
 
     dt, _ = one_step(0, 512)
     per_out = dt / 512
-    budget = 120.0
+    budget = args.ref_budget
     P = int(max(16, min(1 << 16, budget / max(args.steps + args.warmup, 1) / per_out)))
     for i in range(args.warmup):
         one_step(i, P)
@@ -495,6 +495,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of oracle work for --impl reference (warm-up and timed steps together)")
     ap.add_argument("--skip-gemm", action="store_true")
     ap.add_argument("--skip-quant", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
