@@ -155,7 +155,7 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream) {
     DeviceInfo* d = nullptr;
     w4a16_status st = device_info(&d);
     if (st != W4A16_OK) return st;
-    if (a.K > gemv_max_k()) return W4A16_ERR_UNSUPPORTED;
+    if (a.K > gemv_max_k() || !gemv_fits((int)a.N, (int)a.K, d->num_sms)) return W4A16_ERR_UNSUPPORTED;
     if (a.workspace == nullptr) return W4A16_ERR_NULL;
     if (!aligned(a.workspace, 16)) return W4A16_ERR_ALIGN;
     if (a.workspace_bytes < gemv_workspace_bytes((int)a.N, d->num_sms)) return W4A16_ERR_SHAPE;

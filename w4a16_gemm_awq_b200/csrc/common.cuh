@@ -32,6 +32,17 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
     return t;
 }
 
+// Atomic add with acquire-release semantics at GPU scope: the caller's earlier writes are
+// visible to any thread that later observes the new value with acquire semantics, and the
+// writes released by earlier increments are visible to the caller afterwards.
+__device__ __forceinline__ unsigned atomic_add_acq_rel_gpu(unsigned* p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 // ------------------------------------------------------------------ global loads ------
 
 // Streaming 128-bit load that bypasses L1 (each weight byte is read once).

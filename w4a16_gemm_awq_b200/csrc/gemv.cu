@@ -80,7 +80,7 @@ struct GemvArgs {
     float* partials;     // workspace: [2P][128][16] fp32
     unsigned* counters;  // workspace: [N/128], zero between calls
     int M, N, K;
-    long long T;         // work units = (N/128) * (K/512)
+    uint32_t T;          // work units = (N/128) * (K/512); T * P < 2^32 (checked by the caller)
     int P;               // CTAs
     unsigned* err;
 };
@@ -113,12 +113,12 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t out[4]) {
         asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(out[i]) : "r"(w >> (4 * i)), "r"(0x000F000Fu), "r"(0x43004300u));
 }
 
-__device__ __forceinline__ long long unit_begin(int p, long long T, int P) { return T * p / P; }
+// Stream-K index arithmetic in 32 bits (T * P < 2^32), which is far cheaper than 64-bit
+// division on the GPU.
+__device__ __forceinline__ uint32_t unit_begin(uint32_t p, uint32_t T, uint32_t P) { return T * p / P; }
 
 // The CTA whose unit range contains unit u: the largest p with floor(p*T/P) <= u.
-__device__ __forceinline__ int cta_of_unit(long long u, long long T, int P) {
-    return (int)(((u + 1) * (long long)P - 1) / T);
-}
+__device__ __forceinline__ int cta_of_unit(uint32_t u, uint32_t T, uint32_t P) { return (int)(((u + 1) * P - 1) / T); }
 
 // y[m][n] for every token m of channel row n: v[m] + the CSR term of row n, rounded once.
 __device__ __forceinline__ void write_row(const GemvArgs& p, int n, float v[16]) {
@@ -168,20 +168,17 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
     int* reduce_list = reinterpret_cast<int*>(smem + L::kListOff);  // [0] = count, then row blocks
 
     const int GB = p.K >> 9;  // units per row block
-    const long long u0 = unit_begin(blockIdx.x, p.T, p.P);
-    const int n = (int)(unit_begin(blockIdx.x + 1, p.T, p.P) - u0);
+    const uint32_t u0 = unit_begin(blockIdx.x, p.T, (uint32_t)p.P);
+    const int n = (int)(unit_begin(blockIdx.x + 1, p.T, (uint32_t)p.P) - u0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < S; ++i) {
-            mbar_init(&wfull[i], 1);
-            mbar_init(&wempty[i], kGemvConsumers);
-            mbar_init(&xfull[i], kGemvHelpers);
-            mbar_init(&xempty[i], kGemvConsumers);
-        }
-        mbar_init(pfull, kGemvConsumers);
-        mbar_init(pempty, 1);
-        reduce_list[0] = 0;
+    // one barrier per thread, so that the prologue is short
+    if (threadIdx.x < 4 * S + 2) {
+        const int i = threadIdx.x;
+        const uint32_t count = i < S ? 1u : i < 2 * S ? (uint32_t)kGemvConsumers : i < 3 * S ? (uint32_t)kGemvHelpers
+                             : i < 4 * S ? (uint32_t)kGemvConsumers : i == 4 * S ? (uint32_t)kGemvConsumers : 1u;
+        mbar_init(&wfull[i], count);  // wfull, wempty, xfull, xempty, pfull, pempty are contiguous
+        if (i == 0) reduce_list[0] = 0;
         fence_mbarrier_init();
     }
     __syncthreads();
@@ -197,8 +194,8 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                     record_error(p.err, kErrTimeout);
                     break;
                 }
-                const long long u = u0 + s;
-                const int rb = (int)(u / GB), gb = (int)(u - (long long)rb * GB);
+                const uint32_t u = u0 + (uint32_t)s;
+                const int rb = (int)(u / (uint32_t)GB), gb = (int)(u - (uint32_t)rb * GB);
                 mbar_arrive_expect_tx(&wfull[slot], (uint32_t)kGemvWBytes);
                 tma_load_3d(smem + slot * kGemvWBytes, &map_w, &wfull[slot], 0, rb * kGemvRows, gb * kGemvUnitGroups);
                 ++issued;
@@ -215,15 +212,23 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
         const int h = warp - kGemvHelper0;
         const int gq = lane >> 2, t = lane & 3;
         const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};  // bf16 1.0 pairs
-        griddep_wait();  // x belongs to the stream order
         for (int s = 0; s < n; ++s) {
             const int slot = s % S;
-            const long long u = u0 + s;
-            const int rb = (int)(u / GB), gb = (int)(u - (long long)rb * GB);
-            // global loads first: they do not touch the ring and overlap the wait below
+            const uint32_t u = u0 + (uint32_t)s;
+            const int rb = (int)(u / (uint32_t)GB), gb = (int)(u - (uint32_t)rb * GB);
+            // global loads first: they do not touch the ring and overlap the wait below.  The
+            // scales and zero points do not depend on the previous kernel, so the first unit's
+            // are in flight while the helper waits for it; x is loaded after the wait.
             uint4 xv[2][NT][4];
             uint2 scv[2];
             uint32_t zw[2];
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg) {
+                const int g = gb * kGemvUnitGroups + 2 * h + gg;
+                scv[gg] = __ldg(reinterpret_cast<const uint2*>(p.scales + (size_t)g * p.N + (size_t)rb * kGemvRows) + lane);
+                zw[gg] = __ldg(p.zeros + (size_t)g * (p.N >> 3) + (size_t)rb * (kGemvRows / 8) + (lane >> 1));
+            }
+            if (s == 0) griddep_wait();  // x belongs to the stream order
 #pragma unroll
             for (int gg = 0; gg < 2; ++gg) {
                 const int g = gb * kGemvUnitGroups + 2 * h + gg;
@@ -235,8 +240,6 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                         xv[gg][j][w] = m < p.M ? ldg_cached(p.x + (size_t)m * p.K + ((size_t)g << 7) + 32 * t + 8 * w)
                                                : make_uint4(0u, 0u, 0u, 0u);
                 }
-                scv[gg] = __ldg(reinterpret_cast<const uint2*>(p.scales + (size_t)g * p.N + (size_t)rb * kGemvRows) + lane);
-                zw[gg] = __ldg(p.zeros + (size_t)g * (p.N >> 3) + (size_t)rb * (kGemvRows / 8) + (lane >> 1));
             }
             if (s >= S && !__all_sync(0xffffffffu, mbar_wait_bounded(&xempty[slot], ((s / S) - 1) & 1))) {
                 if (lane == 0) record_error(p.err, kErrTimeout);
@@ -307,7 +310,7 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0f;
 
-        int rb = (int)(u0 / GB), gb = (int)(u0 - (long long)rb * GB);  // coordinates of unit u0 + s
+        int rb = (int)(u0 / (uint32_t)GB), gb = (int)(u0 - (uint32_t)rb * GB);  // coordinates of unit u0 + s
         for (int s = 0; s < n; ++s, (gb + 1 == GB ? (gb = 0, ++rb) : ++gb)) {
             const int slot = s % S;
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(&wfull[slot], (s / S) & 1))) {
@@ -425,12 +428,12 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
         // Walks the same segments as the consumers.  Lane l owns rows l, l+32, l+64, l+96.
         bool waited = false;
         int seg = 0;
-        long long seg_first = u0;  // first unit of the current segment
+        uint32_t seg_first = u0;  // first unit of the current segment
         for (int s = 0; s < n; ++s) {
-            const long long u = u0 + s;
-            const int rb = (int)(u / GB), gb = (int)(u - (long long)rb * GB);
+            const uint32_t u = u0 + (uint32_t)s;
+            const int rb = (int)(u / (uint32_t)GB), gb = (int)(u - (uint32_t)rb * GB);
             if (!(gb == GB - 1 || s == n - 1)) continue;
-            const bool whole = seg_first == (long long)rb * GB && gb == GB - 1;
+            const bool whole = seg_first == (uint32_t)rb * GB && gb == GB - 1;
             seg_first = u + 1;
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(pfull, seg & 1))) {
                 if (lane == 0) record_error(p.err, kErrTimeout);
@@ -459,9 +462,9 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                     write_row(p, rb * kGemvRows + r, v);
                 }
             } else {
-                const int pf = cta_of_unit((long long)rb * GB, p.T, p.P);
-                const int pl = cta_of_unit((long long)rb * GB + GB - 1, p.T, p.P);
-                const int mine = 2 * (int)blockIdx.x + (u0 >= (long long)rb * GB ? 0 : 1);
+                const int pf = cta_of_unit((uint32_t)rb * GB, p.T, (uint32_t)p.P);
+                const int pl = cta_of_unit((uint32_t)rb * GB + GB - 1, p.T, (uint32_t)p.P);
+                const int mine = 2 * (int)blockIdx.x + (u0 >= (uint32_t)rb * GB ? 0 : 1);
                 float4* dst = reinterpret_cast<float4*>(p.partials + (size_t)mine * kGemvSlotFloats);
                 const float4* a4 = reinterpret_cast<const float4*>(p0);
                 const float4* b4 = reinterpret_cast<const float4*>(p1);
@@ -469,15 +472,14 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                     const float4 a = a4[q], b = b4[q];
                     __stcg(dst + q, make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w));
                 }
-                // release the partial tile to the completing CTA: the warp's stores, then a fence
-                // and the counter increment by lane 0; the completing CTA fences after it
+                // release the partial tile to the completing CTA: the warp's stores, then the
+                // counter increment by lane 0 with acquire-release semantics at GPU scope.  It
+                // orders the warp's stores (which __syncwarp orders before it) ahead of the
+                // increment, and in the CTA that completes the count it acquires every earlier
+                // contributor's partial; the barrier of the completion phase passes that on.
                 __syncwarp();
                 unsigned old = 0;
-                if (lane == 0) {
-                    __threadfence();
-                    old = atomicAdd(p.counters + rb, 1u);
-                    __threadfence();
-                }
+                if (lane == 0) old = atomic_add_acq_rel_gpu(p.counters + rb, 1u);
                 old = __shfl_sync(0xffffffffu, old, 0);
                 // the CTA that completes the row block sums its partials after the stream ends
                 if (lane == 0 && old == (unsigned)(pl - pf) && reduce_list[0] < 15)
@@ -499,22 +501,26 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
         const int r = threadIdx.x < kGemvRows ? (int)threadIdx.x : -1;
         if (count > 0) {
             griddep_wait();
-            __threadfence();  // acquire: every other contributor's partial is visible
+            fence_acq_rel_gpu();  // acquire: every other contributor's partial is visible
         }
         for (int e = 0; e < count && r >= 0; ++e) {
             const int rb = reduce_list[1 + e];
-            const int pf = cta_of_unit((long long)rb * GB, p.T, p.P);
-            const int pl = cta_of_unit((long long)rb * GB + GB - 1, p.T, p.P);
+            const int pf = cta_of_unit((uint32_t)rb * GB, p.T, (uint32_t)p.P);
+            const int pl = cta_of_unit((uint32_t)rb * GB + GB - 1, p.T, (uint32_t)p.P);
+            const bool first_starts_here = unit_begin((uint32_t)pf, p.T, (uint32_t)p.P) == (uint32_t)rb * GB;
             float v[16];
 #pragma unroll
             for (int m = 0; m < 16; ++m) v[m] = 0.0f;
-            for (int q0 = pf; q0 <= pl; q0 += 2) {
-                float4 a[2][C / 4];
+            constexpr int QB = NT == 1 ? 8 : 4;  // contributors whose loads are in flight together
+            for (int q0 = pf; q0 <= pl; q0 += QB) {
+                float4 a[QB][C / 4];
 #pragma unroll
-                for (int qq = 0; qq < 2; ++qq) {
+                for (int qq = 0; qq < QB; ++qq) {
                     const int q = q0 + qq;
                     if (q <= pl) {
-                        const int slotq = 2 * q + (unit_begin(q, p.T, p.P) >= (long long)rb * GB ? 0 : 1);
+                        // a contributor after the first starts inside the row block, so the row
+                        // block is its first segment; the first one may have started before it
+                        const int slotq = 2 * q + (q == pf && !first_starts_here ? 1 : 0);
                         const float4* sp =
                             reinterpret_cast<const float4*>(p.partials + (size_t)slotq * kGemvSlotFloats + r * C);
 #pragma unroll
@@ -522,7 +528,7 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                     }
                 }
 #pragma unroll
-                for (int qq = 0; qq < 2; ++qq) {
+                for (int qq = 0; qq < QB; ++qq) {
                     if (q0 + qq <= pl) {
 #pragma unroll
                         for (int c = 0; c < C / 4; ++c) {
@@ -549,6 +555,11 @@ int gemv_ctas(int N, int K, int num_sms) {
     return (int)(T < num_sms ? T : num_sms);
 }
 
+bool gemv_fits(int N, int K, int num_sms) {
+    const unsigned long long T = (unsigned long long)(N / kGemvRows) * (K / (128 * kGemvUnitGroups));
+    return T * (unsigned long long)gemv_ctas(N, K, num_sms) < (1ull << 32);
+}
+
 size_t gemv_workspace_bytes(int N, int num_sms) {
     const size_t partials = (size_t)2 * num_sms * kGemvSlotFloats * sizeof(float);
     const size_t counters = (size_t)(N / kGemvRows) * sizeof(unsigned);
@@ -571,7 +582,7 @@ cudaError_t launch_gemv(const GemvMaps& maps, const uint16_t* x, const uint16_t*
     a.M = M;
     a.N = N;
     a.K = K;
-    a.T = (long long)(N / kGemvRows) * (K / (128 * kGemvUnitGroups));
+    a.T = (uint32_t)((N / kGemvRows) * (K / (128 * kGemvUnitGroups)));
     a.P = gemv_ctas(N, K, num_sms);
     a.err = err;
     const size_t partial_bytes = (size_t)2 * num_sms * kGemvSlotFloats * sizeof(float);

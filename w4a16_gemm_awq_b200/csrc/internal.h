@@ -24,6 +24,9 @@ struct GemvMaps {
 // Largest K the GEMV supports.
 int gemv_max_k();
 
+// Whether the GEMV's 32-bit work-unit arithmetic covers this shape (units x CTAs < 2^32).
+bool gemv_fits(int N, int K, int num_sms);
+
 // Bytes of zero-initialised device workspace the GEMV needs for N output channels.
 size_t gemv_workspace_bytes(int N, int num_sms);
 
