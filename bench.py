@@ -396,6 +396,33 @@ def run_gpu(args, world, rank, local):
         qinfo = {"value": qb / qms / 1e6, "unit": "GB/s", "workload": "awq_quantize_g128 on the four Llama-3-8B "
                  "layers (218 M fp32 weights)", "frac_of_hbm": qb / qms / 1e6 / pk["hbm_gbs"]}
 
+    # GPU dense-and-sparse split on the config-3 layers (Llama-2-13B shapes, 0.45% outliers);
+    # algorithmic bytes: read W and a, write W_dense and the CSR
+    sinfo = None
+    if not args.skip_split:
+        sb, sms_ = 0.0, 0.0
+        per_split = []
+        for si, (name, K, N) in enumerate(workloads.CONFIGS[3]["shapes"]):
+            L = workloads.make_layer(workloads.seed_of(3, si), K=K, N=N)
+            W = torch.from_numpy(L.W).cuda()
+            act = torch.from_numpy(L.act_absmean).cuda()
+            nnz = workloads.outlier_nnz(N, K)
+            outs = (torch.empty_like(W), torch.empty(N + 1, dtype=torch.int32, device="cuda"),
+                    torch.empty(nnz, dtype=torch.int32, device="cuda"), torch.empty(nnz, dtype=torch.int16, device="cuda"))
+            wsp = torch.empty(w4.lib().awq_split_outliers_workspace_bytes(N, K), dtype=torch.uint8, device="cuda")
+            ms1, gs = time_graph(torch, lambda: w4.awq_split_outliers(W, act, workloads.ALPHA, nnz, out=outs,
+                                                                      workspace=wsp), 10, 2)
+            del gs
+            w4.check_device_status()
+            b = 8 * N * K + 4 * K + 6 * nnz + 4 * (N + 1)
+            sb += b
+            sms_ += ms1
+            per_split.append({"K": K, "N": N, "nnz": nnz, "ms": round(ms1, 4), "GB/s": round(b / ms1 / 1e6, 1)})
+            del W, act, outs, wsp
+        sinfo = {"value": sb / sms_ / 1e6, "unit": "GB/s", "workload": "awq_split_outliers on the Llama-2-13B "
+                 "layers 5120x5120 and 5120x13824, 0.45% fp16 outliers", "frac_of_hbm": sb / sms_ / 1e6 / pk["hbm_gbs"],
+                 "per_layer": per_split}
+
     if rank != 0:
         return
     cpu = None
@@ -422,6 +449,7 @@ def run_gpu(args, world, rank, local):
         "clocks": clocks,
         "gemm": gemm,
         "quantize": qinfo,
+        "outlier_split": sinfo,
     }
     print(json.dumps(line), flush=True)
 
@@ -500,6 +528,7 @@ def main():
     ap.add_argument("--skip-gemm", action="store_true")
     ap.add_argument("--skip-quant", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-split", action="store_true")
     ap.add_argument("--case", choices=["gemv", "gemm", "quantize"], help="time one kernel on one layer (ncu)")
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)

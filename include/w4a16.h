@@ -189,6 +189,46 @@ w4a16_status w4a16_gemv_noalloc(const uint16_t* x, const uint32_t* qweight, cons
                                 int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
+ * awq_split_outliers -- the dense-and-sparse split of a weight matrix, on the GPU.
+ * [SqueezeLLM article, section 2.2: sensitive weights stay in fp16 in a sparse matrix and
+ *  leave the dense part, W = W_dense + W_sparse; section 5.3: sparsity ratio 0.45%.  The
+ *  sensitivity is read as |w| * a_k, a_k the mean |x| of input channel k.]
+ *   W            fp32 [N][K] device, input (row-major, rows are output channels).
+ *   act_absmean  fp32 [K] device, a_k >= 0 and finite.
+ *   alpha        >= 0: the AWQ exponent; CSR values are fp16(w * s_k) with
+ *                s_k = max(float(pow(a_k, alpha)), 1e-4), the scaled space of the packed
+ *                dense part (see awq_quantize_g128).
+ *   nnz          number of outliers, 0 <= nnz <= N * K (for the 0.45% ratio:
+ *                floor(0.0045 * N * K)).  N * K < 2^32 and nnz < 2^31.
+ *   W_dense      fp32 [N][K] device, output: W with the outliers set to 0 (may not alias W).
+ *   row_ptr      int32 [N + 1], col_idx int32 [nnz], values fp16 bits [nnz], device,
+ *                outputs: CSR with ascending columns in every row.
+ *   workspace    device scratch of awq_split_outliers_workspace_bytes(N, K) bytes, 256-byte
+ *                aligned; its contents need not be initialised.
+ * Selection: the nnz entries with the largest score fp32(|w| * a_k); among equal scores the
+ * lower linear index n * K + k wins.  The result is unique, so it is bit-exact against any
+ * correct implementation of the same rule.
+ * Errors: NULL, SHAPE (sizes, workspace too small), ALIGN, VALUE (alpha < 0 or not finite)
+ * at launch; a non-finite W or a_k, or an fp16 overflow of a value, sets VALUE in the
+ * device status word.  nnz = 0 copies W to W_dense and zeroes row_ptr (no workspace used).
+ */
+size_t awq_split_outliers_workspace_bytes(int64_t N, int64_t K);
+w4a16_status awq_split_outliers(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                                int64_t nnz, float* W_dense, int32_t* row_ptr, int32_t* col_idx,
+                                uint16_t* values, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * w4a16_selftest_timeout -- launch a one-thread kernel whose pipeline wait can never
+ * complete and whose limit is limit_ns nanoseconds (0 .. 1e10; else W4A16_ERR_VALUE).  The
+ * wait runs out through the same bounded-wait loop the kernels use, the kernel records a
+ * timeout in the device status word and returns, and the next
+ * w4a16_check_device_status(stream) reports W4A16_ERR_TIMEOUT.  It exists so that the
+ * timeout path can be tested on a GPU without hanging or faulting it.  The pages have no
+ * counterpart.
+ */
+w4a16_status w4a16_selftest_timeout(int64_t limit_ns, void* stream);
+
+/*
  * w4a16_check_device_status -- synchronize `stream` and return the first problem that a
  * kernel recorded since the last call, or W4A16_OK.  This clears the record.  The record
  * is per device and shared by all streams of that device.

@@ -99,6 +99,28 @@ def test_quantize_validation(L):
     assert q(alpha=float("inf")) == w4.ERR_VALUE
 
 
+def test_split_validation(L):
+    def sp(W=FAKE, a=FAKE, alpha=0.5, N=16, K=256, nnz=10, Wd=FAKE, rp=FAKE, ci=FAKE, v=FAKE, ws=FAKE, wsb=1 << 30):
+        return L.awq_split_outliers(ctypes.c_void_p(W), ctypes.c_void_p(a), ctypes.c_float(alpha), N, K, nnz,
+                                    ctypes.c_void_p(Wd), ctypes.c_void_p(rp), ctypes.c_void_p(ci), ctypes.c_void_p(v),
+                                    ctypes.c_void_p(ws), wsb, None)
+    assert sp(W=0) == w4.ERR_NULL
+    assert sp(rp=0) == w4.ERR_NULL
+    assert sp(nnz=16 * 256 + 1) == w4.ERR_SHAPE
+    assert sp(nnz=-1) == w4.ERR_SHAPE
+    assert sp(N=0) == w4.ERR_SHAPE
+    assert sp(N=1 << 16, K=1 << 16) == w4.ERR_SHAPE  # N * K must stay below 2^32
+    assert sp(alpha=-0.5) == w4.ERR_VALUE
+    assert sp(alpha=float("nan")) == w4.ERR_VALUE
+    assert L.awq_split_outliers_workspace_bytes(0, 5) == 0
+    assert L.awq_split_outliers_workspace_bytes(100, 5) >= 256 + 4096 * 4 + 3 * 400
+
+
+def test_selftest_timeout_validation(L):
+    assert L.w4a16_selftest_timeout(-1, None) == w4.ERR_VALUE
+    assert L.w4a16_selftest_timeout(10 ** 11, None) == w4.ERR_VALUE
+
+
 def test_binding_has_no_cpu_path():
     """The binding refuses CPU tensors instead of computing anything itself."""
     import torch

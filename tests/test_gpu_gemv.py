@@ -131,3 +131,24 @@ def test_gemv_full_shapes_sampled(orc, cfg, i, K, N, M, csr):
     m, n = c.sample(seed=cfg * 10 + i)
     ref, ref_abs = c.reference_at(orc, m, n)
     check_close(y[m, n], ref, ref_abs, 0.0, depth(K), f"{K}x{N} M={M}", xs_abs(c.x, c.sc, m, n))
+
+
+def test_bounded_wait_times_out_and_context_survives(orc):
+    """A wait that can never complete gives up after its limit, reports TIMEOUT through the
+    device status word, and leaves the context usable for the next GEMV."""
+    import time
+    t0 = time.perf_counter()
+    w4.selftest_timeout(2_000_000)  # 2 ms
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.check_device_status()
+    assert e.value.code == w4.ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    w4.check_device_status()  # cleared
+    c = Case(orc, seed=77, K=1024, N=256, M=3)
+    d = c.device()
+    y = host_bf16_as_f64(w4.w4a16_gemv(d["x"], d["qweight"], d["scales"], d["zeros"]))
+    w4.check_device_status()
+    ref, ref_abs = c.reference(orc)
+    check_close(y, ref, ref_abs, 0.0, depth(c.K), "after timeout", xs_abs(c.x, c.sc))
+    with pytest.raises(w4.W4A16Error):
+        w4.selftest_timeout(-1)

@@ -67,11 +67,15 @@ def lib() -> ctypes.CDLL:
         L.w4a16_workspace_bytes.argtypes = [I64, I64, I64]
         L.w4a16_workspace_bytes.restype = ctypes.c_size_t
         L.w4a16_check_device_status.argtypes = [P]
+        L.w4a16_selftest_timeout.argtypes = [I64, P]
+        L.awq_split_outliers.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P, ctypes.c_size_t, P]
+        L.awq_split_outliers_workspace_bytes.argtypes = [I64, I64]
+        L.awq_split_outliers_workspace_bytes.restype = ctypes.c_size_t
         L.w4a16_status_string.argtypes = [ctypes.c_int]
         L.w4a16_status_string.restype = ctypes.c_char_p
         L.w4a16_version.argtypes = []
         for name in ("awq_quantize_g128", "w4a16_linear", "w4a16_gemv", "w4a16_gemm", "w4a16_check_device_status",
-                     "w4a16_version"):
+                     "w4a16_selftest_timeout", "awq_split_outliers", "w4a16_version"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -179,6 +183,35 @@ def check_device_status(stream=None):
     """Synchronize and raise W4A16Error if a kernel recorded a problem since the last check."""
     s = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream(torch.device("cuda"))
     _check(lib().w4a16_check_device_status(s), "device status")
+
+
+def awq_split_outliers(W, act_absmean, alpha: float, nnz: int, out=None, workspace=None):
+    """Dense-and-sparse split on the GPU.  W fp32 [N][K], act_absmean fp32 [K] (cuda).
+    Returns (W_dense fp32 [N][K], (row_ptr int32 [N+1], col_idx int32 [nnz], values int16
+    (fp16 bits) [nnz])), ready for awq_quantize_g128 and the csr= argument of the linear ops."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.dim() == 2 and W.is_contiguous()
+    assert act_absmean.dtype == torch.float32 and act_absmean.is_contiguous()
+    N, K = W.shape
+    dev = W.device
+    if out is None:
+        out = (torch.empty_like(W), torch.empty(N + 1, dtype=torch.int32, device=dev),
+               torch.empty(max(nnz, 1), dtype=torch.int32, device=dev),
+               torch.empty(max(nnz, 1), dtype=torch.int16, device=dev))
+    Wd, rp, ci, vals = out
+    nbytes = lib().awq_split_outliers_workspace_bytes(N, K)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    _check(lib().awq_split_outliers(_ptr(W), _ptr(act_absmean), ctypes.c_float(alpha), N, K, int(nnz), _ptr(Wd),
+                                    _ptr(rp), _ptr(ci), _ptr(vals), _ptr(workspace), workspace.numel(),
+                                    _stream(dev)), "awq_split_outliers")
+    return Wd, (rp, ci[:nnz], vals[:nnz])
+
+
+def selftest_timeout(limit_ns: int, stream=None) -> None:
+    """Launch the kernel whose wait can never complete (limit in ns); the next
+    check_device_status() reports W4A16_ERR_TIMEOUT."""
+    s = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream(torch.device("cuda"))
+    _check(lib().w4a16_selftest_timeout(int(limit_ns), s), "selftest_timeout")
 
 
 def status_string(code: int) -> str:

@@ -311,6 +311,43 @@ w4a16_status w4a16_gemv_noalloc(const uint16_t* x, const uint32_t* qweight, cons
     return run_gemv(a, s);
 }
 
+size_t awq_split_outliers_workspace_bytes(int64_t N, int64_t K) {
+    if (N < 1 || K < 1) return 0;
+    return split_workspace_bytes(N);
+}
+
+w4a16_status awq_split_outliers(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                                int64_t nnz, float* W_dense, int32_t* row_ptr, int32_t* col_idx, uint16_t* values,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    if (!W || !act_absmean || !W_dense || !row_ptr) return W4A16_ERR_NULL;
+    if (N < 1 || K < 1 || nnz < 0 || nnz > N * K || (uint64_t)N * (uint64_t)K >= (1ull << 32) || nnz > 0x7FFFFFFFll)
+        return W4A16_ERR_SHAPE;
+    if (!std::isfinite(alpha) || alpha < 0.0f) return W4A16_ERR_VALUE;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (nnz == 0) {  // nothing moves: W_dense = W, an empty CSR
+        if (cudaMemcpyAsync(W_dense, W, sizeof(float) * (size_t)(N * K), cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+            cudaMemsetAsync(row_ptr, 0, sizeof(int32_t) * (size_t)(N + 1), s) != cudaSuccess)
+            return W4A16_ERR_CUDA;
+        return W4A16_OK;
+    }
+    if (!col_idx || !values || !workspace) return W4A16_ERR_NULL;
+    if (!aligned(workspace, 256)) return W4A16_ERR_ALIGN;
+    if (workspace_bytes < split_workspace_bytes(N)) return W4A16_ERR_SHAPE;
+    return from_cuda(launch_split_outliers(W, act_absmean, alpha, (uint32_t)N, (uint32_t)K, (uint32_t)nnz, W_dense,
+                                           row_ptr, col_idx, values, workspace, d->num_sms, d->status, s));
+}
+
+w4a16_status w4a16_selftest_timeout(int64_t limit_ns, void* stream) {
+    if (limit_ns < 0 || limit_ns > 10000000000ll) return W4A16_ERR_VALUE;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    return from_cuda(launch_selftest_timeout((unsigned long long)limit_ns, d->status, static_cast<cudaStream_t>(stream)));
+}
+
 w4a16_status w4a16_check_device_status(void* stream) {
     DeviceInfo* d = nullptr;
     w4a16_status st = device_info(&d);

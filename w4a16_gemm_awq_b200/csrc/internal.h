@@ -35,6 +35,16 @@ cudaError_t launch_gemv(const GemvMaps& maps, const uint16_t* x, const uint16_t*
                         uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
                         cudaStream_t stream);
 
+// Dense-and-sparse split of W on the GPU (see outliers.cu).  N * K < 2^32, 1 <= nnz <= N * K.
+size_t split_workspace_bytes(int64_t N);
+cudaError_t launch_split_outliers(const float* W, const float* act, float alpha, uint32_t N, uint32_t K, uint32_t nnz,
+                                  float* W_dense, int32_t* row_ptr, int32_t* col_idx, uint16_t* values,
+                                  void* workspace, int num_sms, unsigned* err, cudaStream_t stream);
+
+// A kernel whose only wait never completes: it gives up after limit_ns and records
+// kErrTimeout (tests the bounded-wait path without any fault).
+cudaError_t launch_selftest_timeout(unsigned long long limit_ns, unsigned* err, cudaStream_t stream);
+
 // Tensor maps the GEMM needs, encoded by the caller (api.cu) with the driver's encoder.
 struct GemmMaps {
     CUtensorMap x;   // bf16 [M][K], box 64 (k) x BN (tokens), 128-byte swizzle

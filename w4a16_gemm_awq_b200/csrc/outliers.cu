@@ -1,0 +1,299 @@
+// outliers.cu -- dense-and-sparse split of a weight matrix on the GPU.
+//
+// [SqueezeLLM article, section 2.2: a small set of sensitive weights is kept in fp16 as a
+//  sparse matrix and removed from the dense part, W = W_dense + W_sparse; section 5.3: the
+//  sparsity ratio 0.45%.  The sensitivity is read as |w| * a_k with a_k the mean |x| of input
+//  channel k (the benchmark spec replaces the Hessian-based score, which needs gradients).]
+//
+// What it computes (the same rule as the CPU oracle):
+//   score(n, k) = fp32(|w(n, k)| * a_k)            (one IEEE multiply)
+//   key = (bits(score) << 32) | (0xFFFFFFFF - (n K + k))
+//   the nnz entries with the largest keys are the outliers: larger score first, and among
+//   equal scores the lower linear index first;
+//   W_dense = W with those entries set to 0;
+//   CSR: row_ptr [N+1], col_idx ascending within each row, values fp16(w * s_k) with
+//   s_k = max(float(pow(a_k, alpha)), 1e-4) (the AWQ scale, so the values live in the same
+//   scaled space as the packed dense part).
+//
+// Design: a radix select on the 32-bit score (non-negative floats order like their bit
+// patterns), then the ties at the threshold score are resolved in index order.
+//   1. Three histogram passes over digits of 12, 10 and 10 bits of the score.  Each pass
+//      counts only the entries whose higher digits equal the prefix found so far (shared-
+//      memory histogram per CTA, then global atomics).  After each pass one CTA scans the
+//      histogram from the top and finds the digit where the running count reaches the number
+//      still needed.  The result is the threshold score T and the number r of entries with
+//      score == T to take (1 <= r <= their count).
+//   2. A row pass counts, per row, the entries with score > T and those with score == T.
+//   3. One CTA scans the rows: the ties are taken in index order, so row n takes
+//      clamp(r - ties_before_row_n, 0, ties_in_row_n); row_ptr is the running sum of
+//      (greater + taken).
+//   4. A fill pass (one warp per row, columns in order) writes col_idx and values through a
+//      ballot/popc compaction, and W_dense.
+// Every pass streams W (and a) once; all control stays on the device, so the host issues the
+// whole sequence without waiting.
+#include "common.cuh"
+#include "internal.h"
+
+namespace w4a16 {
+
+constexpr int kSplitThreads = 256;
+constexpr int kSplitBins = 4096;  // the widest digit (12 bits)
+
+// Device-side state of the selection: the prefix found so far and the count still needed.
+struct SplitState {
+    uint32_t prefix;  // the score bits fixed so far (high digits), left-aligned
+    uint32_t need;    // entries still to take at or below the current prefix
+    uint32_t err;     // unused, keeps the struct 16 bytes
+    uint32_t pad;
+};
+
+// digit boundaries: bits [31:20], [19:10], [9:0]
+__device__ __forceinline__ int digit_shift(int level) { return level == 0 ? 20 : (level == 1 ? 10 : 0); }
+__device__ __forceinline__ int digit_bins(int level) { return level == 0 ? 4096 : 1024; }
+
+__device__ __forceinline__ uint32_t score_bits(float w, float a) { return __float_as_uint(__fmul_rn(fabsf(w), a)); }
+
+// Histogram of digit `level` over the entries whose higher digits equal state->prefix.
+__global__ void __launch_bounds__(kSplitThreads)
+split_hist_kernel(const float* __restrict__ W, const float* __restrict__ act, uint32_t N, uint32_t K, int level,
+                  const SplitState* __restrict__ state, unsigned* __restrict__ hist, unsigned* err) {
+    __shared__ unsigned h[kSplitBins];
+    const int bins = digit_bins(level), shift = digit_shift(level);
+    for (int i = threadIdx.x; i < bins; i += kSplitThreads) h[i] = 0;
+    __syncthreads();
+    const uint32_t prefix = level == 0 ? 0u : state->prefix;
+    const uint32_t hi_mask = level == 0 ? 0u : (0xFFFFFFFFu << (shift + 10));  // the digits above this one
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    bool bad = false;
+    // one warp per row, lanes along the row (coalesced, and a_k indexed directly)
+    for (uint32_t n = blockIdx.x * (kSplitThreads / 32) + warp; n < N; n += gridDim.x * (kSplitThreads / 32)) {
+        const float* row = W + (size_t)n * K;
+        for (uint32_t k = lane; k < K; k += 32) {
+            const float w = row[k];
+            const float a = act[k];
+            if (level == 0 && (!isfinite(w) || !(a >= 0.0f) || isinf(a))) bad = true;
+            const uint32_t b = score_bits(w, a);
+            if ((b & hi_mask) == prefix) atomicAdd(&h[(b >> shift) & (uint32_t)(bins - 1)], 1u);
+        }
+    }
+    if (bad) record_error(err, kErrValue);
+    __syncthreads();
+    for (int i = threadIdx.x; i < bins; i += kSplitThreads)
+        if (h[i]) atomicAdd(&hist[i], h[i]);
+}
+
+// One CTA: the digit d where the running count from the top reaches state->need; the prefix
+// gains d and need becomes need - (entries in higher digits).  Clears the histogram for the
+// next pass.
+__global__ void __launch_bounds__(1024)
+split_select_kernel(unsigned* __restrict__ hist, int level, SplitState* __restrict__ state) {
+    __shared__ unsigned part[1024];
+    __shared__ unsigned found_digit, found_above;
+    const int bins = digit_bins(level), shift = digit_shift(level);
+    const int per = bins / 1024;  // 4 or 1 bins per thread, taken from the top down
+    const int t = threadIdx.x;
+    // thread t owns bins [bins - (t+1) per, bins - t per): descending order across threads
+    unsigned c[4] = {0, 0, 0, 0};
+    unsigned sum = 0;
+    for (int j = 0; j < per; ++j) {
+        c[j] = hist[bins - 1 - (t * per + j)];
+        sum += c[j];
+    }
+    part[t] = sum;
+    if (t == 0) {
+        found_digit = 0xFFFFFFFFu;
+        found_above = 0;
+    }
+    __syncthreads();
+    // inclusive scan of part[] (counts from the top)
+    for (int off = 1; off < 1024; off <<= 1) {
+        const unsigned v = t >= off ? part[t - off] : 0u;
+        __syncthreads();
+        part[t] += v;
+        __syncthreads();
+    }
+    const unsigned need = state->need;
+    const unsigned before = t > 0 ? part[t - 1] : 0u;  // entries in bins above this thread's
+    if (before < need && part[t] >= need) {
+        unsigned run = before;
+        for (int j = 0; j < per; ++j) {
+            if (run + c[j] >= need) {
+                found_digit = (unsigned)(bins - 1 - (t * per + j));
+                found_above = run;
+                break;
+            }
+            run += c[j];
+        }
+    }
+    __syncthreads();
+    if (t == 0 && found_digit != 0xFFFFFFFFu) {
+        state->prefix = (level == 0 ? 0u : state->prefix) | (found_digit << shift);
+        state->need = need - found_above;
+    }
+    __syncthreads();
+    for (int i = t; i < bins; i += 1024) hist[i] = 0;
+}
+
+// Per row: entries with score > T and with score == T (T = state->prefix after 3 levels).
+__global__ void __launch_bounds__(kSplitThreads)
+split_rowcount_kernel(const float* __restrict__ W, const float* __restrict__ act, uint32_t N, uint32_t K,
+                      const SplitState* __restrict__ state, unsigned* __restrict__ gt, unsigned* __restrict__ ties) {
+    const uint32_t T = state->prefix;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (uint32_t n = blockIdx.x * (kSplitThreads / 32) + warp; n < N; n += gridDim.x * (kSplitThreads / 32)) {
+        unsigned g = 0, e = 0;
+        const float* row = W + (size_t)n * K;
+        for (uint32_t k = lane; k < K; k += 32) {
+            const uint32_t b = score_bits(row[k], act[k]);
+            g += b > T;
+            e += b == T;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            e += __shfl_xor_sync(0xffffffffu, e, o);
+        }
+        if (lane == 0) {
+            gt[n] = g;
+            ties[n] = e;
+        }
+    }
+}
+
+// One CTA: ties are taken in index order (row by row), row_ptr is the running sum.
+__global__ void __launch_bounds__(1024)
+split_scan_kernel(uint32_t N, const SplitState* __restrict__ state, const unsigned* __restrict__ gt,
+                  unsigned* __restrict__ ties_take, int32_t* __restrict__ row_ptr, unsigned* err) {
+    __shared__ unsigned s_tie[1024], s_cnt[1024];
+    __shared__ unsigned carry_tie, carry_cnt;
+    const unsigned r = state->need;
+    const int t = threadIdx.x;
+    if (t == 0) {
+        carry_tie = 0;
+        carry_cnt = 0;
+        row_ptr[0] = 0;
+    }
+    __syncthreads();
+    for (uint32_t base = 0; base < N; base += 1024) {
+        const uint32_t n = base + t;
+        const unsigned e = n < N ? ties_take[n] : 0u;  // ties in the row (rowcount wrote them here)
+        s_tie[t] = e;
+        __syncthreads();
+        for (int off = 1; off < 1024; off <<= 1) {
+            const unsigned v = t >= off ? s_tie[t - off] : 0u;
+            __syncthreads();
+            s_tie[t] += v;
+            __syncthreads();
+        }
+        const unsigned tie_before = carry_tie + s_tie[t] - e;
+        const unsigned take = tie_before >= r ? 0u : (r - tie_before < e ? r - tie_before : e);
+        const unsigned cnt = n < N ? gt[n] + take : 0u;
+        s_cnt[t] = cnt;
+        __syncthreads();
+        for (int off = 1; off < 1024; off <<= 1) {
+            const unsigned v = t >= off ? s_cnt[t - off] : 0u;
+            __syncthreads();
+            s_cnt[t] += v;
+            __syncthreads();
+        }
+        if (n < N) {
+            ties_take[n] = take;
+            row_ptr[n + 1] = (int32_t)(carry_cnt + s_cnt[t]);
+        }
+        __syncthreads();
+        if (t == 1023) {
+            carry_tie += s_tie[1023];
+            carry_cnt += s_cnt[1023];
+        }
+        __syncthreads();
+    }
+    (void)err;
+}
+
+// One warp per row: columns in order, chosen = score > T or (score == T and among the
+// row's first ties_take[n] ties).  Writes the CSR entries and W_dense.
+__global__ void __launch_bounds__(kSplitThreads)
+split_fill_kernel(const float* __restrict__ W, const float* __restrict__ act, float alpha, uint32_t N, uint32_t K,
+                  uint32_t nnz, const SplitState* __restrict__ state, const unsigned* __restrict__ ties_take,
+                  const int32_t* __restrict__ row_ptr, float* __restrict__ W_dense, int32_t* __restrict__ col_idx,
+                  uint16_t* __restrict__ values, unsigned* err) {
+    const uint32_t T = state->prefix;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    bool bad = false;
+    for (uint32_t n = blockIdx.x * (kSplitThreads / 32) + warp; n < N; n += gridDim.x * (kSplitThreads / 32)) {
+        const float* row = W + (size_t)n * K;
+        float* drow = W_dense + (size_t)n * K;
+        uint32_t pos = (uint32_t)row_ptr[n];
+        const unsigned take = ties_take[n];
+        unsigned ties_seen = 0;
+        for (uint32_t k0 = 0; k0 < K; k0 += 32) {
+            const uint32_t k = k0 + lane;
+            const bool in = k < K;
+            const float w = in ? row[k] : 0.0f;
+            const float a = in ? act[k] : 0.0f;
+            const uint32_t b = score_bits(w, a);
+            const bool tie = in && b == T;
+            const unsigned tie_mask = __ballot_sync(0xffffffffu, tie);
+            const unsigned tie_rank = ties_seen + __popc(tie_mask & ((1u << lane) - 1u));
+            const bool chosen = in && (b > T || (tie && tie_rank < take));
+            const unsigned ch_mask = __ballot_sync(0xffffffffu, chosen);
+            if (chosen) {
+                const uint32_t at = pos + __popc(ch_mask & ((1u << lane) - 1u));
+                if (at < nnz) {  // always true (the counts are exact); never write past the arrays
+                    const float p = (float)pow((double)a, (double)alpha);
+                    const float s = p > 1e-4f ? p : 1e-4f;
+                    const __half hv = __float2half_rn(__fmul_rn(w, s));
+                    if (isinf(__half2float(hv))) bad = true;
+                    col_idx[at] = (int32_t)k;
+                    values[at] = __half_as_ushort(hv);
+                } else {
+                    record_error(err, kErrShape);
+                }
+            }
+            if (in) drow[k] = chosen ? 0.0f : w;
+            pos += __popc(ch_mask);
+            ties_seen += __popc(tie_mask);
+        }
+    }
+    if (bad) record_error(err, kErrValue);
+}
+
+// The selection state starts at (prefix 0, need nnz) and the histogram at zero.  A kernel
+// (not a host-to-device copy) sets them, so the whole split can be captured in a CUDA graph.
+__global__ void split_init_kernel(SplitState* state, unsigned* hist, uint32_t nnz) {
+    if (threadIdx.x == 0) {
+        state->prefix = 0u;
+        state->need = nnz;
+        state->err = 0u;
+        state->pad = 0u;
+    }
+    for (int i = threadIdx.x; i < kSplitBins; i += blockDim.x) hist[i] = 0;
+}
+
+size_t split_workspace_bytes(int64_t N) {
+    return 256 + (size_t)kSplitBins * 4 + 3 * (((size_t)N * 4 + 255) / 256) * 256;
+}
+
+cudaError_t launch_split_outliers(const float* W, const float* act, float alpha, uint32_t N, uint32_t K, uint32_t nnz,
+                                  float* W_dense, int32_t* row_ptr, int32_t* col_idx, uint16_t* values,
+                                  void* workspace, int num_sms, unsigned* err, cudaStream_t stream) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    SplitState* state = reinterpret_cast<SplitState*>(ws);
+    unsigned* hist = reinterpret_cast<unsigned*>(ws + 256);
+    const size_t row_bytes = (((size_t)N * 4 + 255) / 256) * 256;
+    unsigned* gt = reinterpret_cast<unsigned*>(ws + 256 + kSplitBins * 4);
+    unsigned* ties = reinterpret_cast<unsigned*>(ws + 256 + kSplitBins * 4 + row_bytes);
+    split_init_kernel<<<1, 1024, 0, stream>>>(state, hist, nnz);
+    const int grid = 4 * num_sms;
+    for (int level = 0; level < 3; ++level) {
+        split_hist_kernel<<<grid, kSplitThreads, 0, stream>>>(W, act, N, K, level, state, hist, err);
+        split_select_kernel<<<1, 1024, 0, stream>>>(hist, level, state);
+    }
+    split_rowcount_kernel<<<grid, kSplitThreads, 0, stream>>>(W, act, N, K, state, gt, ties);
+    split_scan_kernel<<<1, 1024, 0, stream>>>(N, state, gt, ties, row_ptr, err);
+    split_fill_kernel<<<grid, kSplitThreads, 0, stream>>>(W, act, alpha, N, K, nnz, state, ties, row_ptr, W_dense,
+                                                         col_idx, values, err);
+    return cudaGetLastError();
+}
+
+}  // namespace w4a16
