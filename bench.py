@@ -423,6 +423,30 @@ def run_gpu(args, world, rank, local):
                  "layers 5120x5120 and 5120x13824, 0.45% fp16 outliers", "frac_of_hbm": sb / sms_ / 1e6 / pk["hbm_gbs"],
                  "per_layer": per_split}
 
+    # AWQ alpha search: an 11-point grid on the 4096x4096 layer with 128 calibration tokens
+    # (quantize + fold + W4A16 GEMM + error per alpha, one fp32 reference product)
+    ainfo = None
+    if not args.skip_search:
+        K, N, Mc = 4096, 4096, 128
+        L = workloads.make_layer(workloads.seed_of(1, 1), K=K, N=N)
+        W = torch.from_numpy(L.W).cuda()
+        act = torch.from_numpy(L.act_absmean).cuda()
+        xc = torch.from_numpy(workloads.make_activations(99, Mc, L.mult, alpha=0.0).view(np.int16)).view(
+            torch.bfloat16).cuda()
+        grid = [i / 10 for i in range(11)]
+        wsa = torch.empty(w4.lib().awq_search_alpha_workspace_bytes(Mc, N, K, len(grid)), dtype=torch.uint8,
+                          device="cuda")
+        w4.awq_search_alpha(W, act, xc, grid, workspace=wsa)
+        reps = 5
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            err, best = w4.awq_search_alpha(W, act, xc, grid, workspace=wsa)
+        ms_total = (time.perf_counter() - t0) / reps * 1e3
+        ainfo = {"value": ms_total, "unit": "ms per search", "ms_per_alpha": ms_total / len(grid),
+                 "workload": f"awq_search_alpha, K x N = {K}x{N}, {Mc} calibration tokens, alpha in 0..1 step 0.1",
+                 "best_alpha": grid[best], "errors": [round(e, 6) for e in err]}
+        del W, act, xc, wsa
+
     if rank != 0:
         return
     cpu = None
@@ -450,6 +474,7 @@ def run_gpu(args, world, rank, local):
         "gemm": gemm,
         "quantize": qinfo,
         "outlier_split": sinfo,
+        "alpha_search": ainfo,
     }
     print(json.dumps(line), flush=True)
 
@@ -529,6 +554,7 @@ def main():
     ap.add_argument("--skip-quant", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-split", action="store_true")
+    ap.add_argument("--skip-search", action="store_true")
     ap.add_argument("--case", choices=["gemv", "gemm", "quantize"], help="time one kernel on one layer (ncu)")
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)

@@ -218,6 +218,29 @@ w4a16_status awq_split_outliers(const float* W, const float* act_absmean, float 
                                 uint16_t* values, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * awq_search_alpha -- the AWQ scale search over a grid of exponents, on the GPU.
+ * [AWQ (MLSys 2024) translation, section 3.2: the per-channel scaling factor is searched so
+ *  that the quantized layer's output on calibration activations stays closest to the
+ *  full-precision output; with s = a^alpha the search runs over alpha.]
+ * For every alpha[i] it quantizes W with awq_quantize_g128, folds the scales into the
+ * calibration activations (x' = bf16(x / s_k), IEEE division), runs the W4A16 product of this
+ * library (the GEMV for M <= 16, else the GEMM) and scores it against the fp32 product:
+ *     errors[i] = sum (y_q - y_ref)^2 / sum y_ref^2,   y_ref = x . W^T,
+ * and *best is the index of the smallest error (the first one on ties).
+ *   W fp32 [N][K], act_absmean fp32 [K], x_calib bf16 [M][K]: device inputs (x_calib are the
+ *   activations before the fold).  alphas [n_alpha] (1..64 values, each >= 0 and finite),
+ *   errors [n_alpha] and best: HOST memory.  workspace: device scratch of
+ *   awq_search_alpha_workspace_bytes(M, N, K, n_alpha) bytes, 256-byte aligned.
+ * N % 128 == 0, K % 1024 == 0, 1 <= M <= 65535.
+ * The call is synchronous on `stream` (it reads the errors back) and it also reports any
+ * problem the kernels recorded (as w4a16_check_device_status does).
+ */
+size_t awq_search_alpha_workspace_bytes(int64_t M, int64_t N, int64_t K, int n_alpha);
+w4a16_status awq_search_alpha(const float* W, const float* act_absmean, const uint16_t* x_calib, int64_t M,
+                              int64_t N, int64_t K, const float* alphas, int n_alpha, float* errors, int* best,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * w4a16_selftest_timeout -- launch a one-thread kernel whose pipeline wait can never
  * complete and whose limit is limit_ns nanoseconds (0 .. 1e10; else W4A16_ERR_VALUE).  The
  * wait runs out through the same bounded-wait loop the kernels use, the kernel records a

@@ -67,6 +67,7 @@ def _L():
             "oracle_linear_at": ([P, I64, I64, P, P, P, I64, P, P, P, I64, P, P, I64, P, P],
                                  ctypes.c_int),
             "oracle_split_outliers": ([P, P, F, I64, I64, I64, P, P, P, P], ctypes.c_int),
+            "oracle_awq_search_alpha": ([P, P, P, I64, I64, I64, P, I64, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(_lib, name)
@@ -209,3 +210,18 @@ def split_outliers(W, act_absmean, alpha: float, nnz: int):
     _check(_L().oracle_split_outliers(_p(W), _p(a), ctypes.c_float(alpha), N, K, nnz, _p(Wd), _p(rp),
                                       _p(ci), _p(v)), "split_outliers")
     return Wd, rp, ci[:nnz], v[:nnz]
+
+
+def awq_search_alpha(W, act_absmean, x_bf16_bits, alphas):
+    """Relative squared output error of the quantized layer for every alpha of the grid
+    (see oracle_awq_search_alpha).  Returns float64 [len(alphas)]."""
+    W = _c(W, np.float32)
+    a = _c(act_absmean, np.float32)
+    x = _c(x_bf16_bits, np.uint16)
+    al = _c(alphas, np.float32)
+    N, K = W.shape
+    M = x.shape[0]
+    err = np.zeros(al.size, np.float64)
+    _check(_L().oracle_awq_search_alpha(_p(W), _p(a), _p(x), M, N, K, _p(al), al.size, _p(err)),
+           "awq_search_alpha")
+    return err

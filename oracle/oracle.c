@@ -269,7 +269,6 @@ int oracle_dequant(const uint32_t* qweight, const uint16_t* scales, const uint32
     if (!qweight || !scales || !zeros || !deq) return ORACLE_ERR_NULL;
     int st = check_qshape(N, K);
     if (st) return st;
-    const int64_t G = K / GROUP;
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
         for (int64_t k = 0; k < K; ++k) {
@@ -372,6 +371,64 @@ int oracle_linear_at(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qw
         one_output(x, K, N, qweight, scales, zeros, row_ptr, col_idx, values, m_idx[p], n_idx[p],
                    &y[p], yabs ? &yabs[p] : NULL);
     return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------------------
+ * AWQ scale search [AWQ (MLSys 2024) translation, section 3.2: the per-channel scaling
+ * factor is searched so that the quantized layer's output on calibration activations
+ * stays closest to the full-precision output; with the closed form s = a^alpha the search
+ * is over the exponent alpha].  For every alpha of the grid:
+ *   s_k    = max(float(pow(a_k, alpha)), 1e-4)
+ *   Q      = awq_quantize_g128(W, a, alpha)            (W * s, g128 RTN, packed)
+ *   x'_mk  = bf16(float(x_mk) / s_k)                   (the runtime activation, 1/s folded in)
+ *   yq_mn  = bf16(float(sum_k x'_mk deq_nk))           (the quantized layer, output in bf16)
+ *   err    = sum_mn (yq_mn - yr_mn)^2 / sum_mn yr_mn^2,  yr_mn = sum_k x_mk W_nk  (double)
+ * ---------------------------------------------------------------------------------- */
+int oracle_awq_search_alpha(const float* W, const float* act_absmean, const uint16_t* x, int64_t M,
+                            int64_t N, int64_t K, const float* alphas, int64_t n_alpha,
+                            double* errors) {
+    if (!W || !act_absmean || !x || !alphas || !errors) return ORACLE_ERR_NULL;
+    if (M <= 0 || n_alpha <= 0) return ORACLE_ERR_SHAPE;
+    int st = check_qshape(N, K);
+    if (st) return st;
+    double* yr = (double*)malloc(sizeof(double) * (size_t)(M * N));
+    double* y = (double*)malloc(sizeof(double) * (size_t)(M * N));
+    uint16_t* xs = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(M * K));
+    uint32_t* qw = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)(N * K / 8));
+    uint16_t* sc = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(N * K / 128));
+    uint32_t* z = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)(N * K / 1024));
+    float* s = (float*)malloc(sizeof(float) * (size_t)K);
+    if (!yr || !y || !xs || !qw || !sc || !z || !s) st = ORACLE_ERR_VALUE;
+    /* the full-precision output */
+    double ref2 = 0.0;
+    if (!st) {
+#pragma omp parallel for collapse(2) schedule(static)
+        for (int64_t m = 0; m < M; ++m)
+            for (int64_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k)
+                    acc += (double)oracle_bf16_to_f32(x[m * K + k]) * (double)W[n * K + k];
+                yr[m * N + n] = acc;
+            }
+        for (int64_t i = 0; i < M * N; ++i) ref2 += yr[i] * yr[i];
+    }
+    for (int64_t a = 0; a < n_alpha && !st; ++a) {
+        st = oracle_awq_quantize_g128(W, act_absmean, alphas[a], N, K, qw, sc, z, s);
+        if (st) break;
+        for (int64_t m = 0; m < M; ++m)
+            for (int64_t k = 0; k < K; ++k)
+                xs[m * K + k] = oracle_f32_to_bf16(oracle_bf16_to_f32(x[m * K + k]) / s[k]);
+        st = oracle_linear(xs, M, K, qw, sc, z, N, NULL, NULL, NULL, 0, y, NULL);
+        if (st) break;
+        double e2 = 0.0;
+        for (int64_t i = 0; i < M * N; ++i) {
+            const double yq = (double)oracle_bf16_to_f32(oracle_f32_to_bf16((float)y[i]));
+            e2 += (yq - yr[i]) * (yq - yr[i]);
+        }
+        errors[a] = ref2 > 0.0 ? e2 / ref2 : e2;
+    }
+    free(yr); free(y); free(xs); free(qw); free(sc); free(z); free(s);
+    return st;
 }
 
 /* ------------------------------------------------------------------------------------

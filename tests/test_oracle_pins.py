@@ -447,3 +447,62 @@ def test_split_outliers_edge_counts(orc):
     Wd, rp, ci, v = orc.split_outliers(W, a, 0.0, N * K)
     assert np.all(Wd == 0) and np.array_equal(rp, np.arange(N + 1) * K)
     assert np.array_equal(v, W.ravel().astype(np.float16).view(np.uint16))
+
+
+# ---- AWQ alpha search (oracle_awq_search_alpha) ------------------------------------------
+
+def _raw_activations(seed, M, mult):
+    """Calibration activations before the 1/s fold: N(0,1) * m_k."""
+    return workloads.make_activations(seed, M, mult, alpha=0.0)
+
+
+def test_search_power_of_two_invariance(orc):
+    """a -> 4a multiplies s by 4^alpha = 1, 2, 4 for alpha = 0, 0.5, 1: W*s, the group scales
+    and x/s all change by exact powers of two, so every error is unchanged bit for bit."""
+    L = workloads.make_layer(21, K=1024, N=128)
+    x = _raw_activations(21, 6, L.mult)
+    alphas = [0.0, 0.5, 1.0]
+    e1 = orc.awq_search_alpha(L.W, L.act_absmean, x, alphas)
+    e4 = orc.awq_search_alpha(L.W, (L.act_absmean * np.float32(4.0)).astype(np.float32), x, alphas)
+    assert np.array_equal(e1, e4)
+    assert np.all(np.isfinite(e1)) and np.all(e1 > 0)
+
+
+def test_search_alpha0_is_plain_rtn(orc):
+    """alpha = 0 is plain RTN of W with x unchanged: recompute that error from the dequantized
+    matrix with numpy and torch's bf16 rounding, independently of the oracle's product."""
+    import torch
+    L = workloads.make_layer(22, K=2048, N=128)
+    x = _raw_activations(22, 4, L.mult)
+    e = orc.awq_search_alpha(L.W, L.act_absmean, x, [0.0])[0]
+    qw, sc, z = orc.quantize_with_scales(L.W, np.ones(2048, np.float32))
+    deq = orc.dequant(qw, sc, z, 128, 2048).astype(np.float64)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    yq = xf @ deq.T
+    yq = torch.from_numpy(yq.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    yr = xf @ L.W.astype(np.float64).T
+    want = ((yq - yr) ** 2).sum() / (yr ** 2).sum()
+    assert e == pytest.approx(want, rel=1e-9)
+
+
+def test_search_scaling_protects_a_salient_channel(orc):
+    """One input channel carries 100x larger activations.  Without scaling its weights are
+    quantized with their group's step like all others and the error is dominated by that
+    channel; alpha = 0.5 scales them up by ~10, so they set their group's range and the
+    output error drops -- the effect the AWQ translation describes in section 3.2."""
+    rng = np.random.default_rng(23)
+    N, K = 128, 1024
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    mult = np.ones(K, np.float32)
+    mult[0] = 100.0
+    x = workloads.uniform_bf16(24, (8, K))
+    xf = (x.astype(np.uint32) << 16).view(np.float32) * mult
+    x = torch_bf16(xf)
+    act = np.abs(xf).mean(axis=0).astype(np.float32) + np.float32(1e-3)
+    e = orc.awq_search_alpha(W, act, x, [0.0, 0.5])
+    assert e[1] < 0.5 * e[0]
+
+
+def torch_bf16(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)

@@ -71,11 +71,14 @@ def lib() -> ctypes.CDLL:
         L.awq_split_outliers.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P, ctypes.c_size_t, P]
         L.awq_split_outliers_workspace_bytes.argtypes = [I64, I64]
         L.awq_split_outliers_workspace_bytes.restype = ctypes.c_size_t
+        L.awq_search_alpha.argtypes = [P, P, P, I64, I64, I64, P, ctypes.c_int, P, P, P, ctypes.c_size_t, P]
+        L.awq_search_alpha_workspace_bytes.argtypes = [I64, I64, I64, ctypes.c_int]
+        L.awq_search_alpha_workspace_bytes.restype = ctypes.c_size_t
         L.w4a16_status_string.argtypes = [ctypes.c_int]
         L.w4a16_status_string.restype = ctypes.c_char_p
         L.w4a16_version.argtypes = []
         for name in ("awq_quantize_g128", "w4a16_linear", "w4a16_gemv", "w4a16_gemm", "w4a16_check_device_status",
-                     "w4a16_selftest_timeout", "awq_split_outliers", "w4a16_version"):
+                     "w4a16_selftest_timeout", "awq_split_outliers", "awq_search_alpha", "w4a16_version"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -205,6 +208,24 @@ def awq_split_outliers(W, act_absmean, alpha: float, nnz: int, out=None, workspa
                                     _ptr(rp), _ptr(ci), _ptr(vals), _ptr(workspace), workspace.numel(),
                                     _stream(dev)), "awq_split_outliers")
     return Wd, (rp, ci[:nnz], vals[:nnz])
+
+
+def awq_search_alpha(W, act_absmean, x_calib, alphas, workspace=None):
+    """AWQ scale search on the GPU.  W fp32 [N][K], act_absmean fp32 [K], x_calib bf16 [M][K]
+    (cuda), alphas a sequence of floats.  Returns (errors list, best index); synchronous."""
+    assert W.is_cuda and W.dtype == torch.float32 and W.is_contiguous() and x_calib.dtype == torch.bfloat16
+    N, K = W.shape
+    M = x_calib.shape[0]
+    al = (ctypes.c_float * len(alphas))(*[float(a) for a in alphas])
+    err = (ctypes.c_float * len(alphas))()
+    best = ctypes.c_int(-1)
+    nbytes = lib().awq_search_alpha_workspace_bytes(M, N, K, len(alphas))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=W.device)
+    _check(lib().awq_search_alpha(_ptr(W), _ptr(act_absmean), _ptr(x_calib), M, N, K, al, len(alphas), err,
+                                  ctypes.byref(best), _ptr(workspace), workspace.numel(), _stream(W.device)),
+           "awq_search_alpha")
+    return list(err), best.value
 
 
 def selftest_timeout(limit_ns: int, stream=None) -> None:

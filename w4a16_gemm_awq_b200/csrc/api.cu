@@ -217,6 +217,31 @@ w4a16_status run_gemm(const LinearArgs& a, cudaStream_t stream) {
                                  (int)a.N, (int)a.K, bn, d->num_sms, d->status, stream));
 }
 
+// ---------------------------------------------------------------------------------------
+// AWQ alpha search: layout of the workspace (every part 256-byte aligned).
+struct SearchLayout {
+    size_t qw, sc, z, s, xs, yq, yref, acc, gemv, total;
+};
+
+SearchLayout search_layout(int64_t M, int64_t N, int64_t K, int n_alpha, int num_sms) {
+    auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+    SearchLayout L{};
+    size_t off = 0;
+    L.qw = off; off += up((size_t)N * K / 2);
+    L.sc = off; off += up((size_t)N * (K / 128) * 2);
+    L.z = off; off += up((size_t)N * (K / 1024) * 4);
+    L.s = off; off += up((size_t)K * 4);
+    L.xs = off; off += up((size_t)M * K * 2);
+    L.yq = off; off += up((size_t)M * N * 2);
+    L.yref = off; off += up((size_t)M * N * 4);
+    L.acc = off; off += up((size_t)(n_alpha + 1) * 8);
+    L.gemv = off; off += M <= 16 ? up(gemv_workspace_bytes((int)N, num_sms)) : 0;
+    L.total = off;
+    return L;
+}
+
+constexpr int kMaxAlphas = 64;
+
 }  // namespace
 }  // namespace w4a16
 
@@ -338,6 +363,81 @@ w4a16_status awq_split_outliers(const float* W, const float* act_absmean, float 
     if (workspace_bytes < split_workspace_bytes(N)) return W4A16_ERR_SHAPE;
     return from_cuda(launch_split_outliers(W, act_absmean, alpha, (uint32_t)N, (uint32_t)K, (uint32_t)nnz, W_dense,
                                            row_ptr, col_idx, values, workspace, d->num_sms, d->status, s));
+}
+
+size_t awq_search_alpha_workspace_bytes(int64_t M, int64_t N, int64_t K, int n_alpha) {
+    if (M < 1 || M > 65535 || N < 128 || N % 128 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK ||
+        n_alpha < 1 || n_alpha > kMaxAlphas)
+        return 0;
+    DeviceInfo* d = nullptr;
+    if (device_info(&d) != W4A16_OK) return 0;
+    return search_layout(M, N, K, n_alpha, d->num_sms).total;
+}
+
+w4a16_status awq_search_alpha(const float* W, const float* act_absmean, const uint16_t* x_calib, int64_t M,
+                              int64_t N, int64_t K, const float* alphas, int n_alpha, float* errors, int* best,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    if (!W || !act_absmean || !x_calib || !alphas || !errors || !best || !workspace) return W4A16_ERR_NULL;
+    if (M < 1 || M > 65535 || N < 128 || N % 128 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK ||
+        n_alpha < 1 || n_alpha > kMaxAlphas)
+        return W4A16_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(act_absmean, 16) || !aligned(x_calib, 16) || !aligned(workspace, 256))
+        return W4A16_ERR_ALIGN;
+    for (int i = 0; i < n_alpha; ++i)
+        if (!std::isfinite(alphas[i]) || alphas[i] < 0.0f) return W4A16_ERR_VALUE;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    const SearchLayout L = search_layout(M, N, K, n_alpha, d->num_sms);
+    if (workspace_bytes < L.total) return W4A16_ERR_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint32_t* qw = reinterpret_cast<uint32_t*>(ws + L.qw);
+    uint16_t* sc = reinterpret_cast<uint16_t*>(ws + L.sc);
+    uint32_t* z = reinterpret_cast<uint32_t*>(ws + L.z);
+    float* sv = reinterpret_cast<float*>(ws + L.s);
+    uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
+    uint16_t* yq = reinterpret_cast<uint16_t*>(ws + L.yq);
+    float* yref = reinterpret_cast<float*>(ws + L.yref);
+    double* acc = reinterpret_cast<double*>(ws + L.acc);  // [0] = sum yref^2, [1 + a] = error sums
+    // the error sums start at zero; so does the GEMV's workspace
+    if (cudaMemsetAsync(acc, 0, (size_t)(n_alpha + 1) * 8, s) != cudaSuccess) return W4A16_ERR_CUDA;
+    if (M <= 16 && cudaMemsetAsync(ws + L.gemv, 0, L.total - L.gemv, s) != cudaSuccess) return W4A16_ERR_CUDA;
+    st = from_cuda(launch_search_ref(x_calib, W, yref, (int)M, (int)N, (int)K, s));
+    for (int i = 0; i < n_alpha && st == W4A16_OK; ++i) {
+        st = from_cuda(launch_awq_quantize(W, act_absmean, alphas[i], (int)N, (int)K, qw, sc, z, sv, d->status, s));
+        if (st != W4A16_OK) break;
+        st = from_cuda(launch_search_fold(x_calib, sv, xs, (int)M, (int)K, s));
+        if (st != W4A16_OK) break;
+        LinearArgs a;
+        st = validate_linear(xs, qw, sc, z, nullptr, yq, M, N, K, &a);
+        if (st != W4A16_OK) break;
+        if (M <= 16) {
+            a.workspace = ws + L.gemv;
+            a.workspace_bytes = L.total - L.gemv;
+            st = run_gemv(a, s);
+        } else {
+            st = run_gemm(a, s);
+        }
+        if (st != W4A16_OK) break;
+        st = from_cuda(launch_search_err(yq, yref, (long long)(M * N), acc + 1 + i, i == 0 ? acc : nullptr,
+                                         d->num_sms, s));
+    }
+    if (st != W4A16_OK) return st;
+    double host[kMaxAlphas + 1];
+    if (cudaMemcpyAsync(host, acc, (size_t)(n_alpha + 1) * 8, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return W4A16_ERR_CUDA;
+    // any problem a kernel recorded (bad values, a timeout) makes the result invalid
+    st = w4a16_check_device_status(stream);
+    if (st != W4A16_OK) return st;
+    int bi = 0;
+    for (int i = 0; i < n_alpha; ++i) {
+        errors[i] = (float)(host[0] > 0.0 ? host[1 + i] / host[0] : host[1 + i]);
+        if (errors[i] < errors[bi]) bi = i;
+    }
+    *best = bi;
+    return W4A16_OK;
 }
 
 w4a16_status w4a16_selftest_timeout(int64_t limit_ns, void* stream) {

@@ -41,6 +41,12 @@ cudaError_t launch_split_outliers(const float* W, const float* act, float alpha,
                                   float* W_dense, int32_t* row_ptr, int32_t* col_idx, uint16_t* values,
                                   void* workspace, int num_sms, unsigned* err, cudaStream_t stream);
 
+// Kernels of the AWQ alpha search (see search.cu).
+cudaError_t launch_search_ref(const uint16_t* x, const float* W, float* yref, int M, int N, int K, cudaStream_t stream);
+cudaError_t launch_search_fold(const uint16_t* x, const float* s, uint16_t* xs, int M, int K, cudaStream_t stream);
+cudaError_t launch_search_err(const uint16_t* yq, const float* yref, long long count, double* acc, double* ref2,
+                              int num_sms, cudaStream_t stream);
+
 // A kernel whose only wait never completes: it gives up after limit_ns and records
 // kErrTimeout (tests the bounded-wait path without any fault).
 cudaError_t launch_selftest_timeout(unsigned long long limit_ns, unsigned* err, cudaStream_t stream);
