@@ -241,6 +241,18 @@ w4a16_status awq_search_alpha(const float* W, const float* act_absmean, const ui
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * awq_fold_activations -- x_out[m][k] = bf16(float(x[m][k]) / s[k]) (IEEE division, then
+ * round-to-nearest-even): the runtime activation x' = x / s that the linear entry points
+ * take, for callers that cannot fold 1/s into the preceding operator.
+ * [AWQ (MLSys 2024) translation, section 3.2: the weights are multiplied by s and the
+ *  activations divided by it.]
+ *   x bf16 [M][K], s fp32 [K] (e.g. s_out of awq_quantize_g128), x_out bf16 [M][K]: device.
+ *   1 <= M <= 65535, 1 <= K <= 2^20.  x_out may alias x.
+ */
+w4a16_status awq_fold_activations(const uint16_t* x, const float* s, uint16_t* x_out, int64_t M, int64_t K,
+                                  void* stream);
+
+/*
  * w4a16_selftest_timeout -- launch a one-thread kernel whose pipeline wait can never
  * complete and whose limit is limit_ns nanoseconds (0 .. 1e10; else W4A16_ERR_VALUE).  The
  * wait runs out through the same bounded-wait loop the kernels use, the kernel records a

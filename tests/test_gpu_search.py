@@ -69,3 +69,15 @@ def test_search_argument_errors():
     with pytest.raises(w4.W4A16Error) as e:
         w4.awq_search_alpha(W, a, x, [0.5] * 65)
     assert e.value.code == w4.ERR_SHAPE
+
+
+def test_fold_activations_bit_exact(orc):
+    """x' = bf16(x / s) with IEEE division: bit-exact against the oracle's conversions."""
+    L = workloads.make_layer(41, K=2048, N=128)
+    x = raw_x(41, 5, L.mult)
+    s = orc.awq_scales(L.act_absmean, 0.5)
+    got = w4.awq_fold_activations(dev_bf16(x), dev_f32(s)).view(torch.int16).cpu().numpy().view(np.uint16)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    want = np.array([[orc.f32_to_bf16_bits(float(np.float32(xf[m, k]) / s[k])) for k in range(2048)]
+                     for m in range(5)], np.uint16)
+    assert np.array_equal(got, want)

@@ -74,11 +74,12 @@ def lib() -> ctypes.CDLL:
         L.awq_search_alpha.argtypes = [P, P, P, I64, I64, I64, P, ctypes.c_int, P, P, P, ctypes.c_size_t, P]
         L.awq_search_alpha_workspace_bytes.argtypes = [I64, I64, I64, ctypes.c_int]
         L.awq_search_alpha_workspace_bytes.restype = ctypes.c_size_t
+        L.awq_fold_activations.argtypes = [P, P, P, I64, I64, P]
         L.w4a16_status_string.argtypes = [ctypes.c_int]
         L.w4a16_status_string.restype = ctypes.c_char_p
         L.w4a16_version.argtypes = []
         for name in ("awq_quantize_g128", "w4a16_linear", "w4a16_gemv", "w4a16_gemm", "w4a16_check_device_status",
-                     "w4a16_selftest_timeout", "awq_split_outliers", "awq_search_alpha", "w4a16_version"):
+                     "w4a16_selftest_timeout", "awq_split_outliers", "awq_search_alpha", "awq_fold_activations", "w4a16_version"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -226,6 +227,15 @@ def awq_search_alpha(W, act_absmean, x_calib, alphas, workspace=None):
                                   ctypes.byref(best), _ptr(workspace), workspace.numel(), _stream(W.device)),
            "awq_search_alpha")
     return list(err), best.value
+
+
+def awq_fold_activations(x, s, out=None):
+    """x' = bf16(x / s) for bf16 x [M][K] and fp32 s [K] (cuda)."""
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and s.dtype == torch.float32
+    M, K = x.shape
+    out = torch.empty_like(x) if out is None else out
+    _check(lib().awq_fold_activations(_ptr(x), _ptr(s), _ptr(out), M, K, _stream(x.device)), "awq_fold_activations")
+    return out
 
 
 def selftest_timeout(limit_ns: int, stream=None) -> None:

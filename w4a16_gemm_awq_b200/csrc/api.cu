@@ -440,6 +440,16 @@ w4a16_status awq_search_alpha(const float* W, const float* act_absmean, const ui
     return W4A16_OK;
 }
 
+w4a16_status awq_fold_activations(const uint16_t* x, const float* s, uint16_t* x_out, int64_t M, int64_t K,
+                                  void* stream) {
+    if (!x || !s || !x_out) return W4A16_ERR_NULL;
+    if (M < 1 || M > 65535 || K < 1 || K > kMaxK) return W4A16_ERR_SHAPE;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    return from_cuda(launch_search_fold(x, s, x_out, (int)M, (int)K, static_cast<cudaStream_t>(stream)));
+}
+
 w4a16_status w4a16_selftest_timeout(int64_t limit_ns, void* stream) {
     if (limit_ns < 0 || limit_ns > 10000000000ll) return W4A16_ERR_VALUE;
     DeviceInfo* d = nullptr;
