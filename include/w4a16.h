@@ -155,6 +155,42 @@ w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16
                         int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/*
+ * Schedules of the decode GEMV.  Both stream every packed weight byte once; they differ in
+ * how the work is spread over the SMs and how row blocks split along K are summed.
+ *   STREAM_K  one persistent CTA per SM takes an equal contiguous range of (row block,
+ *             512-k) units.  A row block split between CTAs is completed through fp32
+ *             partial tiles and a counter in the workspace; the last CTA to finish sums.
+ *   CLUSTER   thread-block clusters of 2 to 8 CTAs.  Each cluster takes whole row blocks;
+ *             its CTAs split every row block along K and sum their tiles through
+ *             distributed shared memory.  Suits shapes with few row blocks (N / 128 well
+ *             under the SM count), where the workspace exchange would dominate.
+ *   AUTO      the library's choice for the shape and the current device.
+ * Results of different schedules may differ in the last bit (summation order); a given
+ * schedule gives the same bits on every call.
+ */
+typedef enum {
+    W4A16_GEMV_AUTO = 0,
+    W4A16_GEMV_STREAM_K = 1,
+    W4A16_GEMV_CLUSTER = 2
+} w4a16_gemv_schedule;
+
+/* w4a16_gemv_ex -- w4a16_gemv with an explicit schedule (w4a16_gemv uses AUTO).  The
+ * workspace is required for every schedule.  UNSUPPORTED when the schedule cannot run this
+ * shape on the current device (CLUSTER needs K >= 1024 and a cluster launch the device
+ * can hold). */
+w4a16_status w4a16_gemv_ex(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                           const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
+                           int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                           int schedule, void* stream);
+
+/* w4a16_gemv_plan -- the launch that w4a16_gemv_ex(schedule) would make on the current
+ * device, without launching: *resolved = STREAM_K or CLUSTER, *cluster_size = CTAs per
+ * cluster (0 for STREAM_K), *ctas = CTAs of the grid.  Any output pointer may be NULL.
+ * SHAPE for invalid sizes (as w4a16_gemv), UNSUPPORTED as w4a16_gemv_ex. */
+w4a16_status w4a16_gemv_plan(int64_t M, int64_t N, int64_t K, int schedule, int* resolved,
+                             int* cluster_size, int* ctas);
+
 /* w4a16_gemm -- the tcgen05 tensor-core path of w4a16_linear, for any M >= 1.  Arguments
  * and result are as for w4a16_linear.  The workspace is not used (NULL and 0 are fine).
  * Weights are dequantized to bf16 inside the kernel.  When a CSR is given, its values are

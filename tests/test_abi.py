@@ -84,6 +84,24 @@ def test_gemv_rejects_large_m(L):
     assert _linear(L, "w4a16_gemv", M=17) == w4.ERR_SHAPE
 
 
+def test_gemv_schedule_validation(L):
+    def ex(schedule, **kw):
+        a = dict(x=FAKE, qw=FAKE, sc=FAKE, z=FAKE, y=FAKE, M=1, N=128, K=1024, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.w4a16_gemv_ex(ctypes.c_void_p(a["x"]), ctypes.c_void_p(a["qw"]), ctypes.c_void_p(a["sc"]),
+                               ctypes.c_void_p(a["z"]), None, ctypes.c_void_p(a["y"]), a["M"], a["N"], a["K"],
+                               ctypes.c_void_p(a["ws"]), a["wsb"], schedule, None)
+    assert ex(3) == w4.ERR_VALUE
+    assert ex(-1) == w4.ERR_VALUE
+    assert ex(w4.GEMV_CLUSTER, M=17) == w4.ERR_SHAPE
+    assert ex(w4.GEMV_STREAM_K, x=0) == w4.ERR_NULL
+    r = ctypes.c_int(-5)
+    assert L.w4a16_gemv_plan(1, 100, 1024, 0, ctypes.byref(r), None, None) == w4.ERR_SHAPE
+    assert L.w4a16_gemv_plan(17, 128, 1024, 0, None, None, None) == w4.ERR_SHAPE
+    assert L.w4a16_gemv_plan(1, 128, 1024, 9, None, None, None) == w4.ERR_VALUE
+    assert r.value == -5  # untouched on error
+
+
 def test_quantize_validation(L):
     def q(W=FAKE, a=FAKE, alpha=0.5, N=128, K=1024, qw=FAKE, sc=FAKE, z=FAKE, s=None):
         return L.awq_quantize_g128(ctypes.c_void_p(W), ctypes.c_void_p(a), ctypes.c_float(alpha), N, K,

@@ -103,6 +103,69 @@ def test_gemv_workspace_contract(orc):
     assert int(counters.count_nonzero()) == 0
 
 
+SCHEDULES = [w4.GEMV_STREAM_K, w4.GEMV_CLUSTER]
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES, ids=["stream_k", "cluster"])
+@pytest.mark.parametrize("K,N,M", [(1024, 128, 1), (3072, 384, 16), (4096, 2048, 9), (16384, 640, 5), (8192, 128, 3)])
+def test_gemv_schedules_full_output(orc, schedule, K, N, M):
+    """Both schedules against the oracle on every output, including shapes where a cluster
+    holds several row blocks and where a row block is split over the most CTAs."""
+    c = Case(orc, seed=K + 3 * N + M, K=K, N=N, M=M, csr=True)
+    d = c.device()
+    y = w4.w4a16_gemv_ex(d["x"], d["qweight"], d["scales"], d["zeros"], csr=d["csr"], schedule=schedule)
+    w4.check_device_status()
+    ref, ref_abs = c.reference(orc)
+    check_close(host_bf16_as_f64(y), ref, ref_abs, 0.0, depth(K), f"{K}x{N} M={M} schedule={schedule}",
+                xs_abs(c.x, c.sc))
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES, ids=["stream_k", "cluster"])
+@pytest.mark.parametrize("K,N,M", [(4096, 4096, 1), (4096, 6144, 16), (14336, 4096, 8), (4096, 28672, 4)])
+def test_gemv_schedules_sampled(orc, schedule, K, N, M):
+    c = Case(orc, seed=K + N + M + schedule, K=K, N=N, M=M, csr=False)
+    d = c.device()
+    y = host_bf16_as_f64(w4.w4a16_gemv_ex(d["x"], d["qweight"], d["scales"], d["zeros"], schedule=schedule))
+    w4.check_device_status()
+    m, n = c.sample(seed=K + schedule)
+    ref, ref_abs = c.reference_at(orc, m, n)
+    check_close(y[m, n], ref, ref_abs, 0.0, depth(K), f"{K}x{N} M={M} schedule={schedule}", xs_abs(c.x, c.sc, m, n))
+
+
+def test_gemv_plan_choices():
+    """Few row blocks: clusters of 2..8 CTAs that together cover at most the SMs; many row
+    blocks: stream-K.  A forced schedule is honoured."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    sched, cl, ctas = w4.gemv_plan(1, 4096, 4096)
+    assert sched == w4.GEMV_CLUSTER and 2 <= cl <= 8 and ctas % cl == 0 and ctas <= sms
+    assert w4.gemv_plan(1, 28672, 4096)[0] == w4.GEMV_STREAM_K
+    assert w4.gemv_plan(16, 4096, 4096, w4.GEMV_STREAM_K) == (w4.GEMV_STREAM_K, 0, min(sms, 32 * 8))
+    sched, cl, ctas = w4.gemv_plan(16, 57344, 8192, w4.GEMV_CLUSTER)
+    assert sched == w4.GEMV_CLUSTER and 2 <= cl <= 8 and ctas % cl == 0
+
+
+@pytest.mark.parametrize("schedule", [w4.GEMV_AUTO] + SCHEDULES, ids=["auto", "stream_k", "cluster"])
+@pytest.mark.parametrize("K,N,M", [(4096, 28672, 1), (4096, 28672, 16), (14336, 4096, 4), (4096, 4096, 1),
+                                   (4096, 6144, 9)])
+def test_gemv_repeat_bit_identical(schedule, K, N, M):
+    """Which CTA completes a split row block, and whether it fetched the other partial early,
+    depends on timing; y must not.  Repeated calls give the same bits and leave the
+    workspace counters at zero."""
+    g = torch.Generator(device="cuda").manual_seed(K + N + M)
+    qw = torch.randint(-2**31, 2**31 - 1, (N, K // 8), dtype=torch.int32, device="cuda", generator=g)
+    sc = (torch.rand(K // 128, N, device="cuda", generator=g) * 0.02 + 0.001).half().view(torch.int16)
+    z = torch.randint(-2**31, 2**31 - 1, (K // 128, N // 8), dtype=torch.int32, device="cuda", generator=g)
+    x = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    need = w4.workspace_bytes(M, N, K)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ys = [w4.w4a16_gemv_ex(x, qw, sc, z, workspace=ws, schedule=schedule) for _ in range(12)]
+    w4.check_device_status()
+    for y in ys[1:]:
+        assert torch.equal(ys[0].view(torch.int16), y.view(torch.int16))
+    counters = ws[need - 256 * ((N // 128 * 4 + 255) // 256):]
+    assert int(counters.count_nonzero()) == 0
+
+
 def test_linear_dispatches_to_gemv(orc):
     c = Case(orc, seed=12, K=2048, N=256, M=16, csr=True)
     d = c.device()

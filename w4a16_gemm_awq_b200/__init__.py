@@ -7,6 +7,8 @@ mirror the C ABI in include/w4a16.h:
   awq_quantize_g128(W, act_absmean, alpha)      -> (qweight, scales, zeros, s)
   w4a16_linear(x, qweight, scales, zeros, csr)  -> y      (any M)
   w4a16_gemv(...)                               -> y      (1 <= M <= 16)
+  w4a16_gemv_ex(..., schedule)                  -> y      (GEMV_AUTO, GEMV_STREAM_K or GEMV_CLUSTER)
+  gemv_plan(M, N, K, schedule)                  -> (schedule, cluster size, CTAs) the call would launch
   w4a16_gemm(...)                               -> y      (tcgen05 path, any M)
   workspace_bytes(M, N, K)                      -> bytes of zeroed device workspace a decode call needs
   check_device_status()                         -> raises W4A16Error on a recorded problem
@@ -31,6 +33,7 @@ LIB_PATH = os.path.join(_HERE, "libw4a16.so")
 STATUS = {0: "W4A16_OK", 1: "W4A16_ERR_NULL", 2: "W4A16_ERR_SHAPE", 3: "W4A16_ERR_ALIGN",
           4: "W4A16_ERR_VALUE", 5: "W4A16_ERR_CUDA", 6: "W4A16_ERR_TIMEOUT", 7: "W4A16_ERR_UNSUPPORTED"}
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_VALUE, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = range(8)
+GEMV_AUTO, GEMV_STREAM_K, GEMV_CLUSTER = range(3)
 
 
 class W4A16Error(RuntimeError):
@@ -64,6 +67,10 @@ def lib() -> ctypes.CDLL:
         for name in ("w4a16_linear", "w4a16_gemv", "w4a16_gemm"):
             fn = getattr(L, name)
             fn.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P, ctypes.c_size_t, P]
+        L.w4a16_gemv_ex.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P, ctypes.c_size_t,
+                                    ctypes.c_int, P]
+        PI = ctypes.POINTER(ctypes.c_int)
+        L.w4a16_gemv_plan.argtypes = [I64, I64, I64, ctypes.c_int, PI, PI, PI]
         L.w4a16_workspace_bytes.argtypes = [I64, I64, I64]
         L.w4a16_workspace_bytes.restype = ctypes.c_size_t
         L.w4a16_check_device_status.argtypes = [P]
@@ -78,7 +85,8 @@ def lib() -> ctypes.CDLL:
         L.w4a16_status_string.argtypes = [ctypes.c_int]
         L.w4a16_status_string.restype = ctypes.c_char_p
         L.w4a16_version.argtypes = []
-        for name in ("awq_quantize_g128", "w4a16_linear", "w4a16_gemv", "w4a16_gemm", "w4a16_check_device_status",
+        for name in ("awq_quantize_g128", "w4a16_linear", "w4a16_gemv", "w4a16_gemv_ex", "w4a16_gemv_plan",
+                     "w4a16_gemm", "w4a16_check_device_status",
                      "w4a16_selftest_timeout", "awq_split_outliers", "awq_search_alpha", "awq_fold_activations", "w4a16_version"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -144,7 +152,7 @@ def workspace_bytes(M: int, N: int, K: int) -> int:
     return int(lib().w4a16_workspace_bytes(M, N, K))
 
 
-def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None):
+def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, schedule=None):
     _need(x, torch.bfloat16, 2, "x")
     _need(qweight, torch.int32, 2, "qweight")
     _need(scales, torch.int16, 2, "scales")
@@ -163,9 +171,11 @@ def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None):
     need = workspace_bytes(M, N, K) if name != "w4a16_gemm" else 0
     if ws is None and need > 0:
         ws = workspace(x.device, need)
-    code = getattr(lib(), name)(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros),
-                                ctypes.byref(cs) if cs is not None else None, _ptr(y), M, N, K,
-                                _ptr(ws), ws.numel() if ws is not None else 0, _stream(x.device))
+    args = [_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), ctypes.byref(cs) if cs is not None else None,
+            _ptr(y), M, N, K, _ptr(ws), ws.numel() if ws is not None else 0]
+    if schedule is not None:
+        args.append(int(schedule))
+    code = getattr(lib(), name)(*args, _stream(x.device))
     _check(code, name)
     return y
 
@@ -177,6 +187,18 @@ def w4a16_linear(x, qweight, scales, zeros, csr=None, out=None, workspace=None):
 
 def w4a16_gemv(x, qweight, scales, zeros, csr=None, out=None, workspace=None):
     return _linear("w4a16_gemv", x, qweight, scales, zeros, csr, out, workspace)
+
+
+def w4a16_gemv_ex(x, qweight, scales, zeros, csr=None, out=None, workspace=None, schedule=GEMV_AUTO):
+    return _linear("w4a16_gemv_ex", x, qweight, scales, zeros, csr, out, workspace, schedule)
+
+
+def gemv_plan(M: int, N: int, K: int, schedule: int = GEMV_AUTO):
+    """(schedule, CTAs per cluster or 0, CTAs) that w4a16_gemv_ex would launch on the current device."""
+    r, c, n = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().w4a16_gemv_plan(M, N, K, int(schedule), ctypes.byref(r), ctypes.byref(c), ctypes.byref(n)),
+           "w4a16_gemv_plan")
+    return r.value, c.value, n.value
 
 
 def w4a16_gemm(x, qweight, scales, zeros, csr=None, out=None, workspace=None):

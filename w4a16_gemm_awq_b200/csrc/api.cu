@@ -151,11 +151,18 @@ w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const u
 }
 
 
-w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream) {
+bool valid_schedule(int schedule) {
+    return schedule == W4A16_GEMV_AUTO || schedule == W4A16_GEMV_STREAM_K || schedule == W4A16_GEMV_CLUSTER;
+}
+
+w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W4A16_GEMV_AUTO) {
+    if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
     DeviceInfo* d = nullptr;
     w4a16_status st = device_info(&d);
     if (st != W4A16_OK) return st;
     if (a.K > gemv_max_k() || !gemv_fits((int)a.N, (int)a.K, d->num_sms)) return W4A16_ERR_UNSUPPORTED;
+    const GemvPlan plan = gemv_plan((int)a.M, (int)a.N, (int)a.K, d->num_sms, schedule);
+    if (plan.ctas < 1) return W4A16_ERR_UNSUPPORTED;
     if (a.workspace == nullptr) return W4A16_ERR_NULL;
     if (!aligned(a.workspace, 16)) return W4A16_ERR_ALIGN;
     if (a.workspace_bytes < gemv_workspace_bytes((int)a.N, d->num_sms)) return W4A16_ERR_SHAPE;
@@ -173,7 +180,7 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream) {
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4A16_ERR_CUDA;
     }
-    return from_cuda(launch_gemv(maps, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
+    return from_cuda(launch_gemv(maps, plan, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
                                  a.workspace, (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status, stream));
 }
 
@@ -282,6 +289,36 @@ w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
     return run_gemv(a, static_cast<cudaStream_t>(stream));
+}
+
+w4a16_status w4a16_gemv_ex(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                           const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N,
+                           int64_t K, void* workspace, size_t workspace_bytes, int schedule, void* stream) {
+    LinearArgs a;
+    w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
+    if (st != W4A16_OK) return st;
+    if (M > 16) return W4A16_ERR_SHAPE;
+    if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);
+}
+
+w4a16_status w4a16_gemv_plan(int64_t M, int64_t N, int64_t K, int schedule, int* resolved, int* cluster_size,
+                             int* ctas) {
+    if (M < 1 || M > 16 || N < 128 || N % 128 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK)
+        return W4A16_ERR_SHAPE;
+    if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    if (K > gemv_max_k() || !gemv_fits((int)N, (int)K, d->num_sms)) return W4A16_ERR_UNSUPPORTED;
+    const GemvPlan plan = gemv_plan((int)M, (int)N, (int)K, d->num_sms, schedule);
+    if (plan.ctas < 1) return W4A16_ERR_UNSUPPORTED;
+    if (resolved) *resolved = plan.schedule;
+    if (cluster_size) *cluster_size = plan.cluster;
+    if (ctas) *ctas = plan.ctas;
+    return W4A16_OK;
 }
 
 w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,

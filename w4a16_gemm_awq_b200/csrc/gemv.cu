@@ -44,12 +44,24 @@
 //     k = 32t + 8w + 2p + {0,1}.  The B fragment of thread (token g, t) is then the 16 bytes
 //     x[g][32t + 8w .. +8], whose four 32-bit parts are the same pairs.
 //   - At the end of a row-block segment the consumers drop their accumulators into a
-//     shared-memory partial tile (one half per group pair) and go on streaming; the
-//     epilogue warp adds the halves and does the workspace exchange, the CSR term and the
+//     shared-memory partial tile (warps 0-3 write it, warps 4-7 add theirs) and go on
+//     streaming; the epilogue warp does the exchange between CTAs, the CSR term and the
 //     stores of y.
+//   - Two schedules share everything above and differ in how units map to CTAs:
+//       * stream-K (above): completes split row blocks through the workspace.  A CTA's
+//         last row block is usually shared with the next CTA, which took it first; its
+//         partial tile is then fetched while this CTA still computes, and the row block is
+//         completed without a counter increment.
+//       * cluster split-K: for shapes with few row blocks, thread-block clusters of 2..8
+//         CTAs take whole row blocks, each CTA an equal share of its 512-k units; the
+//         cluster sums its tiles through distributed shared memory, with no workspace
+//         traffic and no CTA waiting on a global counter.
 //   - Programmatic dependent launch.  The weights may be fetched before the previous kernel
 //     on the stream has finished.  The helpers wait for it before they load x; the
 //     epilogue and the completion phase wait before they touch the workspace or y.
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -77,11 +89,13 @@ struct GemvArgs {
     const uint16_t* vals;
     long long nnz;
     uint16_t* y;
-    float* partials;     // workspace: [2P][128][16] fp32
-    unsigned* counters;  // workspace: [N/128], zero between calls
+    float* partials;     // workspace: [2P][128][16] fp32 (stream-K)
+    unsigned* counters;  // workspace: [N/128], zero between calls (stream-K)
     int M, N, K;
     uint32_t T;          // work units = (N/128) * (K/512); T * P < 2^32 (checked by the caller)
     int P;               // CTAs
+    int cl;              // 0: stream-K; else the cluster size of the cluster split-K (2..8, <= K/512)
+    int ncl;             // cluster split-K: clusters (<= N/128); cluster j takes row blocks j, j + ncl, ...
     unsigned* err;
 };
 
@@ -94,9 +108,10 @@ struct GemvSmem {
     static constexpr int kXOff = kGemvStages * kGemvWBytes;
     static constexpr int kParOff = kXOff + kGemvStages * kXBytes;
     static constexpr int kSumOff = kParOff + kGemvStages * kParBytes;
-    static constexpr int kPartOff = kSumOff + kGemvStages * kSumBytes;      // [2 halves][128 rows][kCols]
-    static constexpr int kBarOff = kPartOff + 2 * kGemvRows * kCols * 4;
-    static constexpr int kListOff = kBarOff + (4 * kGemvStages + 2) * 8;    // row blocks this CTA completes
+    static constexpr int kPartOff = kSumOff + kGemvStages * kSumBytes;      // [128 rows][kCols]
+    static constexpr int kRecvOff = kPartOff + kGemvRows * kCols * 4;       // cluster split-K: rows received
+    static constexpr int kBarOff = kRecvOff + kGemvRows * kCols * 4;
+    static constexpr int kListOff = kBarOff + (4 * kGemvStages + 5) * 8;    // row blocks this CTA completes
     static constexpr int kBytes = kListOff + 16 * 4;
     static_assert(kBytes <= 227 * 1024, "shared memory of one CTA");
 };
@@ -111,6 +126,15 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t out[4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(out[i]) : "r"(w >> (4 * i)), "r"(0x000F000Fu), "r"(0x43004300u));
+}
+
+// Next unit of a CTA's walk: gb runs over [kb, ke) within a row block, then the walk moves
+// `step` row blocks on.
+__device__ __forceinline__ void walk_next(int& rb, int& gb, int kb, int ke, int step) {
+    if (++gb == ke) {
+        gb = kb;
+        rb += step;
+    }
 }
 
 // Stream-K index arithmetic in 32 bits (T * P < 2^32), which is far cheaper than 64-bit
@@ -145,6 +169,43 @@ __device__ __forceinline__ void write_row(const GemvArgs& p, int n, float v[16])
         if (m < p.M) p.y[(size_t)m * p.N + n] = float_to_bf16_bits(v[m]);
 }
 
+// Row block rb split between exactly two CTAs: when the other one has published its partial
+// tile (the counter, read with acquire semantics, is 1), loads that tile's rows lane + 32 i
+// into t[i] and returns true.  The calling CTA is then the row block's last contributor and
+// completes it itself.  It adds (0 + own) + other; the completion phase adds the two tiles
+// the same way in contributor order, and since fp32 addition is commutative the two give
+// the same bits, so y does not depend on which CTA finishes last.
+// Returns false otherwise (t undefined).  All lanes of the warp take part.
+template <int C>
+__device__ __forceinline__ bool gather_other(const GemvArgs& p, int rb, int GB, int lane, float t[4][C]) {
+    const uint32_t rb0 = (uint32_t)rb * GB;
+    const int pf = cta_of_unit(rb0, p.T, (uint32_t)p.P);
+    const int pl = cta_of_unit(rb0 + GB - 1, p.T, (uint32_t)p.P);
+    if (pl - pf != 1) return false;
+    if (!__all_sync(0xffffffffu, ld_acquire_gpu(p.counters + rb) == 1u)) return false;
+    const int q = pf == (int)blockIdx.x ? pl : pf;
+    // the second contributor starts inside the row block, so the row block is its first
+    // segment; the first one may have started before it
+    const bool first_starts_here = unit_begin((uint32_t)pf, p.T, (uint32_t)p.P) == rb0;
+    const int slot = 2 * q + (q == pf && !first_starts_here ? 1 : 0);
+    const float4* sp = reinterpret_cast<const float4*>(p.partials + (size_t)slot * kGemvSlotFloats);
+    float4 a[4][C / 4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < C / 4; ++c) a[i][c] = __ldcg(sp + (lane + 32 * i) * (C / 4) + c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < C / 4; ++c) {
+            t[i][4 * c] = a[i][c].x;
+            t[i][4 * c + 1] = a[i][c].y;
+            t[i][4 * c + 2] = a[i][c].z;
+            t[i][4 * c + 3] = a[i][c].w;
+        }
+    return true;
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kGemvThreads, 1)
 gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
@@ -164,38 +225,68 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
     uint64_t* xempty = xfull + S;   // the consumers are done with them
     uint64_t* pfull = xempty + S;   // the partial tile holds a finished segment
     uint64_t* pempty = pfull + 1;   // the epilogue is done with it
+    uint64_t* cready = pempty + 1;  // cluster split-K: the rows the other CTAs send have landed
+    uint64_t* cdone = cready + 1;   // cluster split-K: the other CTAs have summed what this one sent
+    uint64_t* phalf = cdone + 1;    // consumer warps 0-3 have written their part of the tile
     float* part = reinterpret_cast<float*>(smem + L::kPartOff);
     int* reduce_list = reinterpret_cast<int*>(smem + L::kListOff);  // [0] = count, then row blocks
 
+    // The CTA's work: n units, walked row block by row block.  Within a row block the unit
+    // index gb runs over [kb, ke); then the walk moves `step` row blocks on.
     const int GB = p.K >> 9;  // units per row block
-    const uint32_t u0 = unit_begin(blockIdx.x, p.T, (uint32_t)p.P);
-    const int n = (int)(unit_begin(blockIdx.x + 1, p.T, (uint32_t)p.P) - u0);
+    uint32_t u0 = 0;          // stream-K: first unit
+    int n, rb_first, gb_first, kb, ke, step;
+    uint32_t crank = 0;       // cluster split-K: rank in the cluster
+    if (p.cl == 0) {
+        u0 = unit_begin(blockIdx.x, p.T, (uint32_t)p.P);
+        n = (int)(unit_begin(blockIdx.x + 1, p.T, (uint32_t)p.P) - u0);
+        rb_first = (int)(u0 / (uint32_t)GB);
+        gb_first = (int)(u0 - (uint32_t)rb_first * GB);
+        kb = 0;
+        ke = GB;
+        step = 1;
+    } else {
+        // rank r of cluster j takes units [r GB / cl, (r+1) GB / cl) of row blocks j, j + ncl, ...
+        crank = cluster_ctarank();
+        const int j = (int)cluster_id_x();
+        kb = (int)crank * GB / p.cl;
+        ke = ((int)crank + 1) * GB / p.cl;
+        rb_first = j;
+        gb_first = kb;
+        step = p.ncl;
+        n = ((p.N / kGemvRows - 1 - j) / p.ncl + 1) * (ke - kb);
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // one barrier per thread, so that the prologue is short
-    if (threadIdx.x < 4 * S + 2) {
+    if (threadIdx.x < 4 * S + 5) {
         const int i = threadIdx.x;
+        const uint32_t peers = p.cl > 1 ? 32u * (uint32_t)(p.cl - 1) : 1u;  // every epilogue lane of every other CTA
         const uint32_t count = i < S ? 1u : i < 2 * S ? (uint32_t)kGemvConsumers : i < 3 * S ? (uint32_t)kGemvHelpers
-                             : i < 4 * S ? (uint32_t)kGemvConsumers : i == 4 * S ? (uint32_t)kGemvConsumers : 1u;
-        mbar_init(&wfull[i], count);  // wfull, wempty, xfull, xempty, pfull, pempty are contiguous
+                             : i < 4 * S ? (uint32_t)kGemvConsumers : i == 4 * S ? (uint32_t)kGemvConsumers
+                             : i == 4 * S + 3 ? peers : i == 4 * S + 4 ? (uint32_t)(kGemvConsumers / 2) : 1u;
+        mbar_init(&wfull[i], count);  // the ring, pfull, pempty, cready, cdone and phalf are contiguous
         if (i == 0) reduce_list[0] = 0;
         fence_mbarrier_init();
     }
     __syncthreads();
+    // The other CTAs of the cluster arrive on cready and cdone, so those must be initialised
+    // first: every thread arrives on the cluster barrier here, and the epilogue warp waits on
+    // it before its first remote arrival.  The other roles start at once.
+    if (p.cl != 0) cluster_arrive_release();
 
     if (warp == kGemvProducer) {
         // ------------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tensormap(&map_w);
             int issued = 0;
-            for (int s = 0; s < n; ++s) {
+            int rb = rb_first, gb = gb_first;
+            for (int s = 0; s < n; ++s, walk_next(rb, gb, kb, ke, step)) {
                 const int slot = s % S;
                 if (s >= S && !mbar_wait_bounded(&wempty[slot], ((s / S) - 1) & 1)) {
                     record_error(p.err, kErrTimeout);
                     break;
                 }
-                const uint32_t u = u0 + (uint32_t)s;
-                const int rb = (int)(u / (uint32_t)GB), gb = (int)(u - (uint32_t)rb * GB);
                 mbar_arrive_expect_tx(&wfull[slot], (uint32_t)kGemvWBytes);
                 tma_load_3d(smem + slot * kGemvWBytes, &map_w, &wfull[slot], 0, rb * kGemvRows, gb * kGemvUnitGroups);
                 ++issued;
@@ -212,10 +303,9 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
         const int h = warp - kGemvHelper0;
         const int gq = lane >> 2, t = lane & 3;
         const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};  // bf16 1.0 pairs
-        for (int s = 0; s < n; ++s) {
+        int rb = rb_first, gb = gb_first;
+        for (int s = 0; s < n; ++s, walk_next(rb, gb, kb, ke, step)) {
             const int slot = s % S;
-            const uint32_t u = u0 + (uint32_t)s;
-            const int rb = (int)(u / (uint32_t)GB), gb = (int)(u - (uint32_t)rb * GB);
             // global loads first: they do not touch the ring and overlap the wait below.  The
             // scales and zero points do not depend on the previous kernel, so the first unit's
             // are in flight while the helper waits for it; x is loaded after the wait.
@@ -310,8 +400,8 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0f;
 
-        int rb = (int)(u0 / (uint32_t)GB), gb = (int)(u0 - (uint32_t)rb * GB);  // coordinates of unit u0 + s
-        for (int s = 0; s < n; ++s, (gb + 1 == GB ? (gb = 0, ++rb) : ++gb)) {
+        int rb = rb_first, gb = gb_first;
+        for (int s = 0; s < n; ++s, walk_next(rb, gb, kb, ke, step)) {
             const int slot = s % S;
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(&wfull[slot], (s / S) & 1))) {
                 if (lane == 0) record_error(p.err, kErrTimeout);
@@ -400,41 +490,160 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&xempty[slot]);
 
-            if (gb == GB - 1 || s == n - 1) {
+            if (gb == ke - 1 || s == n - 1) {
                 // ---------------------------------------------------------- segment end
                 if (seg > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(pempty, (seg - 1) & 1))) {
                     if (lane == 0) record_error(p.err, kErrTimeout);
                     break;
                 }
-                float* pt = part + half * (kGemvRows * C);
+                // Warps 0-3 (groups 0, 1 of every unit) write the tile; warps 4-7 (groups 2, 3)
+                // then add theirs to the same rows and tokens.
+                if (half == 1 && !__all_sync(0xffffffffu, mbar_wait_bounded(phalf, seg & 1))) {
+                    if (lane == 0) record_error(p.err, kErrTimeout);
+                    break;
+                }
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const int c0 = rbase + 16 * i, c1 = c0 + 8;
 #pragma unroll
                     for (int j = 0; j < NT; ++j) {
                         const int tk = 8 * j + 2 * t;
-                        *reinterpret_cast<float2*>(&pt[c0 * C + tk]) = make_float2(acc[i][j][0], acc[i][j][1]);
-                        *reinterpret_cast<float2*>(&pt[c1 * C + tk]) = make_float2(acc[i][j][2], acc[i][j][3]);
+                        float2* q0 = reinterpret_cast<float2*>(&part[c0 * C + tk]);
+                        float2* q1 = reinterpret_cast<float2*>(&part[c1 * C + tk]);
+                        if (half == 0) {
+                            *q0 = make_float2(acc[i][j][0], acc[i][j][1]);
+                            *q1 = make_float2(acc[i][j][2], acc[i][j][3]);
+                        } else {
+                            const float2 a = *q0, b = *q1;
+                            *q0 = make_float2(a.x + acc[i][j][0], a.y + acc[i][j][1]);
+                            *q1 = make_float2(b.x + acc[i][j][2], b.y + acc[i][j][3]);
+                        }
                         acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.0f;
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(pfull);
+                if (lane == 0) {
+                    if (half == 0) mbar_arrive(phalf);
+                    mbar_arrive(pfull);
+                }
                 ++seg;
             }
         }
+    } else if (p.cl != 0) {
+        // ------------------------------------------------------------------ epilogue warp,
+        // cluster split-K.  Every CTA of the cluster holds a partial tile of the same row
+        // block.  Rank r owns rows [128 r / cl, 128 (r+1) / cl): each other CTA sends it
+        // those rows of its tile with asynchronous stores into r's shared memory, whose bytes
+        // complete r's cready barrier; r then sums the cluster's tiles for its rows in rank
+        // order and writes them.  With several row blocks per cluster, a CTA sends the next
+        // row block's rows only once every receiver has summed the previous ones (cdone).  A
+        // failed wait is recorded and the exchange goes on, so that no CTA leaves while data
+        // may still arrive for it.
+        const int cl = p.cl;
+        const int row0 = (int)crank * kGemvRows / cl, row1 = ((int)crank + 1) * kGemvRows / cl;
+        const int nrow = row1 - row0;  // at most 64
+        const int nseg = n / (ke - kb);
+        const float* recv = reinterpret_cast<const float*>(smem + L::kRecvOff);  // [cl - 1][nrow][C]
+        float* recv_w = reinterpret_cast<float*>(smem + L::kRecvOff);
+        const uint32_t recv_bytes = (uint32_t)((cl - 1) * nrow * C * 4);
+        if (lane == 0) mbar_arrive_expect_tx(cready, recv_bytes);
+        cluster_wait_acquire();  // every CTA of the cluster has initialised its barriers
+        griddep_wait();          // y belongs to the stream order
+        int rb = rb_first;
+        for (int seg = 0; seg < nseg; ++seg, rb += step) {
+            bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(pfull, seg & 1));
+            if (seg > 0) ok = __all_sync(0xffffffffu, mbar_wait_cluster_bounded(cdone, (seg - 1) & 1)) && ok;
+            for (int r = 0; r < cl; ++r) {
+                if (r == (int)crank) continue;
+                const int r0 = r * kGemvRows / cl, nr = (r + 1) * kGemvRows / cl - r0;
+                const int slot = (int)crank < r ? (int)crank : (int)crank - 1;  // this CTA's slot at rank r
+                const uint32_t dst = cluster_map(recv_w + slot * nr * C, (uint32_t)r);
+                const uint32_t bar = cluster_map(cready, (uint32_t)r);
+                const float4* src = reinterpret_cast<const float4*>(part + r0 * C);
+                for (int e = lane; e < nr * C / 4; e += 32) st_async_f4(dst + 16u * (uint32_t)e, src[e], bar);
+            }
+            float own[2][C];  // rows row0 + lane + 32 i of this CTA's tile
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int r = row0 + lane + 32 * i;
+#pragma unroll
+                for (int c = 0; c < C; ++c) own[i][c] = r < row1 ? part[r * C + c] : 0.0f;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pempty);  // the consumers may overwrite the tile
+            ok = __all_sync(0xffffffffu, mbar_wait_cluster_bounded(cready, seg & 1)) && ok;
+            float v[2][16];
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int c = 0; c < 16; ++c) v[i][c] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int r = row0 + lane + 32 * i;
+                if (r < row1) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (q >= cl) continue;
+                        if (q == (int)crank) {
+#pragma unroll
+                            for (int c = 0; c < C; ++c) v[i][c] += own[i][c];
+                        } else {
+                            const float4* t = reinterpret_cast<const float4*>(
+                                recv + ((q < (int)crank ? q : q - 1) * nrow + (r - row0)) * C);
+#pragma unroll
+                            for (int c = 0; c < C / 4; ++c) {
+                                const float4 a = t[c];
+                                v[i][4 * c] += a.x;
+                                v[i][4 * c + 1] += a.y;
+                                v[i][4 * c + 2] += a.z;
+                                v[i][4 * c + 3] += a.w;
+                            }
+                        }
+                    }
+                }
+            }
+            if (seg + 1 < nseg) {
+                // ready for the next row block's rows; tell every sender its rows were summed
+                if (lane == 0) mbar_arrive_expect_tx(cready, recv_bytes);
+                for (int q = 0; q < cl; ++q)
+                    if (q != (int)crank) mbar_arrive_cluster(cluster_map(cdone, (uint32_t)q));
+            }
+            if (ok) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int r = row0 + lane + 32 * i;
+                    if (r < row1) write_row(p, rb * kGemvRows + r, v[i]);
+                }
+            } else if (lane == 0) {
+                record_error(p.err, kErrTimeout);
+            }
+        }
     } else {
-        // ------------------------------------------------------------------ epilogue warp
-        // Walks the same segments as the consumers.  Lane l owns rows l, l+32, l+64, l+96.
+        // ------------------------------------------------------------------ epilogue warp,
+        // stream-K.  Walks the same segments as the consumers.  Lane l owns rows l, l+32,
+        // l+64, l+96.
         bool waited = false;
         int seg = 0;
-        uint32_t seg_first = u0;  // first unit of the current segment
-        for (int s = 0; s < n; ++s) {
-            const uint32_t u = u0 + (uint32_t)s;
-            const int rb = (int)(u / (uint32_t)GB), gb = (int)(u - (uint32_t)rb * GB);
-            if (!(gb == GB - 1 || s == n - 1)) continue;
-            const bool whole = seg_first == (uint32_t)rb * GB && gb == GB - 1;
-            seg_first = u + 1;
+        const uint32_t u_end = u0 + (uint32_t)n;
+        for (uint32_t first = u0; first < u_end; ++seg) {
+            const int rb = (int)(first / (uint32_t)GB);
+            const uint32_t rb0 = (uint32_t)rb * GB;
+            const uint32_t end = rb0 + GB < u_end ? rb0 + GB : u_end;
+            const bool whole = first == rb0 && end == rb0 + GB;
+            const bool last = end == u_end;
+            first = end;
+            // The other contributor of the stream's last row block takes it at the start of
+            // its own stream, so it has usually published its partial by the time this CTA
+            // begins the row block: fetch it now, while the consumers are still computing.
+            float other[4][C];
+            bool gathered = false;
+            if (!whole && last) {
+                if (!waited) {
+                    griddep_wait();  // the workspace belongs to the stream order
+                    waited = true;
+                }
+                gathered = gather_other<C>(p, rb, GB, lane, other);
+            }
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(pfull, seg & 1))) {
                 if (lane == 0) record_error(p.err, kErrTimeout);
                 break;
@@ -444,52 +653,61 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                 waited = true;
             }
             const float* p0 = part;
-            const float* p1 = part + kGemvRows * C;
-            if (whole) {
-                for (int r = lane; r < kGemvRows; r += 32) {
+            if (!whole && !gathered) {
+                // publish this CTA's partial tile
+                const int pf = cta_of_unit(rb0, p.T, (uint32_t)p.P);
+                const int pl = cta_of_unit(rb0 + GB - 1, p.T, (uint32_t)p.P);
+                const int mine = 2 * (int)blockIdx.x + (u0 >= rb0 ? 0 : 1);
+                float4* dst = reinterpret_cast<float4*>(p.partials + (size_t)mine * kGemvSlotFloats);
+                const float4* a4 = reinterpret_cast<const float4*>(p0);
+                for (int q = lane; q < kGemvRows * C / 4; q += 32) __stcg(dst + q, a4[q]);
+                {
+                    // release the partial tile to the completing CTA: the warp's stores, then
+                    // the counter increment by lane 0 with acquire-release semantics at GPU
+                    // scope.  It orders the warp's stores (which __syncwarp orders before it)
+                    // ahead of the increment, and in the CTA that completes the count it
+                    // acquires every earlier contributor's partial; the barrier of the
+                    // completion phase passes that on.
+                    __syncwarp();
+                    unsigned old = 0;
+                    if (lane == 0) old = atomic_add_acq_rel_gpu(p.counters + rb, 1u);
+                    old = __shfl_sync(0xffffffffu, old, 0);
+                    // the CTA that completes the row block sums its partials after the stream ends
+                    if (lane == 0 && old == (unsigned)(pl - pf) && reduce_list[0] < 15)
+                        reduce_list[1 + reduce_list[0]++] = rb;
+                }
+            }
+            if (whole || gathered) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = lane + 32 * i;
                     float v[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) v[c] = 0.0f;
 #pragma unroll
                     for (int c = 0; c < C; c += 4) {
                         const float4 a = *reinterpret_cast<const float4*>(&p0[r * C + c]);
-                        const float4 b = *reinterpret_cast<const float4*>(&p1[r * C + c]);
-                        v[c] = a.x + b.x;
-                        v[c + 1] = a.y + b.y;
-                        v[c + 2] = a.z + b.z;
-                        v[c + 3] = a.w + b.w;
+                        v[c] = a.x;
+                        v[c + 1] = a.y;
+                        v[c + 2] = a.z;
+                        v[c + 3] = a.w;
+                        if (gathered) {  // (0 + own) + other, as the completion phase adds
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) v[c + e] = (0.0f + v[c + e]) + other[i][c + e];
+                        }
                     }
                     write_row(p, rb * kGemvRows + r, v);
                 }
-            } else {
-                const int pf = cta_of_unit((uint32_t)rb * GB, p.T, (uint32_t)p.P);
-                const int pl = cta_of_unit((uint32_t)rb * GB + GB - 1, p.T, (uint32_t)p.P);
-                const int mine = 2 * (int)blockIdx.x + (u0 >= (uint32_t)rb * GB ? 0 : 1);
-                float4* dst = reinterpret_cast<float4*>(p.partials + (size_t)mine * kGemvSlotFloats);
-                const float4* a4 = reinterpret_cast<const float4*>(p0);
-                const float4* b4 = reinterpret_cast<const float4*>(p1);
-                for (int q = lane; q < kGemvRows * C / 4; q += 32) {
-                    const float4 a = a4[q], b = b4[q];
-                    __stcg(dst + q, make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w));
-                }
-                // release the partial tile to the completing CTA: the warp's stores, then the
-                // counter increment by lane 0 with acquire-release semantics at GPU scope.  It
-                // orders the warp's stores (which __syncwarp orders before it) ahead of the
-                // increment, and in the CTA that completes the count it acquires every earlier
-                // contributor's partial; the barrier of the completion phase passes that on.
-                __syncwarp();
-                unsigned old = 0;
-                if (lane == 0) old = atomic_add_acq_rel_gpu(p.counters + rb, 1u);
-                old = __shfl_sync(0xffffffffu, old, 0);
-                // the CTA that completes the row block sums its partials after the stream ends
-                if (lane == 0 && old == (unsigned)(pl - pf) && reduce_list[0] < 15)
-                    reduce_list[1 + reduce_list[0]++] = rb;
+                // the other contributor has arrived, so nothing else touches the counter
+                if (gathered && lane == 0) atomicExch(p.counters + rb, 0u);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(pempty);
-            ++seg;
         }
     }
+    // every thread that arrived on the cluster barrier also waits on it (the epilogue warp
+    // did so before its exchange)
+    if (p.cl != 0 && warp != kGemvEpilogue) cluster_wait_acquire();
     griddep_launch_dependents();
 
     // ---------------------------------------------------------------------- completions
@@ -566,7 +784,93 @@ size_t gemv_workspace_bytes(int N, int num_sms) {
     return partials + ((counters + 255) / 256) * 256;
 }
 
-cudaError_t launch_gemv(const GemvMaps& maps, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
+namespace {
+
+// Cost of a schedule, in work units of the slowest CTA, plus an estimate of the end of the
+// call: stream-K completes split row blocks through the workspace (a release, an acquire and
+// loads of the other partials from L2, about two units' time), the cluster split-K through
+// distributed shared memory (about half a unit).
+constexpr double kStreamKExchange = 2.0;
+constexpr double kClusterExchange = 0.5;
+
+// Most clusters of `cl` CTAs of the kernel instance that can be resident at once (0 when
+// none), per device; asked once and kept.
+int max_active_clusters(bool two, int cl) {
+    constexpr int kDevices = 64;
+    static std::atomic<int> cache[kDevices][2][9];
+    static std::atomic<bool> init{false};
+    static std::mutex mu;
+    if (!init.load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> g(mu);
+        if (!init.load(std::memory_order_relaxed)) {
+            for (auto& d : cache)
+                for (auto& t : d)
+                    for (auto& c : t) c.store(-1, std::memory_order_relaxed);
+            init.store(true, std::memory_order_release);
+        }
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices || cl < 2 || cl > 8) return 0;
+    std::atomic<int>& slot = cache[dev][two ? 1 : 0][cl];
+    int v = slot.load(std::memory_order_relaxed);
+    if (v >= 0) return v;
+    const int smem = two ? GemvSmem<2>::kBytes : GemvSmem<1>::kBytes;
+    const void* fn = two ? (const void*)gemv_w4a16_kernel<2> : (const void*)gemv_w4a16_kernel<1>;
+    v = 0;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(cl, 1, 1);
+        cfg.blockDim = dim3(kGemvThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cl;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) == cudaSuccess && n > 0) v = n;
+    }
+    (void)cudaGetLastError();  // a refused query only rules the cluster schedule out
+    slot.store(v, std::memory_order_relaxed);
+    return v;
+}
+
+}  // namespace
+
+GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule) {
+    const bool two = M > 8;
+    const int NRB = N / kGemvRows, GB = K / (128 * kGemvUnitGroups);
+    const long long T = (long long)NRB * GB;
+    GemvPlan sk{W4A16_GEMV_STREAM_K, 0, 0, gemv_ctas(N, K, num_sms)};
+    const long long per = (T + sk.ctas - 1) / sk.ctas;
+    const bool split = T % sk.ctas != 0 || (T / sk.ctas) % GB != 0;
+    const double cost_sk = (double)per + (split ? kStreamKExchange : 0.0);
+    GemvPlan best{W4A16_GEMV_CLUSTER, 0, 0, 0};
+    double cost_best = 0.0;
+    if (schedule != W4A16_GEMV_STREAM_K) {
+        for (int cl = 2; cl <= 8 && cl <= GB; ++cl) {
+            const int mac = max_active_clusters(two, cl);
+            if (mac < 1) continue;
+            const int ncl = NRB < mac ? NRB : mac;
+            // The automatic choice keeps to one row block per cluster: with several, each
+            // exchange must hide behind the next row block's units, which few CTAs per
+            // cluster can only do for long row blocks.
+            if (schedule == W4A16_GEMV_AUTO && ncl < NRB) continue;
+            const double cost = (double)((NRB + ncl - 1) / ncl) * ((GB + cl - 1) / cl) + kClusterExchange;
+            if (best.cluster == 0 || cost < cost_best) {
+                best = GemvPlan{W4A16_GEMV_CLUSTER, cl, ncl, ncl * cl};
+                cost_best = cost;
+            }
+        }
+    }
+    if (schedule == W4A16_GEMV_CLUSTER) return best;  // cluster == 0: not possible here
+    if (schedule == W4A16_GEMV_STREAM_K || best.cluster == 0 || cost_best >= cost_sk) return sk;
+    return best;
+}
+
+cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
                         const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
                         uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
                         cudaStream_t stream) {
@@ -583,8 +887,11 @@ cudaError_t launch_gemv(const GemvMaps& maps, const uint16_t* x, const uint16_t*
     a.N = N;
     a.K = K;
     a.T = (uint32_t)((N / kGemvRows) * (K / (128 * kGemvUnitGroups)));
-    a.P = gemv_ctas(N, K, num_sms);
+    a.P = plan.ctas;
+    a.cl = plan.cluster;
+    a.ncl = plan.clusters;
     a.err = err;
+    if (plan.ctas < 1 || (plan.cluster != 0 && plan.ctas != plan.cluster * plan.clusters)) return cudaErrorInvalidValue;
     const size_t partial_bytes = (size_t)2 * num_sms * kGemvSlotFloats * sizeof(float);
     a.partials = static_cast<float*>(workspace);
     a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + partial_bytes);
@@ -599,11 +906,15 @@ cudaError_t launch_gemv(const GemvMaps& maps, const uint16_t* x, const uint16_t*
     cfg.blockDim = dim3(kGemvThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = plan.cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = plan.cluster != 0 ? 2 : 1;
     if (two) return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<2>, maps.w, a);
     return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<1>, maps.w, a);
 }

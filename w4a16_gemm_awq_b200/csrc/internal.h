@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "w4a16.h"
+
 namespace w4a16 {
 
 // Bits of the per-device status word that kernels set when they find a problem.
@@ -30,7 +32,19 @@ bool gemv_fits(int N, int K, int num_sms);
 // Bytes of zero-initialised device workspace the GEMV needs for N output channels.
 size_t gemv_workspace_bytes(int N, int num_sms);
 
-cudaError_t launch_gemv(const GemvMaps& maps, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
+// A GEMV launch: schedule (W4A16_GEMV_STREAM_K or _CLUSTER), CTAs per cluster (0 for
+// stream-K), clusters and CTAs of the grid.  ctas == 0: the requested schedule cannot run.
+struct GemvPlan {
+    int schedule;
+    int cluster;
+    int clusters;
+    int ctas;
+};
+
+// The launch for a schedule (W4A16_GEMV_AUTO, _STREAM_K or _CLUSTER) on the current device.
+GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule);
+
+cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
                         const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
                         uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
                         cudaStream_t stream);
