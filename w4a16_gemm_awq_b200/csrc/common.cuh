@@ -143,9 +143,11 @@ __device__ __forceinline__ void mma_16816_bf16_zero_nv(float d[4], const uint32_
 // ------------------------------------------------------------------ cluster / DSMEM --
 
 // Split cluster barrier: every thread of the cluster arrives (without blocking); a thread
-// that needs the others' earlier writes then waits.
-__device__ __forceinline__ void cluster_arrive_release() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+// that needs the others to have got past their arrival then waits.  The relaxed arrival
+// publishes nothing by itself: mbarrier initialisations are published to the cluster by
+// fence_mbarrier_init before it.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void cluster_wait_acquire() {
@@ -244,15 +246,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
-// Asynchronous 16-byte store into the shared memory of a CTA of this cluster; its bytes count
-// as completed transactions on that CTA's mbarrier `remote_bar` (both addresses from
-// cluster_map).  A thread that sees the barrier's phase complete (acquire at cluster scope)
-// sees the data.
-__device__ __forceinline__ void st_async_f4(uint32_t remote, float4 v, uint32_t remote_bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
-                 ::"r"(remote), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(remote_bar)
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this CTA's
+// shared memory into the shared memory of a CTA of this cluster; the bytes count as completed
+// transactions on that CTA's mbarrier (destination and barrier addresses from cluster_map).
+// The source must have been written before a fence_proxy_async_smem by its writers.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "r"(smem_u32(src)), "r"(bytes), "r"(bar)
                  : "memory");
 }
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Returns once every bulk copy this thread committed has finished reading its source.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // Arrive on an mbarrier of a CTA of this cluster (address from cluster_map), releasing this
 // thread's earlier writes at cluster scope.

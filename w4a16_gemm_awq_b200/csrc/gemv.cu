@@ -273,7 +273,7 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
     // The other CTAs of the cluster arrive on cready and cdone, so those must be initialised
     // first: every thread arrives on the cluster barrier here, and the epilogue warp waits on
     // it before its first remote arrival.  The other roles start at once.
-    if (p.cl != 0) cluster_arrive_release();
+    if (p.cl != 0) cluster_arrive_relaxed();
 
     if (warp == kGemvProducer) {
         // ------------------------------------------------------------------ producer
@@ -521,6 +521,7 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                         acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.0f;
                     }
                 }
+                if (p.cl != 0) fence_proxy_async_smem();  // the tile leaves by bulk copy
                 __syncwarp();
                 if (lane == 0) {
                     if (half == 0) mbar_arrive(phalf);
@@ -533,7 +534,7 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
         // ------------------------------------------------------------------ epilogue warp,
         // cluster split-K.  Every CTA of the cluster holds a partial tile of the same row
         // block.  Rank r owns rows [128 r / cl, 128 (r+1) / cl): each other CTA sends it
-        // those rows of its tile with asynchronous stores into r's shared memory, whose bytes
+        // those rows of its tile with one bulk copy into r's shared memory, whose bytes
         // complete r's cready barrier; r then sums the cluster's tiles for its rows in rank
         // order and writes them.  With several row blocks per cluster, a CTA sends the next
         // row block's rows only once every receiver has summed the previous ones (cdone).  A
@@ -553,14 +554,15 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
         for (int seg = 0; seg < nseg; ++seg, rb += step) {
             bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(pfull, seg & 1));
             if (seg > 0) ok = __all_sync(0xffffffffu, mbar_wait_cluster_bounded(cdone, (seg - 1) & 1)) && ok;
-            for (int r = 0; r < cl; ++r) {
-                if (r == (int)crank) continue;
-                const int r0 = r * kGemvRows / cl, nr = (r + 1) * kGemvRows / cl - r0;
-                const int slot = (int)crank < r ? (int)crank : (int)crank - 1;  // this CTA's slot at rank r
-                const uint32_t dst = cluster_map(recv_w + slot * nr * C, (uint32_t)r);
-                const uint32_t bar = cluster_map(cready, (uint32_t)r);
-                const float4* src = reinterpret_cast<const float4*>(part + r0 * C);
-                for (int e = lane; e < nr * C / 4; e += 32) st_async_f4(dst + 16u * (uint32_t)e, src[e], bar);
+            if (lane == 0) {
+                for (int r = 0; r < cl; ++r) {
+                    if (r == (int)crank) continue;
+                    const int r0 = r * kGemvRows / cl, nr = (r + 1) * kGemvRows / cl - r0;
+                    const int slot = (int)crank < r ? (int)crank : (int)crank - 1;  // this CTA's slot at rank r
+                    bulk_copy_to_cluster(cluster_map(recv_w + slot * nr * C, (uint32_t)r), part + r0 * C,
+                                         (uint32_t)(nr * C * 4), cluster_map(cready, (uint32_t)r));
+                }
+                bulk_commit_group();
             }
             float own[2][C];  // rows row0 + lane + 32 i of this CTA's tile
 #pragma unroll
@@ -569,6 +571,7 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
 #pragma unroll
                 for (int c = 0; c < C; ++c) own[i][c] = r < row1 ? part[r * C + c] : 0.0f;
             }
+            if (lane == 0) bulk_wait_read_all();  // the copies have read the tile
             __syncwarp();
             if (lane == 0) mbar_arrive(pempty);  // the consumers may overwrite the tile
             ok = __all_sync(0xffffffffu, mbar_wait_cluster_bounded(cready, seg & 1)) && ok;
