@@ -509,7 +509,8 @@ def run_case(args):
     packs = [(qw, sc, z)] + [(qw.clone(), sc.clone(), z.clone()) for _ in range(copies - 1)]
     x = torch.from_numpy(workloads.make_activations(99, M, L.mult).view(np.int16)).view(torch.bfloat16).cuda()
     y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-    fn = {"gemv": w4.w4a16_gemv, "gemm": w4.w4a16_gemm}.get(args.case)
+    sched = {"auto": w4.GEMV_AUTO, "stream_k": w4.GEMV_STREAM_K, "cluster": w4.GEMV_CLUSTER}[args.schedule]
+    fn = {"gemv": lambda *a, **k: w4.w4a16_gemv_ex(*a, **k, schedule=sched), "gemm": w4.w4a16_gemm}.get(args.case)
     ws = torch.zeros(max(256, w4.workspace_bytes(min(M, 16), N, K)), dtype=torch.uint8, device="cuda")
 
     def once(i):
@@ -536,7 +537,7 @@ def run_case(args):
         print(json.dumps({"case": "quantize", "K": K, "N": N, "ms": ms, "GB/s": b / ms / 1e6}))
     elif args.case == "gemv":
         print(json.dumps({"case": "gemv", "K": K, "N": N, "M": M, "ms": ms, "copies": copies,
-                          "GB/s": gemv_bytes(N, K, M) / ms / 1e6}))
+                          "plan": w4.gemv_plan(M, N, K, sched), "GB/s": gemv_bytes(N, K, M) / ms / 1e6}))
     else:
         print(json.dumps({"case": "gemm", "K": K, "N": N, "M": M, "ms": ms, "TFLOP/s": 2.0 * M * N * K / ms / 1e9}))
 
@@ -559,6 +560,8 @@ def main():
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)
     ap.add_argument("--M", type=int, default=16)
+    ap.add_argument("--schedule", default="auto", choices=["auto", "stream_k", "cluster"],
+                    help="GEMV schedule of --case gemv")
     args = ap.parse_args()
     if args.case:
         run_case(args)

@@ -9,6 +9,8 @@ from parity import Case, check_close, dev_bits, dev_csr, host_bf16_as_f64, xs_ab
 
 pytestmark = pytest.mark.gpu
 
+SCHEDULES = [w4.GEMV_STREAM_K, w4.GEMV_CLUSTER]
+
 
 def gemv(case_dev, fn=None):
     fn = fn or w4.w4a16_gemv
@@ -39,6 +41,34 @@ def test_gemv_odd_shapes(orc, K, N):
     y = host_bf16_as_f64(gemv(c.device()))
     ref, ref_abs = c.reference(orc)
     check_close(y, ref, ref_abs, 0.0, depth(K), f"{K}x{N}", xs_abs(c.x, c.sc))
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES, ids=["stream_k", "cluster"])
+@pytest.mark.parametrize("M", [4, 12])
+def test_gemv_activation_ranges(orc, schedule, M):
+    """Tokens whose magnitudes differ by up to 2^80, groups from 2^-40 to 2^65 (beyond fp16's
+    range), all-zero groups and single huge values: every token keeps its own accuracy."""
+    c = Case(orc, seed=41 + M, K=2048, N=256, M=M, csr=True)
+    rng = np.random.default_rng(M)
+    x = (c.x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    G = c.K // 128
+    for m in range(M):
+        kind = m % 4
+        if kind == 1:
+            x[m] *= 2.0 ** 40
+        elif kind == 2:
+            x[m] *= 2.0 ** -40
+        elif kind == 3:
+            x[m] *= np.repeat(2.0 ** (7.0 * np.arange(G) - 40.0), 128)
+        if m % 3 == 0:
+            x[m, 256:384] = 0.0                      # an all-zero group
+        x[m, rng.integers(0, c.K)] *= 2.0 ** 20      # one value far above the rest of its group
+    c.x = (x.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)  # exact: powers of two
+    d = c.device()
+    y = w4.w4a16_gemv_ex(d["x"], d["qweight"], d["scales"], d["zeros"], csr=d["csr"], schedule=schedule)
+    w4.check_device_status()
+    ref, ref_abs = c.reference(orc)
+    check_close(host_bf16_as_f64(y), ref, ref_abs, 0.0, depth(c.K), f"ranges M={M}", xs_abs(c.x, c.sc))
 
 
 def test_gemv_empty_csr_is_bit_identical(orc):
@@ -101,9 +131,6 @@ def test_gemv_workspace_contract(orc):
     assert int(ws.count_nonzero()) == ws.numel() - int((ws == 0).sum())  # sanity
     counters = ws[need - 256 * ((c.N // 128 * 4 + 255) // 256):]
     assert int(counters.count_nonzero()) == 0
-
-
-SCHEDULES = [w4.GEMV_STREAM_K, w4.GEMV_CLUSTER]
 
 
 @pytest.mark.parametrize("schedule", SCHEDULES, ids=["stream_k", "cluster"])
