@@ -258,15 +258,30 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // one barrier per thread, so that the prologue is short
-    if (threadIdx.x < 4 * S + 5) {
+    // The producer thread initialises the weight ring's full barriers itself and starts its
+    // first copies before the CTA-wide barrier: the first weights are what a call waits for
+    // first.  The copies touch nothing of the previous kernel on the stream.
+    int pre = 0;                       // copies issued here (producer thread only)
+    int prb = rb_first, pgb = gb_first;  // coordinates of the producer's next copy
+    if (threadIdx.x == kGemvProducer * 32) {
+        prefetch_tensormap(&map_w);
+        for (int i = 0; i < S; ++i) mbar_init(&wfull[i], 1u);
+        fence_mbarrier_init();
+        fence_proxy_async_smem();
+        for (; pre < S && pre < n; ++pre, walk_next(prb, pgb, kb, ke, step)) {
+            mbar_arrive_expect_tx(&wfull[pre], (uint32_t)kGemvWBytes);
+            tma_load_3d(smem + pre * kGemvWBytes, &map_w, &wfull[pre], 0, prb * kGemvRows, pgb * kGemvUnitGroups);
+        }
+    }
+    // the other barriers, one per thread, so that the prologue is short
+    if (threadIdx.x >= S && threadIdx.x < 4 * S + 5) {
         const int i = threadIdx.x;
         const uint32_t peers = p.cl > 1 ? 32u * (uint32_t)(p.cl - 1) : 1u;  // every epilogue lane of every other CTA
         const uint32_t count = i < S ? 1u : i < 2 * S ? (uint32_t)kGemvConsumers : i < 3 * S ? (uint32_t)kGemvHelpers
                              : i < 4 * S ? (uint32_t)kGemvConsumers : i == 4 * S ? (uint32_t)kGemvConsumers
                              : i == 4 * S + 3 ? peers : i == 4 * S + 4 ? (uint32_t)(kGemvConsumers / 2) : 1u;
         mbar_init(&wfull[i], count);  // the ring, pfull, pempty, cready, cdone and phalf are contiguous
-        if (i == 0) reduce_list[0] = 0;
+        if (i == S) reduce_list[0] = 0;
         fence_mbarrier_init();
     }
     __syncthreads();
@@ -278,17 +293,15 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
     if (warp == kGemvProducer) {
         // ------------------------------------------------------------------ producer
         if (lane == 0) {
-            prefetch_tensormap(&map_w);
-            int issued = 0;
-            int rb = rb_first, gb = gb_first;
-            for (int s = 0; s < n; ++s, walk_next(rb, gb, kb, ke, step)) {
+            int issued = pre;
+            for (int s = pre; s < n; ++s, walk_next(prb, pgb, kb, ke, step)) {
                 const int slot = s % S;
                 if (s >= S && !mbar_wait_bounded(&wempty[slot], ((s / S) - 1) & 1)) {
                     record_error(p.err, kErrTimeout);
                     break;
                 }
                 mbar_arrive_expect_tx(&wfull[slot], (uint32_t)kGemvWBytes);
-                tma_load_3d(smem + slot * kGemvWBytes, &map_w, &wfull[slot], 0, rb * kGemvRows, gb * kGemvUnitGroups);
+                tma_load_3d(smem + slot * kGemvWBytes, &map_w, &wfull[slot], 0, prb * kGemvRows, pgb * kGemvUnitGroups);
                 ++issued;
             }
             // the copies this CTA started must land before it may exit
