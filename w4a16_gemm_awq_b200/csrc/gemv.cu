@@ -289,6 +289,10 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
     // first: every thread arrives on the cluster barrier here, and the epilogue warp waits on
     // it before its first remote arrival.  The other roles start at once.
     if (p.cl != 0) cluster_arrive_relaxed();
+    // The next kernel on the stream may be scheduled once every CTA of this grid is running:
+    // its CTAs then take SMs as this grid's CTAs leave them and fetch their weights, while
+    // everything it reads or writes of ours waits for this grid to complete.
+    griddep_launch_dependents();
 
     if (warp == kGemvProducer) {
         // ------------------------------------------------------------------ producer
@@ -724,7 +728,6 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
     // every thread that arrived on the cluster barrier also waits on it (the epilogue warp
     // did so before its exchange)
     if (p.cl != 0 && warp != kGemvEpilogue) cluster_wait_acquire();
-    griddep_launch_dependents();
 
     // ---------------------------------------------------------------------- completions
     // The consumer warps and the epilogue warp sum the partial tiles of the row blocks this
