@@ -62,10 +62,16 @@ def _L():
             "oracle_awq_scales": ([P, I64, F, P], ctypes.c_int),
             "oracle_quantize_with_scales": ([P, P, I64, I64, P, P, P], ctypes.c_int),
             "oracle_awq_quantize_g128": ([P, P, F, I64, I64, P, P, P, P], ctypes.c_int),
+            "oracle_awq_quantize_gs": ([P, P, F, I64, I64, I64, P, P, P, P], ctypes.c_int),
+            "oracle_quantize_with_scales_gs": ([P, P, I64, I64, I64, P, P, P], ctypes.c_int),
             "oracle_dequant": ([P, P, P, I64, I64, P], ctypes.c_int),
+            "oracle_dequant_gs": ([P, P, P, I64, I64, I64, P], ctypes.c_int),
             "oracle_linear": ([P, I64, I64, P, P, P, I64, P, P, P, I64, P, P], ctypes.c_int),
+            "oracle_linear_gs": ([P, I64, I64, I64, P, P, P, I64, P, P, P, I64, P, P], ctypes.c_int),
             "oracle_linear_at": ([P, I64, I64, P, P, P, I64, P, P, P, I64, P, P, I64, P, P],
                                  ctypes.c_int),
+            "oracle_linear_at_gs": ([P, I64, I64, I64, P, P, P, I64, P, P, P, I64, P, P, I64, P, P],
+                                    ctypes.c_int),
             "oracle_split_outliers": ([P, P, F, I64, I64, I64, P, P, P, P], ctypes.c_int),
             "oracle_awq_search_alpha": ([P, P, P, I64, I64, I64, P, I64, P], ctypes.c_int),
         }
@@ -129,14 +135,15 @@ def awq_scales(act_absmean, alpha: float) -> np.ndarray:
     return s
 
 
-def quantize_with_scales(W, s):
+def quantize_with_scales(W, s, group_size: int = 128):
     W = _c(W, np.float32)
     s = _c(s, np.float32)
     N, K = W.shape
+    G = max(K // group_size, 1)
     qw = np.zeros((N, K // 8), np.uint32)
-    sc = np.zeros((K // 128, N), np.uint16)
-    z = np.zeros((K // 128, max(N // 8, 1)), np.uint32)
-    _check(_L().oracle_quantize_with_scales(_p(W), _p(s), N, K, _p(qw), _p(sc), _p(z)),
+    sc = np.zeros((G, N), np.uint16)
+    z = np.zeros((G, max(N // 8, 1)), np.uint32)
+    _check(_L().oracle_quantize_with_scales_gs(_p(W), _p(s), N, K, group_size, _p(qw), _p(sc), _p(z)),
            "quantize_with_scales")
     return qw, sc, z
 
@@ -155,10 +162,26 @@ def awq_quantize_g128(W, act_absmean, alpha: float):
     return qw, sc, z, s
 
 
-def dequant(qweight, scales, zeros, N: int, K: int) -> np.ndarray:
+def awq_quantize(W, act_absmean, alpha: float, group_size: int):
+    """AWQ quantize with groups of group_size along K (group_size = K: one group per row)
+    -> (qweight u32 [N][K/8], scales u16 [K/gs][N], zeros u32 [K/gs][N/8], s f32 [K])"""
+    W = _c(W, np.float32)
+    a = _c(act_absmean, np.float32)
+    N, K = W.shape
+    G = max(K // group_size, 1)
+    qw = np.zeros((N, K // 8), np.uint32)
+    sc = np.zeros((G, N), np.uint16)
+    z = np.zeros((G, max(N // 8, 1)), np.uint32)
+    s = np.zeros(K, np.float32)
+    _check(_L().oracle_awq_quantize_gs(_p(W), _p(a), ctypes.c_float(alpha), N, K, group_size, _p(qw), _p(sc),
+                                       _p(z), _p(s)), "awq_quantize")
+    return qw, sc, z, s
+
+
+def dequant(qweight, scales, zeros, N: int, K: int, group_size: int = 128) -> np.ndarray:
     qw, sc, z = _c(qweight, np.uint32), _c(scales, np.uint16), _c(zeros, np.uint32)
     out = np.zeros((N, K), np.float32)
-    _check(_L().oracle_dequant(_p(qw), _p(sc), _p(z), N, K, _p(out)), "dequant")
+    _check(_L().oracle_dequant_gs(_p(qw), _p(sc), _p(z), N, K, group_size, _p(out)), "dequant")
     return out
 
 
@@ -169,7 +192,7 @@ def _csr_args(csr):
     return _c(rp, np.int32), _c(ci, np.int32), _c(v, np.uint16), int(len(ci))
 
 
-def linear(x_bf16_bits, qweight, scales, zeros, N: int, csr=None, with_abs: bool = False):
+def linear(x_bf16_bits, qweight, scales, zeros, N: int, csr=None, with_abs: bool = False, group_size: int = 128):
     """y[m][n] = sum_k x deq + sum_csr x val, in double.  x is bf16 bits (uint16) [M][K].
     csr = (row_ptr int32 [N+1], col_idx int32 [nnz], values fp16 bits [nnz]) or None."""
     x = _c(x_bf16_bits, np.uint16)
@@ -178,13 +201,13 @@ def linear(x_bf16_bits, qweight, scales, zeros, N: int, csr=None, with_abs: bool
     rp, ci, v, nnz = _csr_args(csr)
     y = np.zeros((M, N), np.float64)
     ya = np.zeros((M, N), np.float64) if with_abs else None
-    _check(_L().oracle_linear(_p(x), M, K, _p(qw), _p(sc), _p(z), N, _p(rp), _p(ci), _p(v), nnz,
-                              _p(y), _p(ya)), "linear")
+    _check(_L().oracle_linear_gs(_p(x), M, K, group_size, _p(qw), _p(sc), _p(z), N, _p(rp), _p(ci), _p(v), nnz,
+                                 _p(y), _p(ya)), "linear")
     return (y, ya) if with_abs else y
 
 
 def linear_at(x_bf16_bits, qweight, scales, zeros, N: int, m_idx, n_idx, csr=None,
-              with_abs: bool = False):
+              with_abs: bool = False, group_size: int = 128):
     """The outputs of ``linear`` at the positions (m_idx[p], n_idx[p]) only."""
     x = _c(x_bf16_bits, np.uint16)
     M, K = x.shape
@@ -193,8 +216,8 @@ def linear_at(x_bf16_bits, qweight, scales, zeros, N: int, m_idx, n_idx, csr=Non
     rp, ci, v, nnz = _csr_args(csr)
     y = np.zeros(mi.size, np.float64)
     ya = np.zeros(mi.size, np.float64) if with_abs else None
-    _check(_L().oracle_linear_at(_p(x), M, K, _p(qw), _p(sc), _p(z), N, _p(rp), _p(ci), _p(v), nnz,
-                                 _p(mi), _p(ni), mi.size, _p(y), _p(ya)), "linear_at")
+    _check(_L().oracle_linear_at_gs(_p(x), M, K, group_size, _p(qw), _p(sc), _p(z), N, _p(rp), _p(ci), _p(v),
+                                    nnz, _p(mi), _p(ni), mi.size, _p(y), _p(ya)), "linear_at")
     return (y, ya) if with_abs else y
 
 

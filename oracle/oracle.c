@@ -16,7 +16,9 @@
  *     statement fixes, the pages truncate before it];
  *   - group-wise asymmetric uint4 round-to-nearest on W*s, groups of 128 along K
  *     [DeepCompressor README, perplexity table row "W4A16 g128"; AWQ translation,
- *     section 2 "round-to-nearest (RTN)" and group-wise INT4];
+ *     section 2 "round-to-nearest (RTN)" and group-wise INT4], and the same with other
+ *     group sizes, up to one group per row [SqueezeLLM article, section 4.1: the group
+ *     size option, per-row by default];
  *   - 4-bit weight packing, 8 codes per 32-bit word [AWQ translation, section 1:
  *     TinyChat's 4-bit weight packing];
  *   - the dense-and-sparse product  W x = W_dense x + W_sparse x  with an fp16 CSR
@@ -116,7 +118,7 @@ float oracle_bf16_to_f32(uint16_t h) {
  * Packed format (the interface shared with the CUDA library, restated here):
  *   qweight[n][k/8]  uint32; nibble j (bits 4j..4j+3) holds element k = 8*(k/8) + ORDER[j]
  *                    with ORDER = {0,2,4,6,1,3,5,7};
- *   scales[g][n]     fp16 bits, g = k/128 (group-major);
+ *   scales[g][n]     fp16 bits, g = k/GS (group-major), GS the group size (128 for g128);
  *   zeros[g][n/8]    uint32; nibble j holds the zero point of row 8*(n/8) + j in group g.
  * ---------------------------------------------------------------------------------- */
 static const int ORACLE_ORDER[8] = {0, 2, 4, 6, 1, 3, 5, 7};
@@ -160,15 +162,15 @@ int oracle_awq_scales(const float* act_absmean, int64_t K, float alpha, float* s
     return ORACLE_OK;
 }
 
-/* One group of 128 scaled weights -> fp16 scale bits, zero point, 128 codes.
+/* One group of gs scaled weights -> fp16 scale bits, zero point, gs codes.
  *   scale32 = max((max - min) / 15, 1e-5)          (plain asymmetric min/max range)
  *   sf      = float(fp16_rne(scale32))             (the stored scale is the one used)
  *   z       = clamp(rint(-min / sf), 0, 15)
  *   q_i     = clamp(rint(w_i / sf) + z, 0, 15)     (round first, then add the zero)
  * rint is round-half-to-even; every operation is one IEEE float operation. */
-static int quantize_group(const float* wp, uint16_t* s16_out, uint8_t* z_out, uint8_t* q_out) {
+static int quantize_group(const float* wp, int64_t gs, uint16_t* s16_out, uint8_t* z_out, uint8_t* q_out) {
     float mx = wp[0], mn = wp[0];
-    for (int i = 0; i < GROUP; ++i) {
+    for (int64_t i = 0; i < gs; ++i) {
         if (!isfinite(wp[i])) return ORACLE_ERR_VALUE;
         if (wp[i] > mx) mx = wp[i];
         if (wp[i] < mn) mn = wp[i];
@@ -182,7 +184,7 @@ static int quantize_group(const float* wp, uint16_t* s16_out, uint8_t* z_out, ui
     float zf = rintf(-mn / sf);
     if (zf < 0.0f) zf = 0.0f;
     if (zf > 15.0f) zf = 15.0f;
-    for (int i = 0; i < GROUP; ++i) {
+    for (int64_t i = 0; i < gs; ++i) {
         float qf = rintf(wp[i] / sf) + zf;
         if (qf < 0.0f) qf = 0.0f;
         if (qf > 15.0f) qf = 15.0f;
@@ -198,43 +200,60 @@ static int check_qshape(int64_t N, int64_t K) {
     return ORACLE_OK;
 }
 
+/* group size: a multiple of 8 (whole packed words) that divides K */
+static int check_gs(int64_t K, int64_t gs) {
+    if (gs <= 0 || gs % 8 != 0 || K % gs != 0) return ORACLE_ERR_SHAPE;
+    return ORACLE_OK;
+}
+
 static int zero_of(const uint32_t* zeros, int64_t N, int64_t n, int64_t g) {
     return (int)((zeros[g * (N / 8) + n / 8] >> (4 * (n % 8))) & 15u);
 }
 
-/* Quantize W (fp32 [N][K]) with a given per-channel scale s ([K]):
- * w' = float(w * s_k), then quantize_group on each run of 128 along K, then pack. */
-int oracle_quantize_with_scales(const float* W, const float* s, int64_t N, int64_t K,
-                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros) {
+/* Quantize W (fp32 [N][K]) with a given per-channel scale s ([K]) in groups of gs along K:
+ * w' = float(w * s_k), then quantize_group on each run of gs along K, then pack. */
+int oracle_quantize_with_scales_gs(const float* W, const float* s, int64_t N, int64_t K, int64_t gs,
+                                   uint32_t* qweight, uint16_t* scales, uint32_t* zeros) {
     if (!W || !s || !qweight || !scales || !zeros) return ORACLE_ERR_NULL;
     int st = check_qshape(N, K);
+    if (!st) st = check_gs(K, gs);
     if (st) return st;
-    const int64_t G = K / GROUP;
+    const int64_t G = K / gs;
     int err = ORACLE_OK;
     uint8_t* zcode = (uint8_t*)malloc((size_t)(N * G));
     if (!zcode) return ORACLE_ERR_VALUE;
-#pragma omp parallel for schedule(dynamic, 4)
-    for (int64_t n = 0; n < N; ++n) {
-        float wp[GROUP];
-        uint8_t q[GROUP];
-        for (int64_t g = 0; g < G; ++g) {
-            for (int i = 0; i < GROUP; ++i) wp[i] = W[n * K + g * GROUP + i] * s[g * GROUP + i];
-            uint16_t s16;
-            uint8_t z;
-            int e = quantize_group(wp, &s16, &z, q);
-            if (e) {
+#pragma omp parallel
+    {
+        float* wp = (float*)malloc(sizeof(float) * (size_t)gs);
+        uint8_t* q = (uint8_t*)malloc((size_t)gs);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t n = 0; n < N; ++n) {
+            if (!wp || !q) {
 #pragma omp atomic write
-                err = e;
+                err = ORACLE_ERR_VALUE;
                 continue;
             }
-            scales[g * N + n] = s16;
-            zcode[n * G + g] = z;
-            for (int w = 0; w < GROUP / 8; ++w) {
-                uint32_t word;
-                oracle_pack8(&q[8 * w], &word);
-                qweight[n * (K / 8) + g * (GROUP / 8) + w] = word;
+            for (int64_t g = 0; g < G; ++g) {
+                for (int64_t i = 0; i < gs; ++i) wp[i] = W[n * K + g * gs + i] * s[g * gs + i];
+                uint16_t s16;
+                uint8_t z;
+                int e = quantize_group(wp, gs, &s16, &z, q);
+                if (e) {
+#pragma omp atomic write
+                    err = e;
+                    continue;
+                }
+                scales[g * N + n] = s16;
+                zcode[n * G + g] = z;
+                for (int64_t w = 0; w < gs / 8; ++w) {
+                    uint32_t word;
+                    oracle_pack8(&q[8 * w], &word);
+                    qweight[n * (K / 8) + g * (gs / 8) + w] = word;
+                }
             }
         }
+        free(wp);
+        free(q);
     }
     /* zero points packed along n: nibble j of zeros[g][n/8] is row 8*(n/8) + j */
     for (int64_t g = 0; g < G; ++g)
@@ -247,32 +266,45 @@ int oracle_quantize_with_scales(const float* W, const float* s, int64_t N, int64
     return err;
 }
 
-/* awq_quantize_g128: the scale from act_absmean and alpha, then quantize W*s. */
-int oracle_awq_quantize_g128(const float* W, const float* act_absmean, float alpha, int64_t N,
-                             int64_t K, uint32_t* qweight, uint16_t* scales, uint32_t* zeros,
-                             float* s_out) {
+int oracle_quantize_with_scales(const float* W, const float* s, int64_t N, int64_t K,
+                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros) {
+    return oracle_quantize_with_scales_gs(W, s, N, K, GROUP, qweight, scales, zeros);
+}
+
+/* awq_quantize with group size gs: the scale from act_absmean and alpha, then quantize W*s. */
+int oracle_awq_quantize_gs(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                           int64_t gs, uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out) {
     if (!W || !act_absmean || !qweight || !scales || !zeros) return ORACLE_ERR_NULL;
     int st = check_qshape(N, K);
+    if (!st) st = check_gs(K, gs);
     if (st) return st;
     float* s = (float*)malloc(sizeof(float) * (size_t)K);
     if (!s) return ORACLE_ERR_VALUE;
     st = oracle_awq_scales(act_absmean, K, alpha, s);
-    if (!st) st = oracle_quantize_with_scales(W, s, N, K, qweight, scales, zeros);
+    if (!st) st = oracle_quantize_with_scales_gs(W, s, N, K, gs, qweight, scales, zeros);
     if (!st && s_out) memcpy(s_out, s, sizeof(float) * (size_t)K);
     free(s);
     return st;
 }
 
+/* awq_quantize_g128: the scale from act_absmean and alpha, then quantize W*s. */
+int oracle_awq_quantize_g128(const float* W, const float* act_absmean, float alpha, int64_t N,
+                             int64_t K, uint32_t* qweight, uint16_t* scales, uint32_t* zeros,
+                             float* s_out) {
+    return oracle_awq_quantize_gs(W, act_absmean, alpha, N, K, GROUP, qweight, scales, zeros, s_out);
+}
+
 /* deq[n][k] = (q - z) * sf, exact in fp32 (a 5-bit integer times an 11-bit scale). */
-int oracle_dequant(const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
-                   int64_t N, int64_t K, float* deq) {
+int oracle_dequant_gs(const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
+                      int64_t N, int64_t K, int64_t gs, float* deq) {
     if (!qweight || !scales || !zeros || !deq) return ORACLE_ERR_NULL;
     int st = check_qshape(N, K);
+    if (!st) st = check_gs(K, gs);
     if (st) return st;
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
         for (int64_t k = 0; k < K; ++k) {
-            int64_t g = k / GROUP;
+            int64_t g = k / gs;
             uint8_t codes[8];
             oracle_unpack8(qweight[n * (K / 8) + k / 8], codes);
             int q = codes[k % 8];
@@ -282,6 +314,11 @@ int oracle_dequant(const uint32_t* qweight, const uint16_t* scales, const uint32
         }
     }
     return ORACLE_OK;
+}
+
+int oracle_dequant(const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
+                   int64_t N, int64_t K, float* deq) {
+    return oracle_dequant_gs(qweight, scales, zeros, N, K, GROUP, deq);
 }
 
 static int check_csr(const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
@@ -303,13 +340,13 @@ static int check_csr(const int32_t* row_ptr, const int32_t* col_idx, const uint1
 /* One output y[m][n] = sum_k x[m][k] deq[n][k] + sum_{j in row n} x[m][col_j] val_j, summed
  * in double (each product of a bf16 and a dequantized weight or fp16 value is exact in
  * double), plus the sum of the absolute products, which bounds any rounding error. */
-static void one_output(const uint16_t* x, int64_t K, int64_t N, const uint32_t* qweight,
+static void one_output(const uint16_t* x, int64_t K, int64_t N, int64_t gs, const uint32_t* qweight,
                        const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
                        const int32_t* col_idx, const uint16_t* values, int64_t m, int64_t n,
                        double* y, double* yabs) {
     double acc = 0.0, aacc = 0.0;
     for (int64_t k = 0; k < K; ++k) {
-        int64_t g = k / GROUP;
+        int64_t g = k / gs;
         uint8_t codes[8];
         oracle_unpack8(qweight[n * (K / 8) + k / 8], codes);
         int q = codes[k % 8];
@@ -334,33 +371,42 @@ static void one_output(const uint16_t* x, int64_t K, int64_t N, const uint32_t* 
 /* y = x deq(Q)^T + x W_sparse^T for all (m, n): x bf16 [M][K]; y, yabs double [M][N].
  * The CSR (row_ptr [N+1], col_idx/values [nnz], ascending columns per row) may be absent
  * (row_ptr == NULL and nnz == 0). */
-int oracle_linear(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweight,
-                  const uint16_t* scales, const uint32_t* zeros, int64_t N,
-                  const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
-                  int64_t nnz, double* y, double* yabs) {
+int oracle_linear_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, const uint32_t* qweight,
+                     const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                     const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                     int64_t nnz, double* y, double* yabs) {
     if (!x || !qweight || !scales || !zeros || !y) return ORACLE_ERR_NULL;
     if (M <= 0) return ORACLE_ERR_SHAPE;
     int st = check_qshape(N, K);
+    if (!st) st = check_gs(K, gs);
     if (st) return st;
     st = check_csr(row_ptr, col_idx, values, nnz, N, K);
     if (st) return st;
 #pragma omp parallel for collapse(2) schedule(dynamic, 16)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n)
-            one_output(x, K, N, qweight, scales, zeros, row_ptr, col_idx, values, m, n,
+            one_output(x, K, N, gs, qweight, scales, zeros, row_ptr, col_idx, values, m, n,
                        &y[m * N + n], yabs ? &yabs[m * N + n] : NULL);
     return ORACLE_OK;
 }
 
+int oracle_linear(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweight,
+                  const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                  const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                  int64_t nnz, double* y, double* yabs) {
+    return oracle_linear_gs(x, M, K, GROUP, qweight, scales, zeros, N, row_ptr, col_idx, values, nnz, y, yabs);
+}
+
 /* The same outputs at P sampled positions (m_idx[p], n_idx[p]) only. */
-int oracle_linear_at(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweight,
-                     const uint16_t* scales, const uint32_t* zeros, int64_t N,
-                     const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
-                     int64_t nnz, const int64_t* m_idx, const int64_t* n_idx, int64_t P,
-                     double* y, double* yabs) {
+int oracle_linear_at_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, const uint32_t* qweight,
+                        const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                        const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                        int64_t nnz, const int64_t* m_idx, const int64_t* n_idx, int64_t P,
+                        double* y, double* yabs) {
     if (!x || !qweight || !scales || !zeros || !y || !m_idx || !n_idx) return ORACLE_ERR_NULL;
     if (M <= 0 || P < 0) return ORACLE_ERR_SHAPE;
     int st = check_qshape(N, K);
+    if (!st) st = check_gs(K, gs);
     if (st) return st;
     st = check_csr(row_ptr, col_idx, values, nnz, N, K);
     if (st) return st;
@@ -368,9 +414,18 @@ int oracle_linear_at(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qw
         if (m_idx[p] < 0 || m_idx[p] >= M || n_idx[p] < 0 || n_idx[p] >= N) return ORACLE_ERR_SHAPE;
 #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t p = 0; p < P; ++p)
-        one_output(x, K, N, qweight, scales, zeros, row_ptr, col_idx, values, m_idx[p], n_idx[p],
+        one_output(x, K, N, gs, qweight, scales, zeros, row_ptr, col_idx, values, m_idx[p], n_idx[p],
                    &y[p], yabs ? &yabs[p] : NULL);
     return ORACLE_OK;
+}
+
+int oracle_linear_at(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweight,
+                     const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                     const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                     int64_t nnz, const int64_t* m_idx, const int64_t* n_idx, int64_t P,
+                     double* y, double* yabs) {
+    return oracle_linear_at_gs(x, M, K, GROUP, qweight, scales, zeros, N, row_ptr, col_idx, values, nnz, m_idx,
+                               n_idx, P, y, yabs);
 }
 
 /* ------------------------------------------------------------------------------------

@@ -506,3 +506,101 @@ def test_search_scaling_protects_a_salient_channel(orc):
 def torch_bf16(a):
     import torch
     return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+# ------------------------------------------------------------------ other group sizes -----
+# [SqueezeLLM article, section 4.1: the group size option, per-row by default]
+
+def _equal_range_layer(rng, N, K, gs):
+    """W whose every 128-wide slice of a group of gs holds that group's minimum and maximum,
+    so quantizing with groups of gs and with groups of 128 must agree code for code."""
+    W = rng.uniform(-0.9, 0.9, size=(N, K)).astype(np.float32)
+    for n in range(N):
+        for g in range(K // gs):
+            mn, mx = -1.0 - rng.uniform(0, 2), 1.0 + rng.uniform(0, 2)
+            for c in range(g * gs, (g + 1) * gs, 128):
+                W[n, c + rng.integers(0, 64)] = mn
+                W[n, c + 64 + rng.integers(0, 64)] = mx
+    return W
+
+
+@pytest.mark.parametrize("gs", [256, 1024, 2048, 4096])
+def test_groups_of_equal_range_reduce_to_g128(orc, gs):
+    N, K = 16, 4096
+    rng = np.random.default_rng(gs)
+    W = _equal_range_layer(rng, N, K, gs)
+    act = np.ones(K, np.float32)                           # s = 1 for any alpha
+    qa, sa, za, _ = orc.awq_quantize(W, act, 0.5, gs)
+    qb, sb, zb, _ = orc.awq_quantize_g128(W, act, 0.5)
+    R = gs // 128
+    assert np.array_equal(qa, qb)
+    assert np.array_equal(np.repeat(sa, R, axis=0), sb)
+    assert np.array_equal(np.repeat(za, R, axis=0), zb)
+    assert sa.shape == (K // gs, N) and za.shape == (K // gs, N // 8)
+
+
+@pytest.mark.parametrize("gs", [256, 512, 5120])
+def test_group_rtn_error_bound(orc, gs):
+    """Round-to-nearest with each element's own group parameters: |deq - w s| <= 1.5 sf_g
+    (half a step, plus one step where the fp16-rounded scale makes the top code clamp)."""
+    N, K = 24, 5120
+    rng = np.random.default_rng(gs + 1)
+    W = (rng.standard_normal((N, K)) * rng.uniform(0.01, 2.0, size=(N, 1))).astype(np.float32)
+    act = np.exp(rng.uniform(-3, 3, K)).astype(np.float32)
+    qw, sc, z, s = orc.awq_quantize(W, act, 0.5, gs)
+    deq = orc.dequant(qw, sc, z, N, K, group_size=gs).astype(np.float64)
+    ws = (W * s[None, :]).astype(np.float64)               # one IEEE product per element
+    sf = sc.view(np.float16).astype(np.float64).T          # [N][K/gs]
+    step = np.repeat(sf, gs, axis=1)
+    assert np.all(np.abs(deq - ws) <= 1.5 * step + 1e-12)
+    # every group's range is covered: its extremes land within one step of the group's min/max
+    for g in range(K // gs):
+        blk = slice(g * gs, (g + 1) * gs)
+        assert np.all(np.abs(deq[:, blk].max(1) - ws[:, blk].max(1)) <= 1.5 * sf[:, g] + 1e-12)
+        assert np.all(np.abs(deq[:, blk].min(1) - ws[:, blk].min(1)) <= 1.5 * sf[:, g] + 1e-12)
+
+
+def test_group_dequant_closed_form(orc):
+    """Hand-packed codes q = (n + 3k) mod 16, scales 2^(g mod 5 - 2), zeros (g + n) mod 16."""
+    N, K, gs = 16, 2048, 512
+    G = K // gs
+    n_i, k_i = np.meshgrid(np.arange(N), np.arange(K), indexing="ij")
+    q = (n_i + 3 * k_i) % 16
+    qw = np.zeros((N, K // 8), np.uint32)
+    for n in range(N):
+        for w in range(K // 8):
+            qw[n, w] = orc.pack8(q[n, 8 * w: 8 * w + 8])
+    g_i = np.arange(G)
+    sc = np.repeat((2.0 ** (g_i % 5 - 2)).astype(np.float16).view(np.uint16)[:, None], N, axis=1)
+    zg = (g_i[:, None] + np.arange(N)[None, :]) % 16           # [G][N]
+    zeros = np.zeros((G, N // 8), np.uint32)
+    for j in range(8):
+        zeros |= (zg[:, j::8].astype(np.uint32) << np.uint32(4 * j))
+    deq = orc.dequant(qw, sc, zeros, N, K, group_size=gs)
+    expect = (q - zg.T[:, k_i[0] // gs]) * (2.0 ** (k_i // gs % 5 - 2))
+    assert np.array_equal(deq.astype(np.float64), expect)
+
+
+@pytest.mark.parametrize("gs", [256, 2048])
+def test_group_linear_is_x_times_dequant(orc, gs):
+    """The product with groups of gs equals numpy's matmul of x and the dequantized weights."""
+    N, K, M = 40, 2048, 3
+    rng = np.random.default_rng(gs + 2)
+    W = rng.standard_normal((N, K)).astype(np.float32) * 0.05
+    act = np.exp(rng.uniform(-2, 2, K)).astype(np.float32)
+    qw, sc, z, _ = orc.awq_quantize(W, act, 0.5, gs)
+    x = _torch_bf16_bits(rng.standard_normal((M, K)))
+    y = orc.linear(x, qw, sc, z, N, group_size=gs)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = xf @ orc.dequant(qw, sc, z, N, K, group_size=gs).astype(np.float64).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+    m, n = np.array([0, 2, 1]), np.array([5, 39, 0])
+    assert np.allclose(orc.linear_at(x, qw, sc, z, N, m, n, group_size=gs), ref[m, n], rtol=1e-12, atol=1e-12)
+
+
+def test_group_size_validation(orc):
+    W = np.zeros((8, 2048), np.float32)
+    a = np.ones(2048, np.float32)
+    for gs in (0, 100, 3072, 4096):
+        with pytest.raises(Exception):
+            orc.awq_quantize(W, a, 0.5, gs)
