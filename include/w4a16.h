@@ -106,6 +106,20 @@ w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float a
                                float* s_out, void* stream);
 
 /*
+ * awq_quantize -- awq_quantize_g128 with groups of group_size weights along K instead of 128
+ * [SqueezeLLM article, 4.1: the group size option, one group per row by default].
+ *   group_size   128, 256, 512, 1024, or a multiple of 1024 that divides K and is at most
+ *                32768.  group_size = K gives one scale and zero point per output channel.
+ *   scales       [K/group_size][N] fp16 bits; zeros [K/group_size][N/8] uint32.
+ *   Everything else, including the arithmetic per group, is as for awq_quantize_g128.
+ *   Groups above 1024 are read twice from device memory: once for their range, once to
+ *   quantize.  Errors: as awq_quantize_g128, plus SHAPE for an unsupported group_size.
+ */
+w4a16_status awq_quantize(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                          int64_t group_size, uint32_t* qweight, uint16_t* scales, uint32_t* zeros,
+                          float* s_out, void* stream);
+
+/*
  * Workspace of the decode path.  The GEMV splits the output row blocks evenly over a
  * persistent grid.  Row blocks shared by two or more CTAs are combined through fp32
  * partial tiles and per-row-block counters, which live in a caller-provided device
@@ -190,6 +204,16 @@ w4a16_status w4a16_gemv_ex(const uint16_t* x, const uint32_t* qweight, const uin
  * SHAPE for invalid sizes (as w4a16_gemv), UNSUPPORTED as w4a16_gemv_ex. */
 w4a16_status w4a16_gemv_plan(int64_t M, int64_t N, int64_t K, int schedule, int* resolved,
                              int* cluster_size, int* ctas);
+
+/* w4a16_linear_ex -- w4a16_linear for weights quantized in groups of group_size along K
+ * (awq_quantize), with the decode GEMV's schedule (w4a16_gemv_schedule; ignored when
+ * M > 16).  group_size: a multiple of 128 that divides K; scales and zeros have
+ * K/group_size groups.  SHAPE for another group_size, VALUE for an unknown schedule.
+ * Everything else is as for w4a16_linear. */
+w4a16_status w4a16_linear_ex(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                             const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
+                             int64_t M, int64_t N, int64_t K, int64_t group_size, void* workspace,
+                             size_t workspace_bytes, int schedule, void* stream);
 
 /* w4a16_gemm -- the tcgen05 tensor-core path of w4a16_linear, for any M >= 1.  Arguments
  * and result are as for w4a16_linear.  The workspace is not used (NULL and 0 are fine).

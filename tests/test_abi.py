@@ -117,6 +117,26 @@ def test_quantize_validation(L):
     assert q(alpha=float("inf")) == w4.ERR_VALUE
 
 
+def test_grouped_validation(L):
+    def q(gs, N=128, K=4096, W=FAKE):
+        return L.awq_quantize(ctypes.c_void_p(W), ctypes.c_void_p(FAKE), ctypes.c_float(0.5), N, K, gs,
+                              ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), None, None)
+    for gs in (0, 64, 100, 384, 1536, 3072, 8192, 65536):
+        assert q(gs) == w4.ERR_SHAPE, gs
+    assert q(256, W=0) == w4.ERR_NULL
+    assert q(2048, K=5120) == w4.ERR_SHAPE            # 2048 does not divide 5120
+    assert q(40960, K=40960) == w4.ERR_SHAPE          # above 32768
+
+    def lx(gs, schedule=0, K=4096, M=1):
+        return L.w4a16_linear_ex(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE),
+                                 ctypes.c_void_p(FAKE), None, ctypes.c_void_p(FAKE), M, 128, K, gs,
+                                 ctypes.c_void_p(FAKE), 1 << 30, schedule, None)
+    for gs in (0, 64, 192, 3072, 8192):
+        assert lx(gs) == w4.ERR_SHAPE, gs
+    assert lx(256, schedule=5) == w4.ERR_VALUE
+    assert lx(2048, K=5120) == w4.ERR_SHAPE            # 2048 does not divide 5120
+
+
 def test_split_validation(L):
     def sp(W=FAKE, a=FAKE, alpha=0.5, N=16, K=256, nnz=10, Wd=FAKE, rp=FAKE, ci=FAKE, v=FAKE, ws=FAKE, wsb=1 << 30):
         return L.awq_split_outliers(ctypes.c_void_p(W), ctypes.c_void_p(a), ctypes.c_float(alpha), N, K, nnz,

@@ -5,9 +5,11 @@ kernels.  PyTorch provides device memory and the current stream.  The entry poin
 mirror the C ABI in include/w4a16.h:
 
   awq_quantize_g128(W, act_absmean, alpha)      -> (qweight, scales, zeros, s)
+  awq_quantize(W, act_absmean, alpha, gs)       -> the same with groups of gs along K (gs = K: per row)
   w4a16_linear(x, qweight, scales, zeros, csr)  -> y      (any M)
   w4a16_gemv(...)                               -> y      (1 <= M <= 16)
   w4a16_gemv_ex(..., schedule)                  -> y      (GEMV_AUTO, GEMV_STREAM_K or GEMV_CLUSTER)
+  w4a16_linear_ex(..., group_size, schedule)    -> y      (weights from awq_quantize with that group size)
   gemv_plan(M, N, K, schedule)                  -> (schedule, cluster size, CTAs) the call would launch
   w4a16_gemm(...)                               -> y      (tcgen05 path, any M)
   workspace_bytes(M, N, K)                      -> bytes of zeroed device workspace a decode call needs
@@ -64,6 +66,9 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, I64, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
         L.awq_quantize_g128.argtypes = [P, P, F, I64, I64, P, P, P, P, P]
+        L.awq_quantize.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P]
+        L.w4a16_linear_ex.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, I64, P, ctypes.c_size_t,
+                                      ctypes.c_int, P]
         for name in ("w4a16_linear", "w4a16_gemv", "w4a16_gemm"):
             fn = getattr(L, name)
             fn.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P, ctypes.c_size_t, P]
@@ -85,7 +90,7 @@ def lib() -> ctypes.CDLL:
         L.w4a16_status_string.argtypes = [ctypes.c_int]
         L.w4a16_status_string.restype = ctypes.c_char_p
         L.w4a16_version.argtypes = []
-        for name in ("awq_quantize_g128", "w4a16_linear", "w4a16_gemv", "w4a16_gemv_ex", "w4a16_gemv_plan",
+        for name in ("awq_quantize_g128", "awq_quantize", "w4a16_linear_ex", "w4a16_linear", "w4a16_gemv", "w4a16_gemv_ex", "w4a16_gemv_plan",
                      "w4a16_gemm", "w4a16_check_device_status",
                      "w4a16_selftest_timeout", "awq_split_outliers", "awq_search_alpha", "awq_fold_activations", "w4a16_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -110,6 +115,26 @@ def _need(t, dtype, ndim, name):
     if not (t.is_cuda and t.dtype == dtype and t.dim() == ndim and t.is_contiguous()):
         raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor of rank {ndim}, got "
                          f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def awq_quantize(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, group_size: int, out=None):
+    """awq_quantize_g128 with groups of group_size along K -> (qweight int32 [N][K/8],
+    scales int16 [K/gs][N], zeros int32 [K/gs][N/8], s fp32 [K])."""
+    _need(W, torch.float32, 2, "W")
+    _need(act_absmean, torch.float32, 1, "act_absmean")
+    N, K = W.shape
+    dev = W.device
+    G = max(K // max(group_size, 1), 1)
+    if out is None:
+        out = (torch.empty(N, K // 8, dtype=torch.int32, device=dev),
+               torch.empty(G, N, dtype=torch.int16, device=dev),
+               torch.empty(G, max(N // 8, 1), dtype=torch.int32, device=dev),
+               torch.empty(K, dtype=torch.float32, device=dev))
+    qw, sc, z, s = out
+    code = lib().awq_quantize(_ptr(W), _ptr(act_absmean), ctypes.c_float(alpha), N, K, int(group_size), _ptr(qw),
+                              _ptr(sc), _ptr(z), _ptr(s), _stream(dev))
+    _check(code, "awq_quantize")
+    return qw, sc, z, s
 
 
 def awq_quantize_g128(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, out=None):
@@ -152,7 +177,7 @@ def workspace_bytes(M: int, N: int, K: int) -> int:
     return int(lib().w4a16_workspace_bytes(M, N, K))
 
 
-def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, schedule=None):
+def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, schedule=None, group_size=None):
     _need(x, torch.bfloat16, 2, "x")
     _need(qweight, torch.int32, 2, "qweight")
     _need(scales, torch.int16, 2, "scales")
@@ -172,7 +197,10 @@ def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, s
     if ws is None and need > 0:
         ws = workspace(x.device, need)
     args = [_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), ctypes.byref(cs) if cs is not None else None,
-            _ptr(y), M, N, K, _ptr(ws), ws.numel() if ws is not None else 0]
+            _ptr(y), M, N, K]
+    if group_size is not None:
+        args.append(int(group_size))
+    args += [_ptr(ws), ws.numel() if ws is not None else 0]
     if schedule is not None:
         args.append(int(schedule))
     code = getattr(lib(), name)(*args, _stream(x.device))
@@ -191,6 +219,12 @@ def w4a16_gemv(x, qweight, scales, zeros, csr=None, out=None, workspace=None):
 
 def w4a16_gemv_ex(x, qweight, scales, zeros, csr=None, out=None, workspace=None, schedule=GEMV_AUTO):
     return _linear("w4a16_gemv_ex", x, qweight, scales, zeros, csr, out, workspace, schedule)
+
+
+def w4a16_linear_ex(x, qweight, scales, zeros, csr=None, out=None, workspace=None, group_size=128,
+                    schedule=GEMV_AUTO):
+    """w4a16_linear for weights quantized in groups of group_size along K."""
+    return _linear("w4a16_linear_ex", x, qweight, scales, zeros, csr, out, workspace, schedule, group_size)
 
 
 def gemv_plan(M: int, N: int, K: int, schedule: int = GEMV_AUTO):

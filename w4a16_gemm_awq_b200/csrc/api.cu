@@ -116,6 +116,7 @@ struct LinearArgs {
     long long nnz = 0;
     uint16_t* y;
     int64_t M, N, K;
+    int group_ratio = 1;  // group size / 128
     void* workspace = nullptr;
     size_t workspace_bytes = 0;
 };
@@ -180,7 +181,7 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4A16_ERR_CUDA;
     }
-    return from_cuda(launch_gemv(maps, plan, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
+    return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
                                  a.workspace, (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status, stream));
 }
 
@@ -220,7 +221,7 @@ w4a16_status run_gemm(const LinearArgs& a, cudaStream_t stream) {
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4A16_ERR_CUDA;
     }
-    return from_cuda(launch_gemm(maps, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y, (int)a.M,
+    return from_cuda(launch_gemm(maps, a.group_ratio, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y, (int)a.M,
                                  (int)a.N, (int)a.K, bn, d->num_sms, d->status, stream));
 }
 
@@ -256,10 +257,12 @@ using namespace w4a16;
 
 extern "C" {
 
-w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
-                               uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, void* stream) {
+w4a16_status awq_quantize(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                          int64_t group_size, uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out,
+                          void* stream) {
     if (!W || !act_absmean || !qweight || !scales || !zeros) return W4A16_ERR_NULL;
     if (N < 8 || N % 8 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK) return W4A16_ERR_SHAPE;
+    if (group_size < 128 || group_size > K || !quantize_group_size_ok((int)K, (int)group_size)) return W4A16_ERR_SHAPE;
     if (!aligned(W, 16) || !aligned(act_absmean, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
         !aligned(zeros, 16) || (s_out && !aligned(s_out, 16)))
         return W4A16_ERR_ALIGN;
@@ -267,8 +270,13 @@ w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float a
     DeviceInfo* d = nullptr;
     w4a16_status st = device_info(&d);
     if (st != W4A16_OK) return st;
-    return from_cuda(launch_awq_quantize(W, act_absmean, alpha, (int)N, (int)K, qweight, scales, zeros, s_out,
-                                         d->status, static_cast<cudaStream_t>(stream)));
+    return from_cuda(launch_awq_quantize(W, act_absmean, alpha, (int)N, (int)K, (int)group_size, qweight, scales,
+                                         zeros, s_out, d->status, static_cast<cudaStream_t>(stream)));
+}
+
+w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                               uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, void* stream) {
+    return awq_quantize(W, act_absmean, alpha, N, K, 128, qweight, scales, zeros, s_out, stream);
 }
 
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -342,6 +350,23 @@ w4a16_status w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint
     a.workspace_bytes = workspace_bytes;
     const bool decode = M <= 16 && K <= gemv_max_k();
     return decode ? run_gemv(a, static_cast<cudaStream_t>(stream)) : run_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
+w4a16_status w4a16_linear_ex(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                             const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N,
+                             int64_t K, int64_t group_size, void* workspace, size_t workspace_bytes, int schedule,
+                             void* stream) {
+    LinearArgs a;
+    w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
+    if (st != W4A16_OK) return st;
+    if (group_size < 128 || group_size % 128 != 0 || group_size > K || K % group_size != 0) return W4A16_ERR_SHAPE;
+    if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
+    a.group_ratio = (int)(group_size / 128);
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    const bool decode = M <= 16 && K <= gemv_max_k();
+    return decode ? run_gemv(a, static_cast<cudaStream_t>(stream), schedule)
+                  : run_gemm(a, static_cast<cudaStream_t>(stream));
 }
 
 w4a16_status w4a16_gemv_noalloc(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -442,7 +467,7 @@ w4a16_status awq_search_alpha(const float* W, const float* act_absmean, const ui
     if (M <= 16 && cudaMemsetAsync(ws + L.gemv, 0, L.total - L.gemv, s) != cudaSuccess) return W4A16_ERR_CUDA;
     st = from_cuda(launch_search_ref(x_calib, W, yref, (int)M, (int)N, (int)K, s));
     for (int i = 0; i < n_alpha && st == W4A16_OK; ++i) {
-        st = from_cuda(launch_awq_quantize(W, act_absmean, alphas[i], (int)N, (int)K, qw, sc, z, sv, d->status, s));
+        st = from_cuda(launch_awq_quantize(W, act_absmean, alphas[i], (int)N, (int)K, 128, qw, sc, z, sv, d->status, s));
         if (st != W4A16_OK) break;
         st = from_cuda(launch_search_fold(x_calib, sv, xs, (int)M, (int)K, s));
         if (st != W4A16_OK) break;

@@ -49,6 +49,7 @@ struct GemmArgs {
     long long nnz;
     uint16_t* y;
     int M, N, K;
+    int gr;  // quantization group size / 128: scales and zeros of 128-slice g are those of group g / gr
     unsigned* err;
 };
 
@@ -158,7 +159,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 tma_load_2d(smem + L::kXOff + slot * L::kXStageBytes, &map_x, &full[slot], s * kBK, m0);
                 tma_load_2d(smem + L::kWOff + slot * kWStageBytes, &map_w, &full[slot], s * (kBK / 8), n0);
                 if (first_half) {
-                    const int g = s >> 1;
+                    const int g = (s >> 1) / p.gr;  // the quantization group of this 128-slice
                     uint8_t* par = smem + L::kParOff + slot * 512;
                     bulk_load(par, p.scales + (size_t)g * p.N + n0, 256, &full[slot]);
                     bulk_load(par + 256, p.zeros + (size_t)g * (p.N >> 3) + (n0 >> 3), 64, &full[slot]);
@@ -332,10 +333,10 @@ static cudaError_t launch_bn(const GemmMaps& maps, const GemmArgs& a, cudaStream
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(const GemmMaps& maps, const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
+cudaError_t launch_gemm(const GemmMaps& maps, int group_ratio, const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
                         const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, int M, int N,
                         int K, int bn, int /*num_sms*/, unsigned* err, cudaStream_t stream) {
-    GemmArgs a{scales, zeros, row_ptr, col_idx, vals, nnz, y, M, N, K, err};
+    GemmArgs a{scales, zeros, row_ptr, col_idx, vals, nnz, y, M, N, K, group_ratio, err};
     switch (bn) {
         case 32: return launch_bn<32>(maps, a, stream);
         case 64: return launch_bn<64>(maps, a, stream);

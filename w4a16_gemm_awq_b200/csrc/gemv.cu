@@ -94,6 +94,7 @@ struct GemvArgs {
     int M, N, K;
     uint32_t T;          // work units = (N/128) * (K/512); T * P < 2^32 (checked by the caller)
     int P;               // CTAs
+    int gr;              // quantization group size / 128: scales and zeros of 128-slice g are those of group g / gr
     int cl;              // 0: stream-K; else the cluster size of the cluster split-K (2..8, <= K/512)
     int ncl;             // cluster split-K: clusters (<= N/128); cluster j takes row blocks j, j + ncl, ...
     unsigned* err;
@@ -331,7 +332,7 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
             uint32_t zw[2];
 #pragma unroll
             for (int gg = 0; gg < 2; ++gg) {
-                const int g = gb * kGemvUnitGroups + 2 * h + gg;
+                const int g = (gb * kGemvUnitGroups + 2 * h + gg) / p.gr;  // the quantization group
                 scv[gg] = __ldg(reinterpret_cast<const uint2*>(p.scales + (size_t)g * p.N + (size_t)rb * kGemvRows) + lane);
                 zw[gg] = __ldg(p.zeros + (size_t)g * (p.N >> 3) + (size_t)rb * (kGemvRows / 8) + (lane >> 1));
             }
@@ -889,7 +890,7 @@ GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule) {
     return best;
 }
 
-cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
+cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
                         const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
                         uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
                         cudaStream_t stream) {
@@ -907,6 +908,7 @@ cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, const uint16
     a.K = K;
     a.T = (uint32_t)((N / kGemvRows) * (K / (128 * kGemvUnitGroups)));
     a.P = plan.ctas;
+    a.gr = group_ratio;
     a.cl = plan.cluster;
     a.ncl = plan.clusters;
     a.err = err;

@@ -12,8 +12,13 @@ namespace w4a16 {
 // Bits of the per-device status word that kernels set when they find a problem.
 enum : unsigned { kErrValue = 1u, kErrShape = 2u, kErrTimeout = 4u };
 
-cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, uint32_t* qweight,
-                                uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
+// Group sizes the quantizer supports: 128, 256, 512, 1024, or a multiple of 1024 that
+// divides K, up to kQuantMaxLargeGroup (its scales sit in shared memory).
+constexpr int kQuantMaxLargeGroup = 32768;
+bool quantize_group_size_ok(int K, int gs);
+
+cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, int gs,
+                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
                                 cudaStream_t stream);
 
 // Tensor map the GEMV needs: qweight uint32 [N][K/8] seen as 3-D (16 words of a group,
@@ -44,7 +49,8 @@ struct GemvPlan {
 // The launch for a schedule (W4A16_GEMV_AUTO, _STREAM_K or _CLUSTER) on the current device.
 GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule);
 
-cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
+// group_ratio: the quantization group size / 128 (1 for g128; K / 128 for one group per row)
+cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
                         const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
                         uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
                         cudaStream_t stream);
@@ -71,7 +77,7 @@ struct GemmMaps {
     CUtensorMap qw;  // uint32 [N][K/8], box 16 words (one group) x 128 rows, 64-byte swizzle
 };
 
-cudaError_t launch_gemm(const GemmMaps& maps, const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
+cudaError_t launch_gemm(const GemmMaps& maps, int group_ratio, const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
                         const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, int M, int N,
                         int K, int bn, int num_sms, unsigned* err, cudaStream_t stream);
 

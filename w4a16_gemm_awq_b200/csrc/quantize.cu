@@ -53,14 +53,17 @@ __device__ __forceinline__ uint32_t place_nibbles(const float q[4], bool odd) {
     return (q0 << 8) | (q1 << 24) | (q2 << 12) | (q3 << 28);
 }
 
+// Groups of 128 R weights, R in {1, 2, 4, 8}: a 1024-column chunk holds 8 / R whole groups.
+template <int R>
 __global__ void __launch_bounds__(kQuantThreads)
 awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, float alpha, int N, int K,
                     uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
                     uint32_t* __restrict__ zeros, float* __restrict__ s_out, unsigned* err) {
+    constexpr int GC = 8 / R;  // groups per chunk
     __shared__ __align__(16) float s_sm[1024];
-    __shared__ __align__(16) uint16_t sc_sm[8][kRowsPerCta];  // fp16 scale bits per (group, row)
-    __shared__ uint8_t zc_sm[8][kRowsPerCta];                 // zero point per (group, row)
-    const int kc = blockIdx.x;                 // 1024-column chunk (groups 8 kc .. 8 kc + 7)
+    __shared__ __align__(16) uint16_t sc_sm[GC][kRowsPerCta];  // fp16 scale bits per (group, row)
+    __shared__ uint8_t zc_sm[GC][kRowsPerCta];                 // zero point per (group, row)
+    const int kc = blockIdx.x;                 // 1024-column chunk (groups GC kc .. GC kc + GC - 1)
     const int row0 = blockIdx.y * kRowsPerCta;
 
     for (int i = threadIdx.x; i < 1024; i += kQuantThreads) {
@@ -81,23 +84,32 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
         const float* wrow = W + (size_t)n * K + (size_t)kc * 1024 + 4 * lane;
         float4 v[8];
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            uint4 u = ldg_stream(wrow + g * 128);
-            v[g] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
+        for (int c = 0; c < 8; ++c) {
+            uint4 u = ldg_stream(wrow + c * 128);
+            v[c] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
                                __uint_as_float(u.w));
         }
         bool bad = false;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            const float4 sv = *reinterpret_cast<const float4*>(&s_sm[g * 128 + 4 * lane]);
-            float w[4] = {__fmul_rn(v[g].x, sv.x), __fmul_rn(v[g].y, sv.y), __fmul_rn(v[g].z, sv.z),
-                          __fmul_rn(v[g].w, sv.w)};
-            float mx = w[0], mn = w[0];
+        for (int gi = 0; gi < GC; ++gi) {
+            // the group's R slices of 128: this lane's 4 scaled weights of each
+            float w[R][4];
+            float mx = 0.0f, mn = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                bad |= !isfinite(w[i]);
-                mx = fmaxf(mx, w[i]);
-                mn = fminf(mn, w[i]);
+            for (int c = 0; c < R; ++c) {
+                const int sl = gi * R + c;
+                const float4 sv = *reinterpret_cast<const float4*>(&s_sm[sl * 128 + 4 * lane]);
+                w[c][0] = __fmul_rn(v[sl].x, sv.x);
+                w[c][1] = __fmul_rn(v[sl].y, sv.y);
+                w[c][2] = __fmul_rn(v[sl].z, sv.z);
+                w[c][3] = __fmul_rn(v[sl].w, sv.w);
+                if (c == 0) mx = mn = w[0][0];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    bad |= !isfinite(w[c][i]);
+                    mx = fmaxf(mx, w[c][i]);
+                    mn = fminf(mn, w[c][i]);
+                }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -111,18 +123,21 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
             bad |= isinf(scale32) || isinf(sf);
             float zf = rintf(__fdiv_rn(-mn, sf));
             zf = fminf(fmaxf(zf, 0.0f), 15.0f);
-            float q[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float t = __fadd_rn(round_rne(__fdiv_rn(w[i], sf)), zf);
-                q[i] = fminf(fmaxf(t, 0.0f), 15.0f);
+            for (int c = 0; c < R; ++c) {
+                float q[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float t = __fadd_rn(round_rne(__fdiv_rn(w[c][i], sf)), zf);
+                    q[i] = fminf(fmaxf(t, 0.0f), 15.0f);
+                }
+                uint32_t part = place_nibbles(q, odd);
+                part |= __shfl_xor_sync(0xffffffffu, part, 1);
+                if (!odd) qweight[(size_t)n * (K >> 3) + (size_t)kc * 128 + (gi * R + c) * 16 + (lane >> 1)] = part;
             }
-            uint32_t part = place_nibbles(q, odd);
-            part |= __shfl_xor_sync(0xffffffffu, part, 1);
-            if (!odd) qweight[(size_t)n * (K >> 3) + (size_t)kc * 128 + g * 16 + (lane >> 1)] = part;
             if (lane == 0) {
-                sc_sm[g][r] = __half_as_ushort(h);
-                zc_sm[g][r] = (uint8_t)int_bits(zf);
+                sc_sm[gi][r] = __half_as_ushort(h);
+                zc_sm[gi][r] = (uint8_t)int_bits(zf);
             }
         }
         if (bad) record_error(err, kErrValue);
@@ -132,30 +147,149 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
     // group-major parameters: scales[g][n] (row pairs as one 32-bit store) and zeros[g][n/8]
     // (the nibbles of 8 consecutive rows), both coalesced along n
     {
-        const int g = threadIdx.x >> 5, j = threadIdx.x & 31;  // 8 groups x 32 row pairs
+        const int g = threadIdx.x >> 5, j = threadIdx.x & 31;  // up to 8 groups x 32 row pairs
         const int r = 2 * j;
-        if (row0 + r < N) {
+        if (g < GC && row0 + r < N) {
             const uint32_t pair = (uint32_t)sc_sm[g][r] | ((uint32_t)sc_sm[g][r + 1] << 16);
-            *reinterpret_cast<uint32_t*>(scales + ((size_t)kc * 8 + g) * N + row0 + r) = pair;
+            *reinterpret_cast<uint32_t*>(scales + ((size_t)kc * GC + g) * N + row0 + r) = pair;
         }
         if (threadIdx.x < 64) {
             const int gz = threadIdx.x >> 3, w = threadIdx.x & 7;
-            if (row0 + 8 * w < N) {
+            if (gz < GC && row0 + 8 * w < N) {
                 uint32_t word = 0;
 #pragma unroll
                 for (int b = 0; b < 8; ++b) word |= (uint32_t)(zc_sm[gz][8 * w + b] & 15u) << (4 * b);
-                zeros[((size_t)kc * 8 + gz) * (N >> 3) + (row0 >> 3) + w] = word;
+                zeros[((size_t)kc * GC + gz) * (N >> 3) + (row0 >> 3) + w] = word;
             }
         }
     }
 }
 
-cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, uint32_t* qweight,
-                                uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
+// Groups of gs = 1024 j weights (up to one group per row): a CTA takes kLargeRows rows of
+// one group.  Each warp reads a row's group twice: once for its minimum and maximum, once to
+// quantize (the second read mostly hits L2).  s for the group's columns is in shared memory.
+constexpr int kLargeRows = 32;
+
+__global__ void __launch_bounds__(kQuantThreads)
+awq_quantize_large_kernel(const float* __restrict__ W, const float* __restrict__ act, float alpha, int N, int K,
+                          int gs, uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
+                          uint32_t* __restrict__ zeros, float* __restrict__ s_out, unsigned* err) {
+    extern __shared__ __align__(16) float s_g[];  // gs scales of this group's columns
+    __shared__ __align__(16) uint16_t sc_sm[kLargeRows];
+    __shared__ uint8_t zc_sm[kLargeRows];
+    const int g = blockIdx.x;
+    const int row0 = blockIdx.y * kLargeRows;
+    const size_t c0 = (size_t)g * gs;
+
+    for (int i = threadIdx.x; i < gs; i += kQuantThreads) {
+        const float a = act[c0 + i];
+        const float p = (float)pow((double)a, (double)alpha);
+        if (!(a >= 0.0f) || isinf(a) || !isfinite(p)) record_error(err, kErrValue);
+        const float s = p > 1e-4f ? p : 1e-4f;
+        s_g[i] = s;
+        if (s_out != nullptr && blockIdx.y == 0) s_out[c0 + i] = s;
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool odd = lane & 1;
+    for (int r = warp; r < kLargeRows; r += kQuantThreads / 32) {
+        const int n = row0 + r;
+        if (n >= N) break;  // warp-uniform
+        const float* wrow = W + (size_t)n * K + c0 + 4 * lane;
+        bool bad = false;
+        float mx = 0.0f, mn = 0.0f;
+        for (int c = 0; c < gs; c += 128) {
+            const float4 u = *reinterpret_cast<const float4*>(wrow + c);
+            const float4 sv = *reinterpret_cast<const float4*>(&s_g[c + 4 * lane]);
+            const float w[4] = {__fmul_rn(u.x, sv.x), __fmul_rn(u.y, sv.y), __fmul_rn(u.z, sv.z),
+                                __fmul_rn(u.w, sv.w)};
+            if (c == 0) mx = mn = w[0];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                bad |= !isfinite(w[i]);
+                mx = fmaxf(mx, w[i]);
+                mn = fminf(mn, w[i]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        }
+        float scale32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+        if (scale32 < 1e-5f) scale32 = 1e-5f;
+        const __half h = __float2half_rn(scale32);
+        const float sf = __half2float(h);
+        bad |= isinf(scale32) || isinf(sf);
+        float zf = rintf(__fdiv_rn(-mn, sf));
+        zf = fminf(fmaxf(zf, 0.0f), 15.0f);
+        for (int c = 0; c < gs; c += 128) {
+            const float4 u = *reinterpret_cast<const float4*>(wrow + c);
+            const float4 sv = *reinterpret_cast<const float4*>(&s_g[c + 4 * lane]);
+            const float w[4] = {__fmul_rn(u.x, sv.x), __fmul_rn(u.y, sv.y), __fmul_rn(u.z, sv.z),
+                                __fmul_rn(u.w, sv.w)};
+            float q[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float t = __fadd_rn(round_rne(__fdiv_rn(w[i], sf)), zf);
+                q[i] = fminf(fmaxf(t, 0.0f), 15.0f);
+            }
+            uint32_t part = place_nibbles(q, odd);
+            part |= __shfl_xor_sync(0xffffffffu, part, 1);
+            if (!odd) qweight[(size_t)n * (K >> 3) + ((c0 + c) >> 3) + (lane >> 1)] = part;
+        }
+        if (lane == 0) {
+            sc_sm[r] = __half_as_ushort(h);
+            zc_sm[r] = (uint8_t)int_bits(zf);
+        }
+        if (bad) record_error(err, kErrValue);
+    }
+    __syncthreads();
+    if (threadIdx.x < kLargeRows / 2) {
+        const int r = 2 * threadIdx.x;
+        if (row0 + r < N) {
+            const uint32_t pair = (uint32_t)sc_sm[r] | ((uint32_t)sc_sm[r + 1] << 16);
+            *reinterpret_cast<uint32_t*>(scales + (size_t)g * N + row0 + r) = pair;
+        }
+    }
+    if (threadIdx.x < kLargeRows / 8) {
+        const int w = threadIdx.x;
+        if (row0 + 8 * w < N) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) word |= (uint32_t)(zc_sm[8 * w + b] & 15u) << (4 * b);
+            zeros[(size_t)g * (N >> 3) + (row0 >> 3) + w] = word;
+        }
+    }
+}
+
+bool quantize_group_size_ok(int K, int gs) {
+    if (gs == 128 || gs == 256 || gs == 512 || gs == 1024) return K % 1024 == 0;
+    return gs > 1024 && gs % 1024 == 0 && gs <= kQuantMaxLargeGroup && K % gs == 0;
+}
+
+cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, int gs,
+                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
                                 cudaStream_t stream) {
+    if (!quantize_group_size_ok(K, gs)) return cudaErrorInvalidValue;
+    if (gs > 1024) {
+        const int smem = gs * 4;
+        cudaError_t e = cudaFuncSetAttribute(awq_quantize_large_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             smem);
+        if (e != cudaSuccess) return e;
+        dim3 grid(K / gs, (N + kLargeRows - 1) / kLargeRows);
+        awq_quantize_large_kernel<<<grid, kQuantThreads, smem, stream>>>(W, act, alpha, N, K, gs, qweight, scales,
+                                                                         zeros, s_out, err);
+        return cudaGetLastError();
+    }
     dim3 grid(K / 1024, (N + kRowsPerCta - 1) / kRowsPerCta);
-    awq_quantize_kernel<<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out,
-                                                            err);
+    switch (gs) {
+        case 128: awq_quantize_kernel<1><<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err); break;
+        case 256: awq_quantize_kernel<2><<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err); break;
+        case 512: awq_quantize_kernel<4><<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err); break;
+        default: awq_quantize_kernel<8><<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err); break;
+    }
     return cudaGetLastError();
 }
 
