@@ -459,6 +459,41 @@ def run_gpu(args, world, rank, local):
                  "best_alpha": grid[best], "errors": [round(e, 6) for e in err]}
         del W, act, xc, wsa
 
+    # One group per row (group size = K) [SqueezeLLM article, section 4.1]: quantize the four
+    # layers, then the decode sweep's 16 calls on per-row parameters (own weights per call)
+    rinfo = None
+    if not args.skip_groups:
+        rq_b, rq_ms = 0.0, 0.0
+        rcalls = []
+        for W, act, N, K in quant:
+            ms1, gq = time_graph(torch, lambda: w4.awq_quantize(W, act, workloads.ALPHA, K), 5, 2)
+            del gq
+            rq_b += N * K * 4 + N * K // 2 + N * 2 + N // 8 * 4 + K * 4
+            rq_ms += ms1
+            qw, sc, z, _ = w4.awq_quantize(W, act, workloads.ALPHA, K)
+            for j, M in enumerate(GEMV_MS):
+                packed = (qw, sc, z) if j == 0 else (qw.clone(), sc.clone(), z.clone())
+                x = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+                rcalls.append((x, packed, torch.empty(M, N, dtype=torch.bfloat16, device="cuda"), K,
+                               N * K // 2 + N * 2 + N // 8 * 4 + 2 * M * K + 2 * M * N))
+        w4.check_device_status()
+
+        def rstep():
+            for x, (qw, sc, z), y, K, _ in rcalls:
+                w4.w4a16_linear_ex(x, qw, sc, z, out=y, workspace=ws, group_size=K)
+
+        ms_r, gr = time_graph(torch, rstep, 200, 5)
+        del gr
+        w4.check_device_status()
+        rb = sum(c[4] for c in rcalls)
+        rinfo = {"gemv": {"value": rb / (ms_r * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_r,
+                          "frac_of_hbm": rb / (ms_r * 1e-3) / 1e9 / pk["hbm_gbs"],
+                          "workload": "the decode sweep (4 Llama-3-8B shapes x M in {1, 4, 8, 16}) with one "
+                                      "quantization group per row, own weights per call"},
+                 "quantize": {"value": rq_b / rq_ms / 1e6, "unit": "GB/s",
+                              "workload": "awq_quantize with group size K on the four Llama-3-8B layers"}}
+        del rcalls
+
     if rank != 0:
         return
     cpu = None
@@ -487,6 +522,7 @@ def run_gpu(args, world, rank, local):
         "quantize": qinfo,
         "outlier_split": sinfo,
         "alpha_search": ainfo,
+        "per_row_groups": rinfo,
     }
     print(json.dumps(line), flush=True)
 
@@ -568,6 +604,7 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-split", action="store_true")
     ap.add_argument("--skip-search", action="store_true")
+    ap.add_argument("--skip-groups", action="store_true")
     ap.add_argument("--case", choices=["gemv", "gemm", "quantize"], help="time one kernel on one layer (ncu)")
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)
