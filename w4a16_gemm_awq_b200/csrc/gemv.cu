@@ -5,10 +5,11 @@
 //  bandwidth (section 2: weight-only quantization relieves the memory bottleneck).
 //  SqueezeLLM article, section 2.3: the fp16 sparse term is added to the dense product.]
 //
-// Design (B200).  Each packed weight byte is streamed once from HBM by a persistent grid of
-// one CTA per SM.
-//   - Work units are (128-channel row block, block of 4 quantization groups = 512 k): 32 KB
-//     of packed weights, brought in by ONE TMA copy.  A CTA's TMA copies are served nearly
+// Design (B200).  Each packed weight byte is streamed once from HBM by a grid of at most one
+// CTA per SM.
+//   - Work units are (128-channel row block, 4 slices of 128 k = 512 k): 32 KB of packed
+//     weights, brought in by ONE TMA copy.  A slice is a quantization group for g128; with
+//     larger groups, consecutive slices share their group's scale and zero point.  A CTA's TMA copies are served nearly
 //     one after another, so the bytes per copy set the streaming rate of a CTA: 8 KB copies
 //     stream at ~16 GB/s per CTA, 32 KB copies at ~40 GB/s, enough for one CTA per SM to
 //     saturate HBM.  The copy uses a 3-D view of qweight (16 words of a group, rows, groups;
@@ -694,8 +695,13 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                     if (lane == 0) old = atomic_add_acq_rel_gpu(p.counters + rb, 1u);
                     old = __shfl_sync(0xffffffffu, old, 0);
                     // the CTA that completes the row block sums its partials after the stream ends
-                    if (lane == 0 && old == (unsigned)(pl - pf) && reduce_list[0] < 15)
-                        reduce_list[1 + reduce_list[0]++] = rb;
+                    // (a stream-K CTA shares at most its first and its last row block)
+                    if (lane == 0 && old == (unsigned)(pl - pf)) {
+                        if (reduce_list[0] < 15)
+                            reduce_list[1 + reduce_list[0]++] = rb;
+                        else
+                            record_error(p.err, kErrShape);
+                    }
                 }
             }
             if (whole || gathered) {

@@ -54,10 +54,10 @@ search_ref_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, f
 // x'[m][k] = bf16(float(x[m][k]) / s[k]), IEEE division then round-to-nearest-even.
 __global__ void search_fold_kernel(const uint16_t* __restrict__ x, const float* __restrict__ s,
                                    uint16_t* __restrict__ xs, int M, int K) {
-    const int m = blockIdx.y;
+    const int m = blockIdx.y;  // the grid has exactly M rows of blocks
+    if (m >= M) return;
     for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < K; k += gridDim.x * blockDim.x)
         xs[(size_t)m * K + k] = float_to_bf16_bits(__fdiv_rn(bf16_bits_to_float(x[(size_t)m * K + k]), s[k]));
-    (void)M;
 }
 
 // acc[0] += sum (y_q - y_ref)^2, and when ref2 is given, *ref2 += sum y_ref^2 (double).
