@@ -5,7 +5,7 @@ import torch
 
 import w4a16_gemm_awq_b200 as w4
 import workloads
-from parity import Case, check_close, dev_bits, dev_csr, host_bf16_as_f64, xs_abs
+from parity import Case, check_close, dev_bf16, dev_bits, dev_csr, host_bf16_as_f64, xs_abs
 
 pytestmark = pytest.mark.gpu
 
@@ -242,3 +242,20 @@ def test_bounded_wait_times_out_and_context_survives(orc):
     check_close(y, ref, ref_abs, 0.0, depth(c.K), "after timeout", xs_abs(c.x, c.sc))
     with pytest.raises(w4.W4A16Error):
         w4.selftest_timeout(-1)
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES, ids=["stream_k", "cluster"])
+def test_gemv_maximum_k(orc, schedule):
+    """K = 2^20, the GEMV's largest K (2048 units per row block), on random packed weights:
+    every output against the oracle."""
+    K, N, M = 1 << 20, 128, 2
+    rng = np.random.default_rng(20)
+    qw = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    sc = (rng.uniform(0.002, 0.02, size=(K // 128, N)).astype(np.float16)).view(np.uint16)
+    z = rng.integers(0, 2 ** 32, size=(K // 128, N // 8), dtype=np.uint64).astype(np.uint32)
+    x = workloads.uniform_bf16(21, (M, K))
+    y = w4.w4a16_gemv_ex(dev_bf16(x), dev_bits(qw, torch.int32), dev_bits(sc, torch.int16), dev_bits(z, torch.int32),
+                         schedule=schedule)
+    w4.check_device_status()
+    ref, ref_abs = orc.linear(x, qw, sc, z, N, with_abs=True)
+    check_close(host_bf16_as_f64(y), ref, ref_abs, 0.0, depth(K), f"K=2^20 schedule={schedule}", xs_abs(x, sc))
