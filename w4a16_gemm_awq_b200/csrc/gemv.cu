@@ -22,14 +22,17 @@
 //     CTA then increments the row block's counter.  The CTA that completes the count sums
 //     the partials once its own stream has ended, writes y and resets the counter to zero.
 //     No CTA waits for another, and the workspace is all-zero again after every call.
-//   - Warps: 8 consumers, 1 TMA producer (weights), 2 helpers, 1 epilogue.  Everything
+//   - Warps: 8 consumers, 4 helpers, 1 TMA producer (weights), 1 epilogue.  Everything
 //     except the weights comes in through the helpers with ordinary loads, so the weights
-//     are the only TMA traffic.  For their 2 groups of each unit the helpers
-//       * copy the activations from global memory (L2-resident) into shared memory, already
-//         in the order of the MMA B fragments;
-//       * compute the group sums X_g of every token with tensor-core MMAs against an
+//     are the only TMA traffic.  Warp w runs on SM sub-partition w % 4: the consumers take
+//     two warps of each, the helpers (warps 8..11) one each, so the staging work is spread
+//     evenly (with two helpers it sat on two sub-partitions, measured 4-13% slower).  For
+//     its group of each unit a helper
+//       * copies the activations from global memory (L2-resident) into shared memory,
+//         already in the order of the MMA B fragments;
+//       * computes the group sums X_g of every token with tensor-core MMAs against an
 //         all-ones A operand;
-//       * decode the scales and zero points of the unit's 128 rows into fp32 pairs
+//       * decodes the scales and zero points of the unit's 128 rows into fp32 pairs
 //         (s, -(128 + z)).
 //   - Consumer warp c owns rows 32 (c % 4) .. +31 and groups 2 (c / 4), +1 of every unit
 //     (two m16 tiles x two groups).  The MMA is the legacy mma.sync m16n8k16 with swapped
@@ -73,11 +76,12 @@ constexpr int kGemvUnitGroups = 4;                              // groups of 128
 constexpr int kGemvGroupBytes = kGemvRows * 64;                 // one group of packed weights, 128 rows
 constexpr int kGemvWBytes = kGemvUnitGroups * kGemvGroupBytes;  // 32 KB per unit
 constexpr int kGemvConsumers = 8;                               // warps 0..7
-constexpr int kGemvProducer = 8;                                // warp 8
-constexpr int kGemvHelper0 = 9;                                 // warps 9, 10
-constexpr int kGemvHelpers = 2;
-constexpr int kGemvEpilogue = 11;                               // warp 11
-constexpr int kGemvThreads = 32 * 12;
+constexpr int kGemvProducer = 12;                               // warp 12
+constexpr int kGemvHelper0 = 8;                                 // warps 8..11, one per SMSP
+constexpr int kGemvHelpers = 4;
+constexpr int kGemvEpilogue = 13;                               // warp 13
+constexpr int kGemvThreads = 32 * 14;
+constexpr int kGemvHG = kGemvUnitGroups / kGemvHelpers;         // groups per helper and unit
 constexpr int kGemvStages = 4;
 constexpr int kGemvSlotFloats = kGemvRows * 16;                 // one partial tile in the workspace
 
@@ -316,7 +320,7 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
         }
     } else if (warp >= kGemvHelper0 && warp < kGemvHelper0 + kGemvHelpers) {
         // ------------------------------------------------------------------ helpers
-        // Helper h serves groups 2h, 2h+1 of every unit.  Lane (gq, t) loads the B fragments
+        // Helper h serves group h of every unit.  Lane (gq, t) loads the B fragments
         // of token tile j: x[8j + gq][k0 + 32t + 8w .. +8] for w = 0..3, and the parameters of
         // rows 4 lane .. 4 lane + 3.
         const int h = warp - kGemvHelper0;
@@ -328,19 +332,19 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
             // global loads first: they do not touch the ring and overlap the wait below.  The
             // scales and zero points do not depend on the previous kernel, so the first unit's
             // are in flight while the helper waits for it; x is loaded after the wait.
-            uint4 xv[2][NT][4];
-            uint2 scv[2];
-            uint32_t zw[2];
+            uint4 xv[kGemvHG][NT][4];
+            uint2 scv[kGemvHG];
+            uint32_t zw[kGemvHG];
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-                const int g = (gb * kGemvUnitGroups + 2 * h + gg) / p.gr;  // the quantization group
+            for (int gg = 0; gg < kGemvHG; ++gg) {
+                const int g = (gb * kGemvUnitGroups + kGemvHG * h + gg) / p.gr;  // the quantization group
                 scv[gg] = __ldg(reinterpret_cast<const uint2*>(p.scales + (size_t)g * p.N + (size_t)rb * kGemvRows) + lane);
                 zw[gg] = __ldg(p.zeros + (size_t)g * (p.N >> 3) + (size_t)rb * (kGemvRows / 8) + (lane >> 1));
             }
             if (s == 0) griddep_wait();  // x belongs to the stream order
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-                const int g = gb * kGemvUnitGroups + 2 * h + gg;
+            for (int gg = 0; gg < kGemvHG; ++gg) {
+                const int g = gb * kGemvUnitGroups + kGemvHG * h + gg;
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
                     const int m = 8 * j + gq;
@@ -358,20 +362,20 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
             float4* par = reinterpret_cast<float4*>(smem + L::kParOff + slot * L::kParBytes);
             float* sum = reinterpret_cast<float*>(smem + L::kSumOff + slot * L::kSumBytes);
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg)
+            for (int gg = 0; gg < kGemvHG; ++gg)
 #pragma unroll
                 for (int j = 0; j < NT; ++j)
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
-                        *reinterpret_cast<uint4*>(xs + (((((2 * h + gg) * NT + j) * 4 + w) * 32) + lane) * 16) =
+                        *reinterpret_cast<uint4*>(xs + (((((kGemvHG * h + gg) * NT + j) * 4 + w) * 32) + lane) * 16) =
                             xv[gg][j][w];
             // X_g of tokens 8j + 2t, 8j + 2t + 1: column sums of B against all-ones rows, in
             // 4 NT independent chains of 4 MMAs
-            float dx[2][NT][2][4];
+            float dx[kGemvHG][NT][2][4];
 #pragma unroll
             for (int w = 0; w < 4; ++w)
 #pragma unroll
-                for (int gg = 0; gg < 2; ++gg)
+                for (int gg = 0; gg < kGemvHG; ++gg)
 #pragma unroll
                     for (int j = 0; j < NT; ++j)
 #pragma unroll
@@ -383,8 +387,8 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                                 mma_16816_bf16_nv(dx[gg][j][hh], ones, B);
                         }
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-                const int gp = 2 * h + gg;  // group within the unit
+            for (int gg = 0; gg < kGemvHG; ++gg) {
+                const int gp = kGemvHG * h + gg;  // group within the unit
 #pragma unroll
                 for (int j = 0; j < NT; ++j)
                     if (gq == 0)
