@@ -181,8 +181,9 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4A16_ERR_CUDA;
     }
-    return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
-                                 a.workspace, (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status, stream));
+    return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals,
+                                 a.nnz, a.y, a.workspace, (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status,
+                                 stream));
 }
 
 int pick_bn(int64_t M) {
@@ -221,8 +222,8 @@ w4a16_status run_gemm(const LinearArgs& a, cudaStream_t stream) {
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4A16_ERR_CUDA;
     }
-    return from_cuda(launch_gemm(maps, a.group_ratio, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y, (int)a.M,
-                                 (int)a.N, (int)a.K, bn, d->num_sms, d->status, stream));
+    return from_cuda(launch_gemm(maps, a.group_ratio, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
+                                 (int)a.M, (int)a.N, (int)a.K, bn, d->num_sms, d->status, stream));
 }
 
 // ---------------------------------------------------------------------------------------

@@ -333,7 +333,8 @@ static cudaError_t launch_bn(const GemmMaps& maps, const GemmArgs& a, cudaStream
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(const GemmMaps& maps, int group_ratio, const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
+cudaError_t launch_gemm(const GemmMaps& maps, int group_ratio, const uint16_t* scales, const uint32_t* zeros,
+                        const int32_t* row_ptr,
                         const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, int M, int N,
                         int K, int bn, int /*num_sms*/, unsigned* err, cudaStream_t stream) {
     GemmArgs a{scales, zeros, row_ptr, col_idx, vals, nnz, y, M, N, K, group_ratio, err};

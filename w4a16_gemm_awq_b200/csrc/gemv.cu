@@ -9,10 +9,10 @@
 // CTA per SM.
 //   - Work units are (128-channel row block, 4 slices of 128 k = 512 k): 32 KB of packed
 //     weights, brought in by ONE TMA copy.  A slice is a quantization group for g128; with
-//     larger groups, consecutive slices share their group's scale and zero point.  A CTA's TMA copies are served nearly
-//     one after another, so the bytes per copy set the streaming rate of a CTA: 8 KB copies
-//     stream at ~16 GB/s per CTA, 32 KB copies at ~40 GB/s, enough for one CTA per SM to
-//     saturate HBM.  The copy uses a 3-D view of qweight (16 words of a group, rows, groups;
+//     larger groups, consecutive slices share their group's scale and zero point.  A CTA's
+//     TMA copies are served nearly one after another, so the bytes per copy set the
+//     streaming rate of a CTA: 8 KB copies stream at ~16 GB/s per CTA, 32 KB copies at
+//     ~40 GB/s, enough for one CTA per SM to saturate HBM.  The copy uses a 3-D view of qweight (16 words of a group, rows, groups;
 //     strides K/2 and 64 bytes), so it lands as [4 groups][128 rows][64 bytes] and the
 //     consumers' 128-bit loads of one group are free of bank conflicts.
 //   - Stream-K: CTA p takes the contiguous unit range [p*T/P, (p+1)*T/P), ordered row block
@@ -900,7 +900,8 @@ GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule) {
     return best;
 }
 
-cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
+cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
+                        const uint16_t* scales, const uint32_t* zeros,
                         const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
                         uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
                         cudaStream_t stream) {

@@ -50,7 +50,8 @@ struct GemvPlan {
 GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule);
 
 // group_ratio: the quantization group size / 128 (1 for g128; K / 128 for one group per row)
-cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x, const uint16_t* scales, const uint32_t* zeros,
+cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
+                        const uint16_t* scales, const uint32_t* zeros,
                         const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
                         uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
                         cudaStream_t stream);
@@ -77,7 +78,8 @@ struct GemmMaps {
     CUtensorMap qw;  // uint32 [N][K/8], box 16 words (one group) x 128 rows, 64-byte swizzle
 };
 
-cudaError_t launch_gemm(const GemmMaps& maps, int group_ratio, const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
+cudaError_t launch_gemm(const GemmMaps& maps, int group_ratio, const uint16_t* scales, const uint32_t* zeros,
+                        const int32_t* row_ptr,
                         const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, int M, int N,
                         int K, int bn, int num_sms, unsigned* err, cudaStream_t stream);
 

@@ -284,12 +284,11 @@ cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, i
         return cudaGetLastError();
     }
     dim3 grid(K / 1024, (N + kRowsPerCta - 1) / kRowsPerCta);
-    switch (gs) {
-        case 128: awq_quantize_kernel<1><<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err); break;
-        case 256: awq_quantize_kernel<2><<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err); break;
-        case 512: awq_quantize_kernel<4><<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err); break;
-        default: awq_quantize_kernel<8><<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err); break;
-    }
+    auto* kernel = gs == 128 ? awq_quantize_kernel<1>
+                 : gs == 256 ? awq_quantize_kernel<2>
+                 : gs == 512 ? awq_quantize_kernel<4>
+                             : awq_quantize_kernel<8>;
+    kernel<<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err);
     return cudaGetLastError();
 }
 
