@@ -31,8 +31,10 @@ def assert_same(orc, W, act, alpha, nnz, what):
 
 
 @pytest.mark.parametrize("N,K,frac", [(64, 1024, 0.01), (200, 3072, 0.0045), (37, 1000, 0.05), (1, 4096, 0.1),
-                                      (512, 128, 0.3)])
+                                      (512, 128, 0.3), (29, 1001, 0.02), (70, 250, 0.1), (3, 7, 0.5)])
 def test_split_random_bit_exact(orc, N, K, frac):
+    """K % 4 != 0 (1001, 250, 7) runs the one-column-per-lane passes; the others
+    the 128-bit passes, including K not a multiple of 128 (1000)."""
     L = workloads.make_layer(seed=N + K, K=K, N=N)
     assert_same(orc, L.W, L.act_absmean, workloads.ALPHA, int(np.floor(frac * N * K)), f"{N}x{K}")
 

@@ -53,7 +53,29 @@ __device__ __forceinline__ int digit_bins(int level) { return level == 0 ? 4096 
 
 __device__ __forceinline__ uint32_t score_bits(float w, float a) { return __float_as_uint(__fmul_rn(fabsf(w), a)); }
 
+// Calls f(k, w, a) for every element of row `row` (K entries), lanes of a warp along the row.
+// VEC: K % 4 == 0 and 16-byte aligned rows and act, so that each lane reads 4 consecutive
+// entries with one 128-bit load.
+template <bool VEC, typename F>
+__device__ __forceinline__ void for_row(const float* __restrict__ row, const float* __restrict__ act, uint32_t K,
+                                        int lane, F&& f) {
+    if (VEC) {
+        const float4* r4 = reinterpret_cast<const float4*>(row);
+        const float4* a4 = reinterpret_cast<const float4*>(act);
+        for (uint32_t q = lane; q < (K >> 2); q += 32) {
+            const float4 w = r4[q], a = __ldg(a4 + q);
+            f(4 * q, w.x, a.x);
+            f(4 * q + 1, w.y, a.y);
+            f(4 * q + 2, w.z, a.z);
+            f(4 * q + 3, w.w, a.w);
+        }
+    } else {
+        for (uint32_t k = lane; k < K; k += 32) f(k, row[k], __ldg(act + k));
+    }
+}
+
 // Histogram of digit `level` over the entries whose higher digits equal state->prefix.
+template <bool VEC>
 __global__ void __launch_bounds__(kSplitThreads)
 split_hist_kernel(const float* __restrict__ W, const float* __restrict__ act, uint32_t N, uint32_t K, int level,
                   const SplitState* __restrict__ state, unsigned* __restrict__ hist, unsigned* err) {
@@ -67,14 +89,11 @@ split_hist_kernel(const float* __restrict__ W, const float* __restrict__ act, ui
     bool bad = false;
     // one warp per row, lanes along the row (coalesced, and a_k indexed directly)
     for (uint32_t n = blockIdx.x * (kSplitThreads / 32) + warp; n < N; n += gridDim.x * (kSplitThreads / 32)) {
-        const float* row = W + (size_t)n * K;
-        for (uint32_t k = lane; k < K; k += 32) {
-            const float w = row[k];
-            const float a = act[k];
+        for_row<VEC>(W + (size_t)n * K, act, K, lane, [&](uint32_t, float w, float a) {
             if (level == 0 && (!isfinite(w) || !(a >= 0.0f) || isinf(a))) bad = true;
             const uint32_t b = score_bits(w, a);
             if ((b & hi_mask) == prefix) atomicAdd(&h[(b >> shift) & (uint32_t)(bins - 1)], 1u);
-        }
+        });
     }
     if (bad) record_error(err, kErrValue);
     __syncthreads();
@@ -135,6 +154,7 @@ split_select_kernel(unsigned* __restrict__ hist, int level, SplitState* __restri
 }
 
 // Per row: entries with score > T and with score == T (T = state->prefix after 3 levels).
+template <bool VEC>
 __global__ void __launch_bounds__(kSplitThreads)
 split_rowcount_kernel(const float* __restrict__ W, const float* __restrict__ act, uint32_t N, uint32_t K,
                       const SplitState* __restrict__ state, unsigned* __restrict__ gt, unsigned* __restrict__ ties) {
@@ -142,12 +162,11 @@ split_rowcount_kernel(const float* __restrict__ W, const float* __restrict__ act
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (uint32_t n = blockIdx.x * (kSplitThreads / 32) + warp; n < N; n += gridDim.x * (kSplitThreads / 32)) {
         unsigned g = 0, e = 0;
-        const float* row = W + (size_t)n * K;
-        for (uint32_t k = lane; k < K; k += 32) {
-            const uint32_t b = score_bits(row[k], act[k]);
+        for_row<VEC>(W + (size_t)n * K, act, K, lane, [&](uint32_t, float w, float a) {
+            const uint32_t b = score_bits(w, a);
             g += b > T;
             e += b == T;
-        }
+        });
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             g += __shfl_xor_sync(0xffffffffu, g, o);
@@ -210,8 +229,38 @@ split_scan_kernel(uint32_t N, const SplitState* __restrict__ state, const unsign
     (void)err;
 }
 
+// Exclusive prefix sum over the warp's lanes, and the warp total.
+__device__ __forceinline__ unsigned warp_excl_scan(unsigned v, int lane, unsigned* total) {
+    unsigned x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    *total = __shfl_sync(0xffffffffu, x, 31);
+    return x - v;
+}
+
+// The CSR entry of a chosen weight: column k, value fp16(w * s_k).
+__device__ __forceinline__ bool write_entry(uint32_t at, uint32_t nnz, uint32_t k, float w, float a, float alpha,
+                                            int32_t* col_idx, uint16_t* values, unsigned* err) {
+    if (at >= nnz) {  // never true (the counts are exact); never write past the arrays
+        record_error(err, kErrShape);
+        return false;
+    }
+    const float p = (float)pow((double)a, (double)alpha);
+    const float s = p > 1e-4f ? p : 1e-4f;
+    const __half hv = __float2half_rn(__fmul_rn(w, s));
+    col_idx[at] = (int32_t)k;
+    values[at] = __half_as_ushort(hv);
+    return isinf(__half2float(hv));
+}
+
 // One warp per row: columns in order, chosen = score > T or (score == T and among the
-// row's first ties_take[n] ties).  Writes the CSR entries and W_dense.
+// row's first ties_take[n] ties).  Writes the CSR entries and W_dense.  VEC: each lane takes
+// 4 consecutive columns of every 128-column chunk (ranks within the chunk by a warp scan of
+// the lanes' counts); otherwise one column per lane and 32-column chunks (ranks by ballot).
+template <bool VEC>
 __global__ void __launch_bounds__(kSplitThreads)
 split_fill_kernel(const float* __restrict__ W, const float* __restrict__ act, float alpha, uint32_t N, uint32_t K,
                   uint32_t nnz, const SplitState* __restrict__ state, const unsigned* __restrict__ ties_take,
@@ -226,33 +275,61 @@ split_fill_kernel(const float* __restrict__ W, const float* __restrict__ act, fl
         uint32_t pos = (uint32_t)row_ptr[n];
         const unsigned take = ties_take[n];
         unsigned ties_seen = 0;
-        for (uint32_t k0 = 0; k0 < K; k0 += 32) {
-            const uint32_t k = k0 + lane;
-            const bool in = k < K;
-            const float w = in ? row[k] : 0.0f;
-            const float a = in ? act[k] : 0.0f;
-            const uint32_t b = score_bits(w, a);
-            const bool tie = in && b == T;
-            const unsigned tie_mask = __ballot_sync(0xffffffffu, tie);
-            const unsigned tie_rank = ties_seen + __popc(tie_mask & ((1u << lane) - 1u));
-            const bool chosen = in && (b > T || (tie && tie_rank < take));
-            const unsigned ch_mask = __ballot_sync(0xffffffffu, chosen);
-            if (chosen) {
-                const uint32_t at = pos + __popc(ch_mask & ((1u << lane) - 1u));
-                if (at < nnz) {  // always true (the counts are exact); never write past the arrays
-                    const float p = (float)pow((double)a, (double)alpha);
-                    const float s = p > 1e-4f ? p : 1e-4f;
-                    const __half hv = __float2half_rn(__fmul_rn(w, s));
-                    if (isinf(__half2float(hv))) bad = true;
-                    col_idx[at] = (int32_t)k;
-                    values[at] = __half_as_ushort(hv);
-                } else {
-                    record_error(err, kErrShape);
+        if (VEC) {
+            for (uint32_t q0 = 0; q0 < (K >> 2); q0 += 32) {
+                const uint32_t q = q0 + lane;
+                const bool in = q < (K >> 2);
+                const float4 w4 = in ? reinterpret_cast<const float4*>(row)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 a4 = in ? __ldg(reinterpret_cast<const float4*>(act) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float w[4] = {w4.x, w4.y, w4.z, w4.w}, a[4] = {a4.x, a4.y, a4.z, a4.w};
+                bool gt[4], tie[4];
+                unsigned nt = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t b = score_bits(w[j], a[j]);
+                    gt[j] = in && b > T;
+                    tie[j] = in && b == T;
+                    nt += tie[j];
                 }
+                unsigned tie_total, ch_total;
+                unsigned tie_rank = ties_seen + warp_excl_scan(nt, lane, &tie_total);
+                bool chosen[4];
+                unsigned nc = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    chosen[j] = gt[j] || (tie[j] && tie_rank < take);
+                    tie_rank += tie[j];
+                    nc += chosen[j];
+                }
+                uint32_t at = pos + warp_excl_scan(nc, lane, &ch_total);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (chosen[j]) bad |= write_entry(at++, nnz, 4 * q + j, w[j], a[j], alpha, col_idx, values, err);
+                if (in)
+                    reinterpret_cast<float4*>(drow)[q] = make_float4(chosen[0] ? 0.f : w[0], chosen[1] ? 0.f : w[1],
+                                                                     chosen[2] ? 0.f : w[2], chosen[3] ? 0.f : w[3]);
+                pos += ch_total;
+                ties_seen += tie_total;
             }
-            if (in) drow[k] = chosen ? 0.0f : w;
-            pos += __popc(ch_mask);
-            ties_seen += __popc(tie_mask);
+        } else {
+            for (uint32_t k0 = 0; k0 < K; k0 += 32) {
+                const uint32_t k = k0 + lane;
+                const bool in = k < K;
+                const float w = in ? row[k] : 0.0f;
+                const float a = in ? act[k] : 0.0f;
+                const uint32_t b = score_bits(w, a);
+                const bool tie = in && b == T;
+                const unsigned tie_mask = __ballot_sync(0xffffffffu, tie);
+                const unsigned tie_rank = ties_seen + __popc(tie_mask & ((1u << lane) - 1u));
+                const bool chosen = in && (b > T || (tie && tie_rank < take));
+                const unsigned ch_mask = __ballot_sync(0xffffffffu, chosen);
+                if (chosen)
+                    bad |= write_entry(pos + __popc(ch_mask & ((1u << lane) - 1u)), nnz, k, w, a, alpha, col_idx,
+                                       values, err);
+                if (in) drow[k] = chosen ? 0.0f : w;
+                pos += __popc(ch_mask);
+                ties_seen += __popc(tie_mask);
+            }
         }
     }
     if (bad) record_error(err, kErrValue);
@@ -285,14 +362,26 @@ cudaError_t launch_split_outliers(const float* W, const float* act, float alpha,
     unsigned* ties = reinterpret_cast<unsigned*>(ws + 256 + kSplitBins * 4 + row_bytes);
     split_init_kernel<<<1, 1024, 0, stream>>>(state, hist, nnz);
     const int grid = 4 * num_sms;
+    auto a16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+    const bool vec = (K & 3u) == 0 && a16(W) && a16(act) && a16(W_dense);
     for (int level = 0; level < 3; ++level) {
-        split_hist_kernel<<<grid, kSplitThreads, 0, stream>>>(W, act, N, K, level, state, hist, err);
+        if (vec)
+            split_hist_kernel<true><<<grid, kSplitThreads, 0, stream>>>(W, act, N, K, level, state, hist, err);
+        else
+            split_hist_kernel<false><<<grid, kSplitThreads, 0, stream>>>(W, act, N, K, level, state, hist, err);
         split_select_kernel<<<1, 1024, 0, stream>>>(hist, level, state);
     }
-    split_rowcount_kernel<<<grid, kSplitThreads, 0, stream>>>(W, act, N, K, state, gt, ties);
+    if (vec)
+        split_rowcount_kernel<true><<<grid, kSplitThreads, 0, stream>>>(W, act, N, K, state, gt, ties);
+    else
+        split_rowcount_kernel<false><<<grid, kSplitThreads, 0, stream>>>(W, act, N, K, state, gt, ties);
     split_scan_kernel<<<1, 1024, 0, stream>>>(N, state, gt, ties, row_ptr, err);
-    split_fill_kernel<<<grid, kSplitThreads, 0, stream>>>(W, act, alpha, N, K, nnz, state, ties, row_ptr, W_dense,
-                                                         col_idx, values, err);
+    if (vec)
+        split_fill_kernel<true><<<grid, kSplitThreads, 0, stream>>>(W, act, alpha, N, K, nnz, state, ties, row_ptr,
+                                                                    W_dense, col_idx, values, err);
+    else
+        split_fill_kernel<false><<<grid, kSplitThreads, 0, stream>>>(W, act, alpha, N, K, nnz, state, ties, row_ptr,
+                                                                     W_dense, col_idx, values, err);
     return cudaGetLastError();
 }
 
