@@ -168,7 +168,7 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
 // Groups of gs = 1024 j weights (up to one group per row): a CTA takes kLargeRows rows of
 // one group.  Each warp reads a row's group twice: once for its minimum and maximum, once to
 // quantize (the second read mostly hits L2).  s for the group's columns is in shared memory.
-constexpr int kLargeRows = 32;
+constexpr int kLargeRows = 8;
 
 __global__ void __launch_bounds__(kQuantThreads)
 awq_quantize_large_kernel(const float* __restrict__ W, const float* __restrict__ act, float alpha, int N, int K,
