@@ -370,6 +370,40 @@ def run_gpu(args, world, rank, local):
     h2d = dx_all.numel() * 2
     d2h = dy_all.numel() * 2
 
+    # The same sweep on raw activations with the 1/s fold [AWQ translation, section 3.2]
+    # inside the GEMV's x load, against awq_fold_activations as a separate launch before each
+    # call (x' in a scratch buffer).  The bytes counted are the sweep's, as above.
+    finfo = None
+    if not args.skip_fold:
+        s_of = {}
+        for c in calls:
+            if c["K"] not in s_of:
+                g_ = torch.Generator(device="cuda").manual_seed(c["K"])
+                s_of[c["K"]] = torch.rand(c["K"], device="cuda", generator=g_) * 4.0 + 0.25
+        xp = [torch.empty_like(c["x"]) for c in calls]
+
+        def fused_step():
+            for c in calls:
+                qw, sc, z = c["w"]
+                w4.w4a16_gemv_folded(c["x"], s_of[c["K"]], qw, sc, z, out=c["y"], workspace=ws)
+
+        def separate_step():
+            for c, xb in zip(calls, xp):
+                qw, sc, z = c["w"]
+                w4.awq_fold_activations(c["x"], s_of[c["K"]], out=xb)
+                w4.w4a16_gemv(xb, qw, sc, z, out=c["y"], workspace=ws)
+
+        ms_f, gf = time_graph(torch, fused_step, 500, 5)
+        del gf
+        ms_s, gs_ = time_graph(torch, separate_step, 500, 5)
+        del gs_
+        w4.check_device_status()
+        finfo = {"fused": {"value": step_bytes / (ms_f * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_f},
+                 "separate": {"value": step_bytes / (ms_s * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_s},
+                 "workload": "the decode sweep on raw activations: w4a16_gemv_folded, against "
+                             "awq_fold_activations + w4a16_gemv per call"}
+        del xp
+
     # prefill GEMM on the same shapes (weights of the M = 1 copy; M = 512, 2048, 8192)
     gemm = None
     if not args.skip_gemm:
@@ -523,6 +557,7 @@ def run_gpu(args, world, rank, local):
         "outlier_split": sinfo,
         "alpha_search": ainfo,
         "per_row_groups": rinfo,
+        "fold_in_gemv": finfo,
     }
     print(json.dumps(line), flush=True)
 
@@ -605,6 +640,7 @@ def main():
     ap.add_argument("--skip-split", action="store_true")
     ap.add_argument("--skip-search", action="store_true")
     ap.add_argument("--skip-groups", action="store_true")
+    ap.add_argument("--skip-fold", action="store_true")
     ap.add_argument("--case", choices=["gemv", "gemm", "quantize"], help="time one kernel on one layer (ncu)")
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)

@@ -215,6 +215,28 @@ w4a16_status w4a16_linear_ex(const uint16_t* x, const uint32_t* qweight, const u
                              int64_t M, int64_t N, int64_t K, int64_t group_size, void* workspace,
                              size_t workspace_bytes, int schedule, void* stream);
 
+/* w4a16_gemv_folded -- the decode GEMV on the layer input BEFORE the AWQ scaling: the
+ * kernel divides x by the per-channel scale s as it loads it, so no separate pass over x
+ * is needed.  [AWQ translation, 3.2: the weights are multiplied by s and the activations
+ * divided by it; 1 (TinyChat): kernel fusion to avoid intermediate DRAM round trips and
+ * launches.]
+ *   x   [M][K] bf16 bits, device: the raw layer input.
+ *   s   [K] fp32, device, 16-byte aligned: the scales awq_quantize wrote to s_out; or NULL,
+ *       for an x that is already divided (the call is then w4a16_linear_ex's decode path).
+ *   The kernel uses x'[m][k] = bf16_rne(float(x[m][k]) / s[k]) (IEEE division), for the
+ *   quantized product and for the sparse term: the values awq_fold_activations writes, so
+ *   y is bit-identical to awq_fold_activations followed by w4a16_gemv_ex with the same
+ *   schedule.  s is read after the previous kernel on the stream has finished.
+ *   group_size, schedule: as w4a16_linear_ex.  1 <= M <= 16 (SHAPE otherwise).
+ *   Everything else is as for w4a16_gemv_ex; ALIGN also for a misaligned s.
+ * For M > 16 the tensor-core GEMM loads x with TMA, which cannot divide: run
+ * awq_fold_activations first, then w4a16_gemm. */
+w4a16_status w4a16_gemv_folded(const uint16_t* x, const float* s, const uint32_t* qweight,
+                               const uint16_t* scales, const uint32_t* zeros,
+                               const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N,
+                               int64_t K, int64_t group_size, void* workspace,
+                               size_t workspace_bytes, int schedule, void* stream);
+
 /* w4a16_gemm -- the tcgen05 tensor-core path of w4a16_linear, for any M >= 1.  Arguments
  * and result are as for w4a16_linear.  The workspace is not used (NULL and 0 are fine).
  * Weights are dequantized to bf16 inside the kernel.  When a CSR is given, its values are

@@ -137,6 +137,20 @@ def test_grouped_validation(L):
     assert lx(2048, K=5120) == w4.ERR_SHAPE            # 2048 does not divide 5120
 
 
+def test_folded_gemv_validation(L):
+    def f(s=FAKE, M=1, gs=128, schedule=0, K=4096, x=FAKE):
+        return L.w4a16_gemv_folded(ctypes.c_void_p(x), ctypes.c_void_p(s) if s else None, ctypes.c_void_p(FAKE),
+                                   ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), None, ctypes.c_void_p(FAKE), M,
+                                   128, K, gs, ctypes.c_void_p(FAKE), 1 << 30, schedule, None)
+    assert f(x=0) == w4.ERR_NULL
+    assert f(M=17) == w4.ERR_SHAPE                     # decode only
+    assert f(M=0) == w4.ERR_SHAPE
+    assert f(gs=192) == w4.ERR_SHAPE
+    assert f(gs=2048, K=5120) == w4.ERR_SHAPE
+    assert f(schedule=4) == w4.ERR_VALUE
+    assert f(s=FAKE + 4) == w4.ERR_ALIGN               # s is read 16 bytes at a time
+
+
 def test_split_validation(L):
     def sp(W=FAKE, a=FAKE, alpha=0.5, N=16, K=256, nnz=10, Wd=FAKE, rp=FAKE, ci=FAKE, v=FAKE, ws=FAKE, wsb=1 << 30):
         return L.awq_split_outliers(ctypes.c_void_p(W), ctypes.c_void_p(a), ctypes.c_float(alpha), N, K, nnz,

@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             fn.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P, ctypes.c_size_t, P]
         L.w4a16_gemv_ex.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P, ctypes.c_size_t,
                                     ctypes.c_int, P]
+        L.w4a16_gemv_folded.argtypes = [P, P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, I64, P,
+                                        ctypes.c_size_t, ctypes.c_int, P]
         PI = ctypes.POINTER(ctypes.c_int)
         L.w4a16_gemv_plan.argtypes = [I64, I64, I64, ctypes.c_int, PI, PI, PI]
         L.w4a16_workspace_bytes.argtypes = [I64, I64, I64]
@@ -177,8 +179,11 @@ def workspace_bytes(M: int, N: int, K: int) -> int:
     return int(lib().w4a16_workspace_bytes(M, N, K))
 
 
-def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, schedule=None, group_size=None):
+def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, schedule=None, group_size=None,
+            fold=False, s=None):
     _need(x, torch.bfloat16, 2, "x")
+    if s is not None:
+        _need(s, torch.float32, 1, "s")
     _need(qweight, torch.int32, 2, "qweight")
     _need(scales, torch.int16, 2, "scales")
     _need(zeros, torch.int32, 2, "zeros")
@@ -186,6 +191,8 @@ def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, s
     N = qweight.shape[0]
     if qweight.shape[1] * 8 != K:
         raise ValueError(f"qweight {tuple(qweight.shape)} does not match K = {K}")
+    if s is not None and s.numel() != K:
+        raise ValueError(f"s has {s.numel()} entries, K = {K}")
     y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
     cs = None
     if csr is not None:
@@ -196,8 +203,8 @@ def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, s
     need = workspace_bytes(M, N, K) if name != "w4a16_gemm" else 0
     if ws is None and need > 0:
         ws = workspace(x.device, need)
-    args = [_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), ctypes.byref(cs) if cs is not None else None,
-            _ptr(y), M, N, K]
+    args = [_ptr(x)] + ([_ptr(s)] if fold else []) + [
+        _ptr(qweight), _ptr(scales), _ptr(zeros), ctypes.byref(cs) if cs is not None else None, _ptr(y), M, N, K]
     if group_size is not None:
         args.append(int(group_size))
     args += [_ptr(ws), ws.numel() if ws is not None else 0]
@@ -225,6 +232,14 @@ def w4a16_linear_ex(x, qweight, scales, zeros, csr=None, out=None, workspace=Non
                     schedule=GEMV_AUTO):
     """w4a16_linear for weights quantized in groups of group_size along K."""
     return _linear("w4a16_linear_ex", x, qweight, scales, zeros, csr, out, workspace, schedule, group_size)
+
+
+def w4a16_gemv_folded(x, s, qweight, scales, zeros, csr=None, out=None, workspace=None, group_size=128,
+                      schedule=GEMV_AUTO):
+    """The decode GEMV on the raw layer input: x is divided by the channel scales s (fp32 [K],
+    or None for an already divided x) inside the kernel, as awq_fold_activations would."""
+    return _linear("w4a16_gemv_folded", x, qweight, scales, zeros, csr, out, workspace, schedule, group_size,
+                   fold=True, s=s)
 
 
 def gemv_plan(M: int, N: int, K: int, schedule: int = GEMV_AUTO):

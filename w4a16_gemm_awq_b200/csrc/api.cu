@@ -107,6 +107,7 @@ inline w4a16_status from_cuda(cudaError_t e) { return e == cudaSuccess ? W4A16_O
 
 struct LinearArgs {
     const uint16_t* x;
+    const float* s = nullptr;  // the decode GEMV divides x by s as it loads it
     const uint32_t* qweight;
     const uint16_t* scales;
     const uint32_t* zeros;
@@ -129,7 +130,7 @@ w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const u
         return W4A16_ERR_SHAPE;
     if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(zeros, 16) || !aligned(y, 16))
         return W4A16_ERR_ALIGN;
-    *a = LinearArgs{x, qweight, scales, zeros};
+    *a = LinearArgs{x, nullptr, qweight, scales, zeros};
     a->y = y;
     a->M = M;
     a->N = N;
@@ -181,7 +182,7 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4A16_ERR_CUDA;
     }
-    return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals,
+    return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.s, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals,
                                  a.nnz, a.y, a.workspace, (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status,
                                  stream));
 }
@@ -308,6 +309,24 @@ w4a16_status w4a16_gemv_ex(const uint16_t* x, const uint32_t* qweight, const uin
     if (st != W4A16_OK) return st;
     if (M > 16) return W4A16_ERR_SHAPE;
     if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);
+}
+
+w4a16_status w4a16_gemv_folded(const uint16_t* x, const float* s, const uint32_t* qweight, const uint16_t* scales,
+                               const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N,
+                               int64_t K, int64_t group_size, void* workspace, size_t workspace_bytes, int schedule,
+                               void* stream) {
+    LinearArgs a;
+    w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
+    if (st != W4A16_OK) return st;
+    if (M > 16) return W4A16_ERR_SHAPE;
+    if (group_size < 128 || group_size % 128 != 0 || group_size > K || K % group_size != 0) return W4A16_ERR_SHAPE;
+    if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
+    if (s != nullptr && !aligned(s, 16)) return W4A16_ERR_ALIGN;
+    a.s = s;
+    a.group_ratio = (int)(group_size / 128);
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
     return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);

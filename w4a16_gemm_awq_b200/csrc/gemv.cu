@@ -87,6 +87,7 @@ constexpr int kGemvSlotFloats = kGemvRows * 16;                 // one partial t
 
 struct GemvArgs {
     const uint16_t* x;
+    const float* s;      // nullptr, or the AWQ channel scales: the kernel uses x' = bf16(x / s)
     const uint16_t* scales;
     const uint32_t* zeros;
     const int32_t* row_ptr;
@@ -150,6 +151,21 @@ __device__ __forceinline__ uint32_t unit_begin(uint32_t p, uint32_t T, uint32_t 
 // The CTA whose unit range contains unit u: the largest p with floor(p*T/P) <= u.
 __device__ __forceinline__ int cta_of_unit(uint32_t u, uint32_t T, uint32_t P) { return (int)(((u + 1) * P - 1) / T); }
 
+// x' = bf16_rne(float(x) / s) with IEEE division: one bf16 value, and the 8 of a 16-byte load
+// (element e in half e % 2 of word e / 2) against the scales of their 8 channels.
+__device__ __forceinline__ uint16_t fold_bf16(uint16_t x, float s) {
+    return float_to_bf16_bits(__fdiv_rn(bf16_bits_to_float(x), s));
+}
+
+__device__ __forceinline__ uint32_t fold_bf16x2(uint32_t v, float s_lo, float s_hi) {
+    return (uint32_t)fold_bf16((uint16_t)(v & 0xFFFFu), s_lo) | ((uint32_t)fold_bf16((uint16_t)(v >> 16), s_hi) << 16);
+}
+
+__device__ __forceinline__ uint4 fold_bf16x8(uint4 v, float4 s0, float4 s1) {
+    return make_uint4(fold_bf16x2(v.x, s0.x, s0.y), fold_bf16x2(v.y, s0.z, s0.w), fold_bf16x2(v.z, s1.x, s1.y),
+                      fold_bf16x2(v.w, s1.z, s1.w));
+}
+
 // y[m][n] for every token m of channel row n: v[m] + the CSR term of row n, rounded once.
 __device__ __forceinline__ void write_row(const GemvArgs& p, int n, float v[16]) {
     if (p.row_ptr != nullptr) {
@@ -164,9 +180,15 @@ __device__ __forceinline__ void write_row(const GemvArgs& p, int n, float v[16])
                     continue;
                 }
                 const float val = fp16_bits_to_float(p.vals[j]);
+                const float sc = p.s != nullptr ? p.s[c] : 1.0f;
 #pragma unroll
                 for (int m = 0; m < 16; ++m)
-                    if (m < p.M) v[m] = fmaf(val, bf16_bits_to_float(p.x[(size_t)m * p.K + c]), v[m]);
+                    if (m < p.M) {
+                        const uint16_t xb = p.x[(size_t)m * p.K + c];
+                        const float xm = p.s != nullptr ? bf16_bits_to_float(fold_bf16(xb, sc))
+                                                        : bf16_bits_to_float(xb);
+                        v[m] = fmaf(val, xm, v[m]);
+                    }
             }
         }
     }
@@ -352,6 +374,21 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                     for (int w = 0; w < 4; ++w)
                         xv[gg][j][w] = m < p.M ? ldg_cached(p.x + (size_t)m * p.K + ((size_t)g << 7) + 32 * t + 8 * w)
                                                : make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            if (p.s != nullptr) {
+                // the 1/s fold on the way in: the same conversions as awq_fold_activations
+#pragma unroll
+                for (int gg = 0; gg < kGemvHG; ++gg) {
+                    const float* sg = p.s + ((size_t)(gb * kGemvUnitGroups + kGemvHG * h + gg) << 7) + 32 * t;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const float4 s0 = __ldg(reinterpret_cast<const float4*>(sg + 8 * w));
+                        const float4 s1 = __ldg(reinterpret_cast<const float4*>(sg + 8 * w) + 1);
+#pragma unroll
+                        for (int j = 0; j < NT; ++j)
+                            if (8 * j + gq < p.M) xv[gg][j][w] = fold_bf16x8(xv[gg][j][w], s0, s1);
+                    }
                 }
             }
             if (s >= S && !__all_sync(0xffffffffu, mbar_wait_bounded(&xempty[slot], ((s / S) - 1) & 1))) {
@@ -901,12 +938,13 @@ GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule) {
 }
 
 cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
-                        const uint16_t* scales, const uint32_t* zeros,
+                        const float* s, const uint16_t* scales, const uint32_t* zeros,
                         const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
                         uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
                         cudaStream_t stream) {
     GemvArgs a{};
     a.x = x;
+    a.s = s;
     a.scales = scales;
     a.zeros = zeros;
     a.row_ptr = row_ptr;

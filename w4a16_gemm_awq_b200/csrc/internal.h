@@ -49,9 +49,10 @@ struct GemvPlan {
 // The launch for a schedule (W4A16_GEMV_AUTO, _STREAM_K or _CLUSTER) on the current device.
 GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule);
 
-// group_ratio: the quantization group size / 128 (1 for g128; K / 128 for one group per row)
+// group_ratio: the quantization group size / 128 (1 for g128; K / 128 for one group per row).
+// s: nullptr, or [K] channel scales that the kernel divides x by as it loads it.
 cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
-                        const uint16_t* scales, const uint32_t* zeros,
+                        const float* s, const uint16_t* scales, const uint32_t* zeros,
                         const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
                         uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
                         cudaStream_t stream);
