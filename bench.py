@@ -36,8 +36,8 @@ METRIC = "W4A16 GEMV achieved GB/s (% HBM peak); GEMM TFLOPS (% bf16 TC peak)"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DATA = "synthetic: seeded N(0, 0.02^2) weights, lognormal-channel activations (no checkpoints)"
 GEMV_SHAPES = workloads.LLAMA3_8B
-GEMV_MS = workloads.CONFIGS[1]["Ms"]
-GEMM_MS = workloads.CONFIGS[2]["Ms"]
+GEMV_MS = workloads.DECODE_SWEEP["Ms"]
+GEMM_MS = workloads.PREFILL_SWEEP["Ms"]
 WORKLOAD = ("decode GEMV sweep, Llama-3-8B linear shapes (K x N = 4096x6144, 4096x4096, 4096x28672, "
             "14336x4096) x M in {1, 4, 8, 16}, W4 g128 (alpha 0.5)")
 
@@ -442,13 +442,13 @@ def run_gpu(args, world, rank, local):
         qinfo = {"value": qb / qms / 1e6, "unit": "GB/s", "workload": "awq_quantize_g128 on the four Llama-3-8B "
                  "layers (218 M fp32 weights)", "frac_of_hbm": qb / qms / 1e6 / pk["hbm_gbs"]}
 
-    # GPU dense-and-sparse split on the config-3 layers (Llama-2-13B shapes, 0.45% outliers);
+    # GPU dense-and-sparse split on the Llama-2-13B layers (0.45% outliers);
     # algorithmic bytes: read W and a, write W_dense and the CSR
     sinfo = None
     if not args.skip_split:
         sb, sms_ = 0.0, 0.0
         per_split = []
-        for si, (name, K, N) in enumerate(workloads.CONFIGS[3]["shapes"]):
+        for si, (name, K, N) in enumerate(workloads.DENSE_SPARSE_13B["shapes"]):
             L = workloads.make_layer(workloads.seed_of(3, si), K=K, N=N)
             W = torch.from_numpy(L.W).cuda()
             act = torch.from_numpy(L.act_absmean).cuda()

@@ -1,7 +1,7 @@
 """Shared helpers of the GPU parity tests: moving seeded host inputs to the device, and the
 comparison of a bf16 GPU result with the oracle's double-precision result.
 
-Tolerance (spec criterion): max_i |y_i - r_i| / max_i |r_i| <= 1e-2 per output row of
+Tolerance (the output criterion): max_i |y_i - r_i| / max_i |r_i| <= 1e-2 per output row of
 tokens.  The tests also check a per-element bound derived from the arithmetic:
   |y - r| <= 2^-8 |r|                       (one bf16 rounding of the output, with slack)
            + c_w * sum_k |x_k w_k|           (c_w: relative error of the weights fed to the MMA;
@@ -15,7 +15,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-NORTH_STAR_REL = 1e-2
+Y_REL_TOL = 1e-2
 
 
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:
@@ -76,7 +76,7 @@ def check_close(y: np.ndarray, ref: np.ndarray, ref_abs: np.ndarray, c_w: float,
         rel = err.max(axis=1) / np.maximum(np.abs(ref).max(axis=1), 1e-30)
     else:
         rel = np.array([err.max() / max(np.abs(ref).max(), 1e-30)])
-    assert rel.max() <= NORTH_STAR_REL, f"{what}: max relative error {rel.max():.3e} > {NORTH_STAR_REL}"
+    assert rel.max() <= Y_REL_TOL, f"{what}: max relative error {rel.max():.3e} > {Y_REL_TOL}"
     bound = 2.0 ** -8 * np.abs(ref) + (c_w + depth * 2.0 ** -22) * ref_abs + 1e-30
     if xsabs is not None:
         bound = bound + GEMV_XS_COEF * xsabs

@@ -201,12 +201,12 @@ def test_linear_dispatches_to_gemv(orc):
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-def test_gemv_config0_full(orc):
+def test_gemv_single_layer_full(orc):
     """4096 x 4096, M = 1, alpha = 0.5: the whole output against the oracle."""
     c = Case(orc, seed=workloads.seed_of(0, 0), K=4096, N=4096, M=1)
     y = host_bf16_as_f64(gemv(c.device()))
     ref, ref_abs = c.reference(orc)
-    check_close(y, ref, ref_abs, 0.0, depth(c.K), "config 0", xs_abs(c.x, c.sc))
+    check_close(y, ref, ref_abs, 0.0, depth(c.K), "4096x4096 M=1", xs_abs(c.x, c.sc))
 
 
 FULL = ([(1, i, K, N, M, False) for i, (_, K, N) in enumerate(workloads.LLAMA3_8B) for M in (1, 4, 8, 16)]

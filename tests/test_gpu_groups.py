@@ -1,6 +1,6 @@
 """Group sizes other than 128 (up to one group per row) on the GPU, against the oracle:
 quantize bit for bit, the decode GEMV (both schedules) and the tcgen05 GEMM within the
-spec tolerance.  [SqueezeLLM article, section 4.1: the group size option.]"""
+output tolerance.  [SqueezeLLM article, section 4.1: the group size option.]"""
 import numpy as np
 import pytest
 import torch

@@ -76,7 +76,8 @@ def test_quantize_reports_bad_values():
     w4.check_device_status()  # cleared
 
 
-ALL_SHAPES = [(cfg, i, K, N) for cfg in (1, 4) for i, (_, K, N) in enumerate(workloads.CONFIGS[cfg]["shapes"])]
+ALL_SHAPES = [(w["family"], i, K, N) for w in (workloads.DECODE_SWEEP, workloads.LARGE_LAYERS_70B)
+              for i, (_, K, N) in enumerate(w["shapes"])]
 
 
 @pytest.mark.parametrize("cfg,i,K,N", ALL_SHAPES, ids=[f"c{c}_{K}x{N}" for c, _, K, N in ALL_SHAPES])

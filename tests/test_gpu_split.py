@@ -81,7 +81,7 @@ def test_split_errors():
     w4.check_device_status()
 
 
-SPLIT_SHAPES = [(i, K, N) for i, (_, K, N) in enumerate(workloads.CONFIGS[3]["shapes"])]
+SPLIT_SHAPES = [(i, K, N) for i, (_, K, N) in enumerate(workloads.DENSE_SPARSE_13B["shapes"])]
 
 
 @pytest.mark.parametrize("i,K,N", SPLIT_SHAPES, ids=[f"{K}x{N}" for _, K, N in SPLIT_SHAPES])

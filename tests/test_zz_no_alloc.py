@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import w4a16_gemm_awq_b200 as w4
-from parity import NORTH_STAR_REL, Case, host_bf16_as_f64
+from parity import Y_REL_TOL, Case, host_bf16_as_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -43,7 +43,7 @@ def test_gemv_noalloc_matches_gemv_twice(orc, K, N, M, csr):
         got = host_bf16_as_f64(y)
         assert np.all(np.isfinite(got))
         err = np.abs(got - want).max(axis=1) / np.abs(want).max(axis=1)
-        assert err.max() <= NORTH_STAR_REL, err.max()
+        assert err.max() <= Y_REL_TOL, err.max()
 
 
 def test_gemv_noalloc_rejects_oversize(orc):

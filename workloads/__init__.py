@@ -33,15 +33,17 @@ LLAMA2_13B = [("attn_5120x5120", 5120, 5120), ("mlp_5120x13824", 5120, 13824)]
 LLAMA2_70B = [("qkv_proj", 8192, 10240), ("o_proj", 8192, 8192), ("gate_up_proj", 8192, 57344),
               ("down_proj", 28672, 8192)]
 
-# Workload configurations (M = tokens).
-CONFIGS = {
-    0: dict(name="single layer 4096x4096, M=1", shapes=[("layer", 4096, 4096)], Ms=[1], csr=False),
-    1: dict(name="decode GEMV sweep, Llama-3-8B shapes", shapes=LLAMA3_8B, Ms=[1, 4, 8, 16], csr=False),
-    2: dict(name="prefill GEMM, Llama-3-8B shapes", shapes=LLAMA3_8B, Ms=[512, 2048, 8192], csr=False),
-    3: dict(name="dense-and-sparse, 13B shapes, 0.45% fp16 CSR", shapes=LLAMA2_13B, Ms=[1, 16, 1024],
-            csr=True),
-    4: dict(name="large layers, 70B shapes", shapes=LLAMA2_70B, Ms=[1, 64, 4096], csr=False),
-}
+# Workloads (M = tokens).  `family` numbers the seeds of a workload's layers (seed_of).
+SINGLE_LAYER = dict(family=0, name="single layer 4096x4096, M=1", shapes=[("layer", 4096, 4096)], Ms=[1],
+                    csr=False)
+DECODE_SWEEP = dict(family=1, name="decode GEMV sweep, Llama-3-8B shapes", shapes=LLAMA3_8B, Ms=[1, 4, 8, 16],
+                    csr=False)
+PREFILL_SWEEP = dict(family=2, name="prefill GEMM, Llama-3-8B shapes", shapes=LLAMA3_8B, Ms=[512, 2048, 8192],
+                     csr=False)
+DENSE_SPARSE_13B = dict(family=3, name="dense-and-sparse, 13B shapes, 0.45% fp16 CSR", shapes=LLAMA2_13B,
+                        Ms=[1, 16, 1024], csr=True)
+LARGE_LAYERS_70B = dict(family=4, name="large layers, 70B shapes", shapes=LLAMA2_70B, Ms=[1, 64, 4096], csr=False)
+WORKLOADS = (SINGLE_LAYER, DECODE_SWEEP, PREFILL_SWEEP, DENSE_SPARSE_13B, LARGE_LAYERS_70B)
 ALPHA = 0.5
 OUTLIER_FRACTION = 0.0045
 N_OUTLIER_CHANNELS = 8
@@ -49,8 +51,8 @@ OUTLIER_CHANNEL_GAIN = 20.0
 CALIB_ROWS = 512
 
 
-def seed_of(config: int, shape_index: int) -> int:
-    return 1000 * config + shape_index
+def seed_of(family: int, shape_index: int) -> int:
+    return 1000 * family + shape_index
 
 
 def _streams(seed: int):
