@@ -12,9 +12,10 @@
 //     larger groups, consecutive slices share their group's scale and zero point.  A CTA's
 //     TMA copies are served nearly one after another, so the bytes per copy set the
 //     streaming rate of a CTA: 8 KB copies stream at ~16 GB/s per CTA, 32 KB copies at
-//     ~40 GB/s, enough for one CTA per SM to saturate HBM.  The copy uses a 3-D view of qweight (16 words of a group, rows, groups;
-//     strides K/2 and 64 bytes), so it lands as [4 groups][128 rows][64 bytes] and the
-//     consumers' 128-bit loads of one group are free of bank conflicts.
+//     ~40 GB/s, enough for one CTA per SM to saturate HBM.  The copy uses a 3-D view of
+//     qweight (16 words of a group, rows, groups; strides K/2 and 64 bytes), so it lands as
+//     [4 groups][128 rows][64 bytes] and the consumers' 128-bit loads of one group are free
+//     of bank conflicts.
 //   - Stream-K: CTA p takes the contiguous unit range [p*T/P, (p+1)*T/P), ordered row block
 //     by row block, so every CTA streams the same number of bytes in one balanced wave.  A
 //     row block processed whole by one CTA is written straight to y.  A row block split
@@ -63,6 +64,10 @@
 //   - Programmatic dependent launch.  The weights may be fetched before the previous kernel
 //     on the stream has finished.  The helpers wait for it before they load x; the
 //     epilogue and the completion phase wait before they touch the workspace or y.
+//   - Optional 1/s fold [AWQ translation, section 3.2: the activations are divided by the
+//     channel scales s].  Given s, the helpers turn every x they load into
+//     x' = bf16(x / s) (IEEE division) before staging it, and the CSR term does the same,
+//     so the result is bit-identical to folding x in a separate pass first.
 #include <atomic>
 #include <mutex>
 
