@@ -535,7 +535,7 @@ def run_gpu(args, world, rank, local):
         v, secs, outs, desc = oracle_sample(args.cpu_budget)
         cpu = {"value": v, "unit": "GB/s", "cores": omp_threads(), "kind": "oracle", "sample": desc,
                "seconds": round(secs, 2)}
-    traffic = profile_traffic()
+    traffic, traffic_note = profile_traffic()
     per_gpu_gbs = step_bytes / (ms_local * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -546,7 +546,8 @@ def run_gpu(args, world, rank, local):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": per_gpu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": per_gpu_gbs / pk["hbm_gbs"], "traffic": traffic, "peak_kind": f"{pk_kind} HBM copy",
-                     "kernel": "gemv_w4a16_kernel", "bytes_per_launch": step_bytes / len(calls)},
+                     "kernel": "gemv_w4a16_kernel", "bytes_per_launch": step_bytes / len(calls),
+                     **({"traffic_note": traffic_note} if traffic_note else {})},
         "cpu_baseline": cpu,
         "e2e": {"value": step_bytes * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
@@ -562,19 +563,51 @@ def run_gpu(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+GEMV_SOURCE = os.path.join(ROOT, "w4a16_gemm_awq_b200", "csrc", "gemv.cu")
+GEMV_PROFILE = os.path.join(ROOT, "profiles", "gemv_w4a16_llama3_8b_decode.md")
+
+
+def code_digest_text(text: str) -> str:
+    """16 hex digits of the sha256 of C/CUDA source text without its comments and whitespace:
+    it changes with the code, not with comments or formatting."""
+    import hashlib
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return hashlib.sha256(re.sub(r"\s+", "", text).encode()).hexdigest()[:16]
+
+
+def code_digest(path: str) -> str:
+    with open(path) as f:
+        return code_digest_text(f.read())
+
+
+def traffic_from_summary(lines, current_digest: str):
+    """(DRAM bytes per GEMV launch, note) from the lines of an ncu summary:
+    'traffic_bytes_per_launch: <int>' and 'kernel_code_digest: <hex>'.  The bytes are
+    returned only while the digest matches the kernel code as it is now; counters taken on
+    other code give (None, why)."""
+    fields = {}
+    for line in lines:
+        if ":" in line and line.split(":", 1)[0] in ("traffic_bytes_per_launch", "kernel_code_digest"):
+            k, v = line.split(":", 1)
+            fields[k] = v.strip()
+    try:
+        traffic = int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None, "no traffic line in the ncu summary"
+    if fields.get("kernel_code_digest") != current_digest:
+        return None, (f"the ncu counters ({traffic} B per launch) were taken on other kernel code "
+                      f"(digest {fields.get('kernel_code_digest')}, now {current_digest})")
+    return traffic, None
+
+
 def profile_traffic():
-    """DRAM bytes per GEMV launch from the committed ncu summary, if one exists for the
-    current kernel (a line 'traffic_bytes_per_launch: <int>'); else None."""
-    path = os.path.join(ROOT, "profiles", "gemv_w4a16_llama3_8b_decode.md")
-    if not os.path.exists(path):
-        return None
-    for line in open(path):
-        if line.startswith("traffic_bytes_per_launch:"):
-            try:
-                return int(line.split(":", 1)[1].strip())
-            except ValueError:
-                return None
-    return None
+    """traffic_from_summary for the committed GEMV summary and the current gemv.cu."""
+    if not os.path.exists(GEMV_PROFILE):
+        return None, "no ncu summary"
+    with open(GEMV_PROFILE) as f:
+        return traffic_from_summary(f.readlines(), code_digest(GEMV_SOURCE))
 
 
 def run_case(args):
