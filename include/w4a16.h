@@ -27,8 +27,8 @@
  *   - Element types are passed as raw bits: bf16 and fp16 as uint16_t, fp32 as float.
  *   - Shapes: W is [N][K] (out x in), x is [M][K], y is [M][N], all row-major and dense.
  *     K must be a positive multiple of 1024 and N a positive multiple of 128 (the quantizer
- *     accepts any positive multiple of 8, so zero points fill whole words).  Every pointer must be 16-byte aligned, except the
- *     CSR arrays, which need only natural alignment.
+ *     accepts any positive multiple of 8, so zero points fill whole words).  Every pointer
+ *     must be 16-byte aligned, except the CSR arrays, which need only natural alignment.
  *
  * Packed weight format (shared with any reader of the quantized weights):
  *   qweight[n][k/8]  uint32.  Nibble j (bits 4j..4j+3) holds the code of element
