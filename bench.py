@@ -47,6 +47,14 @@ def gemv_bytes(N: int, K: int, M: int) -> int:
     return workloads.packed_bytes(N, K) + 2 * M * K + 2 * M * N
 
 
+def sweep_config(world: int) -> dict:
+    """The workload's `config`, the same for both arms."""
+    step_bytes = sum(gemv_bytes(N, K, M) for _, K, N in GEMV_SHAPES for M in GEMV_MS)
+    return {"workload": WORKLOAD, "M": GEMV_MS, "step": "16 GEMV calls (4 shapes x 4 M), one CUDA graph",
+            "l2": "inputs larger than L2: one packed-weight copy per call, %.0f MB per step" % (step_bytes / 1e6),
+            "parallelism": f"replicas x{world}"}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -235,7 +243,8 @@ def run_reference(args, world, rank):
     line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_tot / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
-            "config": {"workload": WORKLOAD, "sample": f"{P} sampled outputs per step, one layer/M per step"},
+            "config": sweep_config(world),
+            "sample": f"each step: {P} sampled outputs of one (layer, M) of the sweep, computed by the oracle",
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": omp_threads(), "kind": "oracle",
                              "sample": f"{P} sampled GEMV outputs per step over {args.steps} steps"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -541,9 +550,7 @@ def run_gpu(args, world, rank, local):
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": DATA,
-        "config": {"workload": WORKLOAD, "M": GEMV_MS, "step": "16 GEMV calls (4 shapes x 4 M), one CUDA graph",
-                   "l2": "inputs larger than L2: one packed-weight copy per call, %.0f MB per step" % (step_bytes / 1e6),
-                   "parallelism": f"replicas x{world}"},
+        "config": sweep_config(world),
         "roofline": {"bound": "hbm", "achieved": per_gpu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": per_gpu_gbs / pk["hbm_gbs"], "traffic": traffic, "peak_kind": f"{pk_kind} HBM copy",
                      "kernel": "gemv_w4a16_kernel", "bytes_per_launch": step_bytes / len(calls),
