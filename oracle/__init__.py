@@ -74,6 +74,13 @@ def _L():
                                     ctypes.c_int),
             "oracle_split_outliers": ([P, P, F, I64, I64, I64, P, P, P, P], ctypes.c_int),
             "oracle_awq_search_alpha": ([P, P, P, I64, I64, I64, P, I64, P], ctypes.c_int),
+            "oracle_pack32x3": ([P, P], ctypes.c_int),
+            "oracle_unpack32x3": ([P, P], None),
+            "oracle_awq_quantize3_gs": ([P, P, F, I64, I64, I64, P, P, P, P], ctypes.c_int),
+            "oracle_dequant3_gs": ([P, P, P, I64, I64, I64, P], ctypes.c_int),
+            "oracle_linear3_gs": ([P, I64, I64, I64, P, P, P, I64, P, P, P, I64, P, P], ctypes.c_int),
+            "oracle_linear3_at_gs": ([P, I64, I64, I64, P, P, P, I64, P, P, P, I64, P, P, I64, P, P],
+                                     ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(_lib, name)
@@ -123,6 +130,21 @@ def pack8(codes) -> int:
 def unpack8(word: int) -> np.ndarray:
     q = np.zeros(8, np.uint8)
     _L().oracle_unpack8(ctypes.c_uint32(word), _p(q))
+    return q
+
+
+def pack32x3(codes) -> np.ndarray:
+    """32 codes (0..7, element order) -> the 3 words of the 3-bit layout."""
+    q = _c(codes, np.uint8)
+    w = np.zeros(3, np.uint32)
+    _check(_L().oracle_pack32x3(_p(q), _p(w)), "pack32x3")
+    return w
+
+
+def unpack32x3(words) -> np.ndarray:
+    w = _c(words, np.uint32)
+    q = np.zeros(32, np.uint8)
+    _L().oracle_unpack32x3(_p(w), _p(q))
     return q
 
 
@@ -218,6 +240,58 @@ def linear_at(x_bf16_bits, qweight, scales, zeros, N: int, m_idx, n_idx, csr=Non
     ya = np.zeros(mi.size, np.float64) if with_abs else None
     _check(_L().oracle_linear_at_gs(_p(x), M, K, group_size, _p(qw), _p(sc), _p(z), N, _p(rp), _p(ci), _p(v),
                                     nnz, _p(mi), _p(ni), mi.size, _p(y), _p(ya)), "linear_at")
+    return (y, ya) if with_abs else y
+
+
+def awq_quantize3(W, act_absmean, alpha: float, group_size: int = 128):
+    """AWQ quantize with 3-bit codes -> (qweight3 u32 [N][3K/32], scales u16 [K/gs][N],
+    zeros u32 [K/gs][N/8] (nibbles 0..7), s f32 [K])"""
+    W = _c(W, np.float32)
+    a = _c(act_absmean, np.float32)
+    N, K = W.shape
+    G = max(K // group_size, 1)
+    qw = np.zeros((N, 3 * K // 32), np.uint32)
+    sc = np.zeros((G, N), np.uint16)
+    z = np.zeros((G, max(N // 8, 1)), np.uint32)
+    s = np.zeros(K, np.float32)
+    _check(_L().oracle_awq_quantize3_gs(_p(W), _p(a), ctypes.c_float(alpha), N, K, group_size, _p(qw), _p(sc),
+                                        _p(z), _p(s)), "awq_quantize3")
+    return qw, sc, z, s
+
+
+def dequant3(qweight3, scales, zeros, N: int, K: int, group_size: int = 128) -> np.ndarray:
+    qw, sc, z = _c(qweight3, np.uint32), _c(scales, np.uint16), _c(zeros, np.uint32)
+    out = np.zeros((N, K), np.float32)
+    _check(_L().oracle_dequant3_gs(_p(qw), _p(sc), _p(z), N, K, group_size, _p(out)), "dequant3")
+    return out
+
+
+def linear3(x_bf16_bits, qweight3, scales, zeros, N: int, csr=None, with_abs: bool = False,
+            group_size: int = 128):
+    """``linear`` on 3-bit weights."""
+    x = _c(x_bf16_bits, np.uint16)
+    M, K = x.shape
+    qw, sc, z = _c(qweight3, np.uint32), _c(scales, np.uint16), _c(zeros, np.uint32)
+    rp, ci, v, nnz = _csr_args(csr)
+    y = np.zeros((M, N), np.float64)
+    ya = np.zeros((M, N), np.float64) if with_abs else None
+    _check(_L().oracle_linear3_gs(_p(x), M, K, group_size, _p(qw), _p(sc), _p(z), N, _p(rp), _p(ci), _p(v), nnz,
+                                  _p(y), _p(ya)), "linear3")
+    return (y, ya) if with_abs else y
+
+
+def linear3_at(x_bf16_bits, qweight3, scales, zeros, N: int, m_idx, n_idx, csr=None,
+               with_abs: bool = False, group_size: int = 128):
+    """The outputs of ``linear3`` at the positions (m_idx[p], n_idx[p]) only."""
+    x = _c(x_bf16_bits, np.uint16)
+    M, K = x.shape
+    qw, sc, z = _c(qweight3, np.uint32), _c(scales, np.uint16), _c(zeros, np.uint32)
+    mi, ni = _c(m_idx, np.int64), _c(n_idx, np.int64)
+    rp, ci, v, nnz = _csr_args(csr)
+    y = np.zeros(mi.size, np.float64)
+    ya = np.zeros(mi.size, np.float64) if with_abs else None
+    _check(_L().oracle_linear3_at_gs(_p(x), M, K, group_size, _p(qw), _p(sc), _p(z), N, _p(rp), _p(ci), _p(v),
+                                     nnz, _p(mi), _p(ni), mi.size, _p(y), _p(ya)), "linear3_at")
     return (y, ya) if with_abs else y
 
 

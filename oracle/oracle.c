@@ -21,6 +21,8 @@
  *     size option, per-row by default];
  *   - 4-bit weight packing, 8 codes per 32-bit word [AWQ translation, section 1:
  *     TinyChat's 4-bit weight packing];
+ *   - a 3-bit variant: the same RTN with eight levels, 32 codes per three 32-bit words
+ *     [SqueezeLLM article, sections 2.1-2.2: the dense part quantized as coarse as 3 bits];
  *   - the dense-and-sparse product  W x = W_dense x + W_sparse x  with an fp16 CSR
  *     W_sparse [SqueezeLLM article, sections 2.2 and 2.3; the page lost the "=" and
  *     "+" signs, read here as written above];
@@ -162,20 +164,22 @@ int oracle_awq_scales(const float* act_absmean, int64_t K, float alpha, float* s
     return ORACLE_OK;
 }
 
-/* One group of gs scaled weights -> fp16 scale bits, zero point, gs codes.
- *   scale32 = max((max - min) / 15, 1e-5)          (plain asymmetric min/max range)
+/* One group of gs scaled weights -> fp16 scale bits, zero point, gs codes, with qmax + 1
+ * levels (qmax = 15 for 4-bit codes, 7 for 3-bit):
+ *   scale32 = max((max - min) / qmax, 1e-5)        (plain asymmetric min/max range)
  *   sf      = float(fp16_rne(scale32))             (the stored scale is the one used)
- *   z       = clamp(rint(-min / sf), 0, 15)
- *   q_i     = clamp(rint(w_i / sf) + z, 0, 15)     (round first, then add the zero)
+ *   z       = clamp(rint(-min / sf), 0, qmax)
+ *   q_i     = clamp(rint(w_i / sf) + z, 0, qmax)   (round first, then add the zero)
  * rint is round-half-to-even; every operation is one IEEE float operation. */
-static int quantize_group(const float* wp, int64_t gs, uint16_t* s16_out, uint8_t* z_out, uint8_t* q_out) {
+static int quantize_group(const float* wp, int64_t gs, float qmax, uint16_t* s16_out, uint8_t* z_out,
+                          uint8_t* q_out) {
     float mx = wp[0], mn = wp[0];
     for (int64_t i = 0; i < gs; ++i) {
         if (!isfinite(wp[i])) return ORACLE_ERR_VALUE;
         if (wp[i] > mx) mx = wp[i];
         if (wp[i] < mn) mn = wp[i];
     }
-    float scale32 = (mx - mn) / 15.0f;
+    float scale32 = (mx - mn) / qmax;
     if (scale32 < 1e-5f) scale32 = 1e-5f;
     if (isinf(scale32)) return ORACLE_ERR_VALUE; /* max - min overflowed */
     uint16_t s16 = oracle_f32_to_f16(scale32);
@@ -183,11 +187,11 @@ static int quantize_group(const float* wp, int64_t gs, uint16_t* s16_out, uint8_
     float sf = oracle_f16_to_f32(s16);
     float zf = rintf(-mn / sf);
     if (zf < 0.0f) zf = 0.0f;
-    if (zf > 15.0f) zf = 15.0f;
+    if (zf > qmax) zf = qmax;
     for (int64_t i = 0; i < gs; ++i) {
         float qf = rintf(wp[i] / sf) + zf;
         if (qf < 0.0f) qf = 0.0f;
-        if (qf > 15.0f) qf = 15.0f;
+        if (qf > qmax) qf = qmax;
         q_out[i] = (uint8_t)qf;
     }
     *s16_out = s16;
@@ -210,14 +214,20 @@ static int zero_of(const uint32_t* zeros, int64_t N, int64_t n, int64_t g) {
     return (int)((zeros[g * (N / 8) + n / 8] >> (4 * (n % 8))) & 15u);
 }
 
+int oracle_pack32x3(const uint8_t* q, uint32_t* words);
+
 /* Quantize W (fp32 [N][K]) with a given per-channel scale s ([K]) in groups of gs along K:
- * w' = float(w * s_k), then quantize_group on each run of gs along K, then pack. */
-int oracle_quantize_with_scales_gs(const float* W, const float* s, int64_t N, int64_t K, int64_t gs,
-                                   uint32_t* qweight, uint16_t* scales, uint32_t* zeros) {
+ * w' = float(w * s_k), then quantize_group on each run of gs along K, then pack: 4-bit
+ * codes 8 per word, or 3-bit codes 32 per 3 words (gs a multiple of 32). */
+static int quantize_with_scales_bits(const float* W, const float* s, int64_t N, int64_t K, int64_t gs, int bits,
+                                     uint32_t* qweight, uint16_t* scales, uint32_t* zeros) {
     if (!W || !s || !qweight || !scales || !zeros) return ORACLE_ERR_NULL;
     int st = check_qshape(N, K);
     if (!st) st = check_gs(K, gs);
+    if (!st && bits == 3 && gs % 32 != 0) st = ORACLE_ERR_SHAPE;
+    if (!st && bits != 3 && bits != 4) st = ORACLE_ERR_SHAPE;
     if (st) return st;
+    const float qmax = bits == 4 ? 15.0f : 7.0f;
     const int64_t G = K / gs;
     int err = ORACLE_OK;
     uint8_t* zcode = (uint8_t*)malloc((size_t)(N * G));
@@ -237,7 +247,7 @@ int oracle_quantize_with_scales_gs(const float* W, const float* s, int64_t N, in
                 for (int64_t i = 0; i < gs; ++i) wp[i] = W[n * K + g * gs + i] * s[g * gs + i];
                 uint16_t s16;
                 uint8_t z;
-                int e = quantize_group(wp, gs, &s16, &z, q);
+                int e = quantize_group(wp, gs, qmax, &s16, &z, q);
                 if (e) {
 #pragma omp atomic write
                     err = e;
@@ -245,10 +255,15 @@ int oracle_quantize_with_scales_gs(const float* W, const float* s, int64_t N, in
                 }
                 scales[g * N + n] = s16;
                 zcode[n * G + g] = z;
-                for (int64_t w = 0; w < gs / 8; ++w) {
-                    uint32_t word;
-                    oracle_pack8(&q[8 * w], &word);
-                    qweight[n * (K / 8) + g * (gs / 8) + w] = word;
+                if (bits == 4) {
+                    for (int64_t w = 0; w < gs / 8; ++w) {
+                        uint32_t word;
+                        oracle_pack8(&q[8 * w], &word);
+                        qweight[n * (K / 8) + g * (gs / 8) + w] = word;
+                    }
+                } else {
+                    for (int64_t b = 0; b < gs / 32; ++b)
+                        oracle_pack32x3(&q[32 * b], &qweight[n * (K / 32) * 3 + (g * (gs / 32) + b) * 3]);
                 }
             }
         }
@@ -264,6 +279,11 @@ int oracle_quantize_with_scales_gs(const float* W, const float* s, int64_t N, in
         }
     free(zcode);
     return err;
+}
+
+int oracle_quantize_with_scales_gs(const float* W, const float* s, int64_t N, int64_t K, int64_t gs,
+                                   uint32_t* qweight, uint16_t* scales, uint32_t* zeros) {
+    return quantize_with_scales_bits(W, s, N, K, gs, 4, qweight, scales, zeros);
 }
 
 int oracle_quantize_with_scales(const float* W, const float* s, int64_t N, int64_t K,
@@ -337,19 +357,31 @@ static int check_csr(const int32_t* row_ptr, const int32_t* col_idx, const uint1
     return ORACLE_OK;
 }
 
+void oracle_unpack32x3(const uint32_t* words, uint8_t* q);
+
+/* The code of element k of row n: 4-bit layout (8 per word) or 3-bit layout (32 per 3 words). */
+static int code_at(const uint32_t* qweight, int bits, int64_t K, int64_t n, int64_t k) {
+    if (bits == 4) {
+        uint8_t codes[8];
+        oracle_unpack8(qweight[n * (K / 8) + k / 8], codes);
+        return codes[k % 8];
+    }
+    uint8_t codes[32];
+    oracle_unpack32x3(&qweight[n * (K / 32) * 3 + (k / 32) * 3], codes);
+    return codes[k % 32];
+}
+
 /* One output y[m][n] = sum_k x[m][k] deq[n][k] + sum_{j in row n} x[m][col_j] val_j, summed
  * in double (each product of a bf16 and a dequantized weight or fp16 value is exact in
  * double), plus the sum of the absolute products, which bounds any rounding error. */
-static void one_output(const uint16_t* x, int64_t K, int64_t N, int64_t gs, const uint32_t* qweight,
+static void one_output(const uint16_t* x, int64_t K, int64_t N, int64_t gs, int bits, const uint32_t* qweight,
                        const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
                        const int32_t* col_idx, const uint16_t* values, int64_t m, int64_t n,
                        double* y, double* yabs) {
     double acc = 0.0, aacc = 0.0;
     for (int64_t k = 0; k < K; ++k) {
         int64_t g = k / gs;
-        uint8_t codes[8];
-        oracle_unpack8(qweight[n * (K / 8) + k / 8], codes);
-        int q = codes[k % 8];
+        int q = code_at(qweight, bits, K, n, k);
         int z = zero_of(zeros, N, n, g);
         double w = (double)((float)(q - z) * oracle_f16_to_f32(scales[g * N + n]));
         double p = (double)oracle_bf16_to_f32(x[m * K + k]) * w;
@@ -371,10 +403,10 @@ static void one_output(const uint16_t* x, int64_t K, int64_t N, int64_t gs, cons
 /* y = x deq(Q)^T + x W_sparse^T for all (m, n): x bf16 [M][K]; y, yabs double [M][N].
  * The CSR (row_ptr [N+1], col_idx/values [nnz], ascending columns per row) may be absent
  * (row_ptr == NULL and nnz == 0). */
-int oracle_linear_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, const uint32_t* qweight,
-                     const uint16_t* scales, const uint32_t* zeros, int64_t N,
-                     const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
-                     int64_t nnz, double* y, double* yabs) {
+static int linear_bits(const uint16_t* x, int64_t M, int64_t K, int64_t gs, int bits, const uint32_t* qweight,
+                       const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                       const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                       int64_t nnz, double* y, double* yabs) {
     if (!x || !qweight || !scales || !zeros || !y) return ORACLE_ERR_NULL;
     if (M <= 0) return ORACLE_ERR_SHAPE;
     int st = check_qshape(N, K);
@@ -385,9 +417,16 @@ int oracle_linear_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, const 
 #pragma omp parallel for collapse(2) schedule(dynamic, 16)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n)
-            one_output(x, K, N, gs, qweight, scales, zeros, row_ptr, col_idx, values, m, n,
+            one_output(x, K, N, gs, bits, qweight, scales, zeros, row_ptr, col_idx, values, m, n,
                        &y[m * N + n], yabs ? &yabs[m * N + n] : NULL);
     return ORACLE_OK;
+}
+
+int oracle_linear_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, const uint32_t* qweight,
+                     const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                     const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                     int64_t nnz, double* y, double* yabs) {
+    return linear_bits(x, M, K, gs, 4, qweight, scales, zeros, N, row_ptr, col_idx, values, nnz, y, yabs);
 }
 
 int oracle_linear(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweight,
@@ -398,11 +437,11 @@ int oracle_linear(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweig
 }
 
 /* The same outputs at P sampled positions (m_idx[p], n_idx[p]) only. */
-int oracle_linear_at_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, const uint32_t* qweight,
-                        const uint16_t* scales, const uint32_t* zeros, int64_t N,
-                        const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
-                        int64_t nnz, const int64_t* m_idx, const int64_t* n_idx, int64_t P,
-                        double* y, double* yabs) {
+static int linear_at_bits(const uint16_t* x, int64_t M, int64_t K, int64_t gs, int bits,
+                          const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                          const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                          int64_t nnz, const int64_t* m_idx, const int64_t* n_idx, int64_t P,
+                          double* y, double* yabs) {
     if (!x || !qweight || !scales || !zeros || !y || !m_idx || !n_idx) return ORACLE_ERR_NULL;
     if (M <= 0 || P < 0) return ORACLE_ERR_SHAPE;
     int st = check_qshape(N, K);
@@ -414,9 +453,18 @@ int oracle_linear_at_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, con
         if (m_idx[p] < 0 || m_idx[p] >= M || n_idx[p] < 0 || n_idx[p] >= N) return ORACLE_ERR_SHAPE;
 #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t p = 0; p < P; ++p)
-        one_output(x, K, N, gs, qweight, scales, zeros, row_ptr, col_idx, values, m_idx[p], n_idx[p],
+        one_output(x, K, N, gs, bits, qweight, scales, zeros, row_ptr, col_idx, values, m_idx[p], n_idx[p],
                    &y[p], yabs ? &yabs[p] : NULL);
     return ORACLE_OK;
+}
+
+int oracle_linear_at_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, const uint32_t* qweight,
+                        const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                        const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                        int64_t nnz, const int64_t* m_idx, const int64_t* n_idx, int64_t P,
+                        double* y, double* yabs) {
+    return linear_at_bits(x, M, K, gs, 4, qweight, scales, zeros, N, row_ptr, col_idx, values, nnz, m_idx, n_idx,
+                          P, y, yabs);
 }
 
 int oracle_linear_at(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweight,
@@ -426,6 +474,93 @@ int oracle_linear_at(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qw
                      double* y, double* yabs) {
     return oracle_linear_at_gs(x, M, K, GROUP, qweight, scales, zeros, N, row_ptr, col_idx, values, nnz, m_idx,
                                n_idx, P, y, yabs);
+}
+
+/* ------------------------------------------------------------------------------------
+ * 3-bit codes [SqueezeLLM article, sections 2.1 and 2.2: once its few outliers are split
+ * off, the dense part takes uniform quantization as coarse as 3 bits, eight levels].  Read
+ * as the same asymmetric min/max RTN with 2^3 - 1 steps (quantize_group with qmax = 7),
+ * the same groups, scales [K/gs][N] fp16 and zeros [K/gs][N/8] (nibbles, values 0..7).
+ * Packed layout, 3 bits per weight: the 32 codes of k = 32 b .. 32 b + 31 of row n sit in
+ * the three words qweight3[n][3 b + w], w = 0, 1, 2:
+ *   - bits 4j .. 4j+2 of word w: the code of element 8 w + ORDER[j]     (elements 0..23);
+ *   - bit 4j + 3 of word w: bit w of the code of element 24 + ORDER[j]  (elements 24..31).
+ * Then (word >> 4i) & 0x00070007 holds elements (8 w + 2i, 8 w + 2i + 1) in its two 16-bit
+ * halves, as 0x000F000F does for the 4-bit layout, and the bit-3 planes of the three words,
+ * shifted by 4i + 3, 4i + 2 and 4i + 1 and masked with 0x00010001, 0x00020002 and
+ * 0x00040004, hold elements (24 + 2i, 24 + 2i + 1) the same way.
+ * ---------------------------------------------------------------------------------- */
+int oracle_pack32x3(const uint8_t* q /* 32 codes, element order */, uint32_t* words /* 3 */) {
+    uint32_t w[3] = {0u, 0u, 0u};
+    for (int e = 0; e < 32; ++e)
+        if (q[e] > 7) return ORACLE_ERR_VALUE;
+    for (int wi = 0; wi < 3; ++wi)
+        for (int j = 0; j < 8; ++j) {
+            w[wi] |= (uint32_t)q[8 * wi + ORACLE_ORDER[j]] << (4 * j);
+            w[wi] |= (uint32_t)((q[24 + ORACLE_ORDER[j]] >> wi) & 1u) << (4 * j + 3);
+        }
+    memcpy(words, w, sizeof w);
+    return ORACLE_OK;
+}
+
+void oracle_unpack32x3(const uint32_t* words /* 3 */, uint8_t* q /* 32 codes, element order */) {
+    for (int e = 0; e < 24; ++e) q[e] = (uint8_t)((words[e / 8] >> (4 * nibble_of_element(e % 8))) & 7u);
+    for (int e = 24; e < 32; ++e) {
+        const int j = nibble_of_element(e - 24);
+        uint8_t c = 0;
+        for (int wi = 0; wi < 3; ++wi) c |= (uint8_t)(((words[wi] >> (4 * j + 3)) & 1u) << wi);
+        q[e] = c;
+    }
+}
+
+/* awq_quantize with 3-bit codes: s from act_absmean and alpha, then W*s in groups of gs
+ * (a multiple of 32 dividing K); qweight3 is [N][3K/32]. */
+int oracle_awq_quantize3_gs(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                            int64_t gs, uint32_t* qweight3, uint16_t* scales, uint32_t* zeros, float* s_out) {
+    if (!W || !act_absmean || !qweight3 || !scales || !zeros) return ORACLE_ERR_NULL;
+    int st = check_qshape(N, K);
+    if (!st) st = check_gs(K, gs);
+    if (!st && gs % 32 != 0) st = ORACLE_ERR_SHAPE;
+    if (st) return st;
+    float* s = (float*)malloc(sizeof(float) * (size_t)K);
+    if (!s) return ORACLE_ERR_VALUE;
+    st = oracle_awq_scales(act_absmean, K, alpha, s);
+    if (!st) st = quantize_with_scales_bits(W, s, N, K, gs, 3, qweight3, scales, zeros);
+    if (!st && s_out) memcpy(s_out, s, sizeof(float) * (size_t)K);
+    free(s);
+    return st;
+}
+
+/* deq[n][k] = (q - z) * sf for the 3-bit layout, exact in fp32. */
+int oracle_dequant3_gs(const uint32_t* qweight3, const uint16_t* scales, const uint32_t* zeros, int64_t N,
+                       int64_t K, int64_t gs, float* deq) {
+    if (!qweight3 || !scales || !zeros || !deq) return ORACLE_ERR_NULL;
+    int st = check_qshape(N, K);
+    if (!st) st = check_gs(K, gs);
+    if (st) return st;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            const int64_t g = k / gs;
+            deq[n * K + k] = (float)(code_at(qweight3, 3, K, n, k) - zero_of(zeros, N, n, g)) *
+                             oracle_f16_to_f32(scales[g * N + n]);
+        }
+    return ORACLE_OK;
+}
+
+/* The linear (all outputs, or P sampled ones) on 3-bit weights; otherwise as oracle_linear_gs. */
+int oracle_linear3_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, const uint32_t* qweight3,
+                      const uint16_t* scales, const uint32_t* zeros, int64_t N, const int32_t* row_ptr,
+                      const int32_t* col_idx, const uint16_t* values, int64_t nnz, double* y, double* yabs) {
+    return linear_bits(x, M, K, gs, 3, qweight3, scales, zeros, N, row_ptr, col_idx, values, nnz, y, yabs);
+}
+
+int oracle_linear3_at_gs(const uint16_t* x, int64_t M, int64_t K, int64_t gs, const uint32_t* qweight3,
+                         const uint16_t* scales, const uint32_t* zeros, int64_t N, const int32_t* row_ptr,
+                         const int32_t* col_idx, const uint16_t* values, int64_t nnz, const int64_t* m_idx,
+                         const int64_t* n_idx, int64_t P, double* y, double* yabs) {
+    return linear_at_bits(x, M, K, gs, 3, qweight3, scales, zeros, N, row_ptr, col_idx, values, nnz, m_idx, n_idx,
+                          P, y, yabs);
 }
 
 /* ------------------------------------------------------------------------------------
