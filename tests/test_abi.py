@@ -180,3 +180,13 @@ def test_binding_has_no_cpu_path():
     with pytest.raises(ValueError):
         w4.w4a16_linear(x, torch.zeros(128, 128, dtype=torch.int32), torch.zeros(128, 8, dtype=torch.int16),
                         torch.zeros(128, 1, dtype=torch.int32))
+
+
+def test_binding_has_every_entry_point_by_name():
+    """The Python binding offers each C entry point under the same name."""
+    for name in declared_functions():
+        assert callable(getattr(w4, name, None)), name
+    want = int(w4.lib().awq_split_outliers_workspace_bytes(256, 1024))
+    assert w4.awq_split_outliers_workspace_bytes(256, 1024) == want
+    assert w4.w4a16_version() == w4.version()
+    assert w4.w4a16_status_string(w4.ERR_SHAPE) == w4.status_string(w4.ERR_SHAPE)

@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
                                     ctypes.c_int, P]
         L.w4a16_gemv_folded.argtypes = [P, P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, I64, P,
                                         ctypes.c_size_t, ctypes.c_int, P]
+        L.w4a16_gemv_noalloc.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P]
         PI = ctypes.POINTER(ctypes.c_int)
         L.w4a16_gemv_plan.argtypes = [I64, I64, I64, ctypes.c_int, PI, PI, PI]
         L.w4a16_workspace_bytes.argtypes = [I64, I64, I64]
@@ -322,3 +323,42 @@ def status_string(code: int) -> str:
 
 def version() -> int:
     return lib().w4a16_version()
+
+
+# ---- the remaining entry points under their C names -------------------------------------
+
+def w4a16_gemv_noalloc(x, qweight, scales, zeros, csr=None, out=None):
+    """The decode GEMV without a caller workspace (the library's static scratch)."""
+    _need(x, torch.bfloat16, 2, "x")
+    _need(qweight, torch.int32, 2, "qweight")
+    _need(scales, torch.int16, 2, "scales")
+    _need(zeros, torch.int32, 2, "zeros")
+    M, K = x.shape
+    N = qweight.shape[0]
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    cs = None
+    if csr is not None:
+        rp, ci, v = csr
+        _need(rp, torch.int32, 1, "row_ptr")
+        cs = Csr(rp.data_ptr(), ci.data_ptr() if ci.numel() else None, v.data_ptr() if v.numel() else None,
+                 int(ci.numel()))
+    _check(lib().w4a16_gemv_noalloc(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros),
+                                    ctypes.byref(cs) if cs is not None else None, _ptr(y), M, N, K,
+                                    _stream(x.device)), "w4a16_gemv_noalloc")
+    return y
+
+
+def awq_split_outliers_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().awq_split_outliers_workspace_bytes(N, K))
+
+
+def awq_search_alpha_workspace_bytes(M: int, N: int, K: int, n_alpha: int) -> int:
+    return int(lib().awq_search_alpha_workspace_bytes(M, N, K, int(n_alpha)))
+
+
+w4a16_workspace_bytes = workspace_bytes
+w4a16_gemv_plan = gemv_plan
+w4a16_check_device_status = check_device_status
+w4a16_selftest_timeout = selftest_timeout
+w4a16_status_string = status_string
+w4a16_version = version
