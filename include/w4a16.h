@@ -123,16 +123,18 @@ w4a16_status awq_quantize(const float* W, const float* act_absmean, float alpha,
  * Workspace of the decode path.  The GEMV splits the output row blocks evenly over a
  * persistent grid.  Row blocks shared by two or more CTAs are combined through fp32
  * partial tiles and per-row-block counters, which live in a caller-provided device
- * workspace.
+ * workspace; w4a16_gemv_folded also writes its x / s there.
  *   - It must hold at least w4a16_workspace_bytes(M, N, K) bytes and be 16-byte aligned.
- *   - It must be zero-filled before its first use.  Every call that completes leaves it
- *     zero-filled again, so one workspace serves any number of calls in stream order.
+ *   - It must be zero-filled before its first use.  Every call that completes leaves the
+ *     parts that must start at zero zero-filled again, whatever its sizes, so one workspace
+ *     of the largest size needed serves any number of calls of any sizes in stream order.
  *   - Calls that may run at the same time (on different streams without ordering between
  *     them) need different workspaces.
  *   - After a call reports W4A16_ERR_TIMEOUT, zero the workspace again before reusing it.
  * w4a16_workspace_bytes returns the size for the CURRENT device (it depends on the number
  * of SMs), or 0 when the call with these sizes needs no workspace (M > 16) or the sizes
- * are invalid.  Its value for a given device and N does not depend on M or K.
+ * are invalid.  It is 128 KiB of counters, 16 KiB of partial tiles per SM, and M x K bf16
+ * for the folded activations (rounded up to 256 bytes); it does not depend on N.
  */
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -215,22 +217,21 @@ w4a16_status w4a16_linear_ex(const uint16_t* x, const uint32_t* qweight, const u
                              int64_t M, int64_t N, int64_t K, int64_t group_size, void* workspace,
                              size_t workspace_bytes, int schedule, void* stream);
 
-/* w4a16_gemv_folded -- the decode GEMV on the layer input BEFORE the AWQ scaling: the
- * kernel divides x by the per-channel scale s as it loads it, so no separate pass over x
- * is needed.  [AWQ translation, 3.2: the weights are multiplied by s and the activations
- * divided by it; 1 (TinyChat): kernel fusion to avoid intermediate DRAM round trips and
- * launches.]
+/* w4a16_gemv_folded -- the decode GEMV on the layer input BEFORE the AWQ scaling, as one call.
+ * [AWQ translation, 3.2: the weights are multiplied by s and the activations divided by it.]
  *   x   [M][K] bf16 bits, device: the raw layer input.
  *   s   [K] fp32, device, 16-byte aligned: the scales awq_quantize wrote to s_out; or NULL,
  *       for an x that is already divided (the call is then w4a16_linear_ex's decode path).
- *   The kernel uses x'[m][k] = bf16_rne(float(x[m][k]) / s[k]) (IEEE division), for the
- *   quantized product and for the sparse term: the values awq_fold_activations writes, so
- *   y is bit-identical to awq_fold_activations followed by w4a16_gemv_ex with the same
- *   schedule.  s is read after the previous kernel on the stream has finished.
+ *   With s, the call first writes x'[m][k] = bf16_rne(float(x[m][k]) / s[k]) (IEEE division)
+ *   into the workspace, once, and the GEMV (launched so that it streams its weights while
+ *   that pass runs) then reads x' for the quantized product and the sparse term: the values
+ *   awq_fold_activations writes, so y is bit-identical to awq_fold_activations followed by
+ *   w4a16_gemv_ex with the same schedule.  (Dividing inside the GEMV's own activation load
+ *   was built and measured slower: every CTA divides the activations of every unit it
+ *   streams, so each element is divided once per row block instead of once.)
  *   group_size, schedule: as w4a16_linear_ex.  1 <= M <= 16 (SHAPE otherwise).
  *   Everything else is as for w4a16_gemv_ex; ALIGN also for a misaligned s.
- * For M > 16 the tensor-core GEMM loads x with TMA, which cannot divide: run
- * awq_fold_activations first, then w4a16_gemm. */
+ * For M > 16 run awq_fold_activations first, then w4a16_gemm. */
 w4a16_status w4a16_gemv_folded(const uint16_t* x, const float* s, const uint32_t* qweight,
                                const uint16_t* scales, const uint32_t* zeros,
                                const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N,

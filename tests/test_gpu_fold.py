@@ -1,11 +1,10 @@
-"""The decode GEMV with the 1/s fold inside its activation load (w4a16_gemv_folded).
+"""The decode GEMV on raw activations with the 1/s fold in the same call (w4a16_gemv_folded).
 
 x' = bf16(x / s) is what the linear entry points take [AWQ translation, section 3.2: the
-weights are multiplied by s and the activations divided by it]; folding that division into
-the kernel's load of x saves a pass over x [AWQ translation, section 1: TinyChat's kernel
-fusion].  The fused call must give the same bits as awq_fold_activations followed by the
-GEMV (same conversions, same arithmetic afterwards), and the oracle's result for the folded
-activations within the tolerance of the unfused GEMV."""
+weights are multiplied by s and the activations divided by it].  The folded call divides x
+once into its workspace and runs the GEMV on the result; it must give the same bits as
+awq_fold_activations followed by the GEMV (same conversions, same arithmetic afterwards), and
+the oracle's result for the folded activations within the tolerance of the unfused GEMV."""
 import numpy as np
 import pytest
 import torch

@@ -237,8 +237,9 @@ def w4a16_linear_ex(x, qweight, scales, zeros, csr=None, out=None, workspace=Non
 
 def w4a16_gemv_folded(x, s, qweight, scales, zeros, csr=None, out=None, workspace=None, group_size=128,
                       schedule=GEMV_AUTO):
-    """The decode GEMV on the raw layer input: x is divided by the channel scales s (fp32 [K],
-    or None for an already divided x) inside the kernel, as awq_fold_activations would."""
+    """The decode GEMV on the raw layer input in one call: x is divided by the channel scales s
+    (fp32 [K], or None for an already divided x) into the workspace, as awq_fold_activations
+    would, and the GEMV reads the result."""
     return _linear("w4a16_gemv_folded", x, qweight, scales, zeros, csr, out, workspace, schedule, group_size,
                    fold=True, s=s)
 

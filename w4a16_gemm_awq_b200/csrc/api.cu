@@ -17,20 +17,24 @@ namespace w4a16 {
 // Problems found by kernels while they run (bit set of kErrValue / kErrShape / kErrTimeout).
 __device__ unsigned g_device_status;
 
-// Scratch of w4a16_gemv_noalloc: the decode GEMV's workspace (fp32 partial tiles, then the
-// per-row-block counters) for devices with up to kNoallocMaxSms SMs and N up to
-// kNoallocMaxN.  It is part of the loaded module: every GPU that loads the library holds
-// it until the process exits, and every call of w4a16_gemv_noalloc on that GPU uses it.
+// Scratch of w4a16_gemv_noalloc: the decode GEMV's row-block counters for N up to
+// kNoallocMaxN, then its fp32 partial tiles for devices with up to kNoallocMaxSms SMs.  It is
+// part of the loaded module: every GPU that loads the library holds it until the process
+// exits, and every call of w4a16_gemv_noalloc on that GPU uses it.
 constexpr int kNoallocMaxSms = 160;
 constexpr int kNoallocMaxN = 131072;
+constexpr size_t kNoallocCounterBytes = (size_t)(kNoallocMaxN / 128) * sizeof(unsigned);
 constexpr size_t kNoallocScratchBytes =
-    (size_t)2 * 2 * kNoallocMaxSms * 128 * 16 * sizeof(float) + (size_t)(kNoallocMaxN / 128) * sizeof(unsigned);
+    kNoallocCounterBytes + (size_t)2 * kNoallocMaxSms * kGemvSlotFloats * sizeof(float);
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxN = int64_t(1) << 22;
+// The decode workspace of the public entry points starts with the row-block counters of the
+// largest N, so that their place never depends on the call's sizes.
+constexpr size_t kCounterRegionBytes = (size_t)(kMaxN / 128) * sizeof(unsigned);
 constexpr int64_t kMaxK = int64_t(1) << 20;
 constexpr int64_t kMaxM = int64_t(1) << 24;
 
@@ -107,7 +111,6 @@ inline w4a16_status from_cuda(cudaError_t e) { return e == cudaSuccess ? W4A16_O
 
 struct LinearArgs {
     const uint16_t* x;
-    const float* s = nullptr;  // the decode GEMV divides x by s as it loads it
     const uint32_t* qweight;
     const uint16_t* scales;
     const uint32_t* zeros;
@@ -118,8 +121,8 @@ struct LinearArgs {
     uint16_t* y;
     int64_t M, N, K;
     int group_ratio = 1;  // group size / 128
-    void* workspace = nullptr;
-    size_t workspace_bytes = 0;
+    float* partials = nullptr;   // the GEMV's scratch (gemv_partial_bytes)
+    unsigned* counters = nullptr;  // zero when the call starts (gemv_counter_bytes)
 };
 
 w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -130,7 +133,7 @@ w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const u
         return W4A16_ERR_SHAPE;
     if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(zeros, 16) || !aligned(y, 16))
         return W4A16_ERR_ALIGN;
-    *a = LinearArgs{x, nullptr, qweight, scales, zeros};
+    *a = LinearArgs{x, qweight, scales, zeros};
     a->y = y;
     a->M = M;
     a->N = N;
@@ -165,14 +168,13 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
     if (a.K > gemv_max_k() || !gemv_fits((int)a.N, (int)a.K, d->num_sms)) return W4A16_ERR_UNSUPPORTED;
     const GemvPlan plan = gemv_plan((int)a.M, (int)a.N, (int)a.K, d->num_sms, schedule);
     if (plan.ctas < 1) return W4A16_ERR_UNSUPPORTED;
-    if (a.workspace == nullptr) return W4A16_ERR_NULL;
-    if (!aligned(a.workspace, 16)) return W4A16_ERR_ALIGN;
-    if (a.workspace_bytes < gemv_workspace_bytes((int)a.N, d->num_sms)) return W4A16_ERR_SHAPE;
+    if (a.partials == nullptr || a.counters == nullptr) return W4A16_ERR_NULL;
     GemvMaps maps;
     {
         EncodeTiledFn enc = nullptr;
         st = encoder(&enc);
         if (st != W4A16_OK) return st;
+        // qweight: 16 words of a group x 128 rows x 4 groups per copy
         cuuint64_t dims[3] = {16, (cuuint64_t)a.N, (cuuint64_t)(a.K / 128)};
         cuuint64_t strides[2] = {(cuuint64_t)(a.K / 2), 64};
         cuuint32_t box[3] = {16, 128, 4};
@@ -182,9 +184,36 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4A16_ERR_CUDA;
     }
-    return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.s, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals,
-                                 a.nnz, a.y, a.workspace, (int)a.M, (int)a.N, (int)a.K, d->num_sms, d->status,
+    return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals,
+                                 a.nnz, a.y, a.partials, a.counters, (int)a.M, (int)a.N, (int)a.K, d->status,
                                  stream));
+}
+
+// The decode workspace of the public entry points:
+//   [0, kCounterRegionBytes)   the GEMV's row-block counters (zero between calls);
+//   then gemv_partial_bytes    its fp32 partial tiles;
+//   then M x K bf16            x / s of w4a16_gemv_folded, rounded up to 256 bytes.
+// Only the last part depends on the call's sizes, and it lies after everything else, so one
+// zeroed workspace serves calls of any sizes in stream order.
+size_t fold_region_bytes(int64_t M, int64_t K) { return ((size_t)M * (size_t)K * 2 + 255) / 256 * 256; }
+
+size_t decode_workspace_bytes(int64_t M, int64_t K, int num_sms) {
+    return kCounterRegionBytes + gemv_partial_bytes(num_sms) + fold_region_bytes(M, K);
+}
+
+// Checks the caller's decode workspace and points a at its parts; *fold = the x / s region.
+w4a16_status take_decode_workspace(LinearArgs* a, void* workspace, size_t workspace_bytes, uint16_t** fold) {
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    if (workspace == nullptr) return W4A16_ERR_NULL;
+    if (!aligned(workspace, 16)) return W4A16_ERR_ALIGN;
+    if (workspace_bytes < decode_workspace_bytes(a->M, a->K, d->num_sms)) return W4A16_ERR_SHAPE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a->counters = reinterpret_cast<unsigned*>(ws);
+    a->partials = reinterpret_cast<float*>(ws + kCounterRegionBytes);
+    if (fold) *fold = reinterpret_cast<uint16_t*>(ws + kCounterRegionBytes + gemv_partial_bytes(d->num_sms));
+    return W4A16_OK;
 }
 
 int pick_bn(int64_t M) {
@@ -245,7 +274,7 @@ SearchLayout search_layout(int64_t M, int64_t N, int64_t K, int n_alpha, int num
     L.yq = off; off += up((size_t)M * N * 2);
     L.yref = off; off += up((size_t)M * N * 4);
     L.acc = off; off += up((size_t)(n_alpha + 1) * 8);
-    L.gemv = off; off += M <= 16 ? up(gemv_workspace_bytes((int)N, num_sms)) : 0;
+    L.gemv = off; off += M <= 16 ? gemv_counter_bytes((int)N) + up(gemv_partial_bytes(num_sms)) : 0;
     L.total = off;
     return L;
 }
@@ -286,7 +315,7 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
         return 0;
     DeviceInfo* d = nullptr;
     if (device_info(&d) != W4A16_OK) return 0;
-    return gemv_workspace_bytes((int)N, d->num_sms);
+    return decode_workspace_bytes(M, K, d->num_sms);
 }
 
 w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
@@ -296,8 +325,8 @@ w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16
     w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
     if (st != W4A16_OK) return st;
     if (M > 16) return W4A16_ERR_SHAPE;
-    a.workspace = workspace;
-    a.workspace_bytes = workspace_bytes;
+    st = take_decode_workspace(&a, workspace, workspace_bytes, nullptr);
+    if (st != W4A16_OK) return st;
     return run_gemv(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -309,8 +338,8 @@ w4a16_status w4a16_gemv_ex(const uint16_t* x, const uint32_t* qweight, const uin
     if (st != W4A16_OK) return st;
     if (M > 16) return W4A16_ERR_SHAPE;
     if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
-    a.workspace = workspace;
-    a.workspace_bytes = workspace_bytes;
+    st = take_decode_workspace(&a, workspace, workspace_bytes, nullptr);
+    if (st != W4A16_OK) return st;
     return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);
 }
 
@@ -325,10 +354,17 @@ w4a16_status w4a16_gemv_folded(const uint16_t* x, const float* s, const uint32_t
     if (group_size < 128 || group_size % 128 != 0 || group_size > K || K % group_size != 0) return W4A16_ERR_SHAPE;
     if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
     if (s != nullptr && !aligned(s, 16)) return W4A16_ERR_ALIGN;
-    a.s = s;
     a.group_ratio = (int)(group_size / 128);
-    a.workspace = workspace;
-    a.workspace_bytes = workspace_bytes;
+    uint16_t* xf = nullptr;
+    st = take_decode_workspace(&a, workspace, workspace_bytes, &xf);
+    if (st != W4A16_OK) return st;
+    if (s != nullptr) {
+        // x' = x / s goes to the workspace's fold region, once per call; the GEMV then streams
+        // its weights while the fold runs and reads x' when the fold has finished
+        st = from_cuda(launch_search_fold(x, s, xf, (int)M, (int)K, static_cast<cudaStream_t>(stream)));
+        if (st != W4A16_OK) return st;
+        a.x = xf;
+    }
     return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);
 }
 
@@ -366,10 +402,11 @@ w4a16_status w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint
     LinearArgs a;
     w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
     if (st != W4A16_OK) return st;
-    a.workspace = workspace;
-    a.workspace_bytes = workspace_bytes;
     const bool decode = M <= 16 && K <= gemv_max_k();
-    return decode ? run_gemv(a, static_cast<cudaStream_t>(stream)) : run_gemm(a, static_cast<cudaStream_t>(stream));
+    if (!decode) return run_gemm(a, static_cast<cudaStream_t>(stream));
+    st = take_decode_workspace(&a, workspace, workspace_bytes, nullptr);
+    if (st != W4A16_OK) return st;
+    return run_gemv(a, static_cast<cudaStream_t>(stream));
 }
 
 w4a16_status w4a16_linear_ex(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -382,11 +419,11 @@ w4a16_status w4a16_linear_ex(const uint16_t* x, const uint32_t* qweight, const u
     if (group_size < 128 || group_size % 128 != 0 || group_size > K || K % group_size != 0) return W4A16_ERR_SHAPE;
     if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
     a.group_ratio = (int)(group_size / 128);
-    a.workspace = workspace;
-    a.workspace_bytes = workspace_bytes;
     const bool decode = M <= 16 && K <= gemv_max_k();
-    return decode ? run_gemv(a, static_cast<cudaStream_t>(stream), schedule)
-                  : run_gemm(a, static_cast<cudaStream_t>(stream));
+    if (!decode) return run_gemm(a, static_cast<cudaStream_t>(stream));
+    st = take_decode_workspace(&a, workspace, workspace_bytes, nullptr);
+    if (st != W4A16_OK) return st;
+    return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);
 }
 
 w4a16_status w4a16_gemv_noalloc(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -404,17 +441,12 @@ w4a16_status w4a16_gemv_noalloc(const uint16_t* x, const uint32_t* qweight, cons
     void* scratch = nullptr;
     st = noalloc_scratch(&scratch);
     if (st != W4A16_OK) return st;
-    const size_t need = gemv_workspace_bytes((int)N, d->num_sms);
-    if (need > kNoallocScratchBytes) return W4A16_ERR_UNSUPPORTED;
-    // The row-block counters sit at the end of the workspace and must start at zero.  A
-    // completed call leaves them zero, but one that failed may not have, so clear them.
-    const size_t counter_bytes = (((size_t)(N / 128) * sizeof(unsigned)) + 255) / 256 * 256;
+    // The row-block counters must start at zero.  A completed call leaves them zero, but one
+    // that failed may not have, so clear them.
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + (need - counter_bytes), 0, counter_bytes, s) !=
-        cudaSuccess)
-        return W4A16_ERR_CUDA;
-    a.workspace = scratch;
-    a.workspace_bytes = kNoallocScratchBytes;
+    if (cudaMemsetAsync(scratch, 0, (size_t)(N / 128) * sizeof(unsigned), s) != cudaSuccess) return W4A16_ERR_CUDA;
+    a.counters = static_cast<unsigned*>(scratch);
+    a.partials = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kNoallocCounterBytes);
     return run_gemv(a, s);
 }
 
@@ -495,8 +527,8 @@ w4a16_status awq_search_alpha(const float* W, const float* act_absmean, const ui
         st = validate_linear(xs, qw, sc, z, nullptr, yq, M, N, K, &a);
         if (st != W4A16_OK) break;
         if (M <= 16) {
-            a.workspace = ws + L.gemv;
-            a.workspace_bytes = L.total - L.gemv;
+            a.counters = reinterpret_cast<unsigned*>(ws + L.gemv);
+            a.partials = reinterpret_cast<float*>(ws + L.gemv + gemv_counter_bytes((int)N));
             st = run_gemv(a, s);
         } else {
             st = run_gemm(a, s);

@@ -64,10 +64,6 @@
 //   - Programmatic dependent launch.  The weights may be fetched before the previous kernel
 //     on the stream has finished.  The helpers wait for it before they load x; the
 //     epilogue and the completion phase wait before they touch the workspace or y.
-//   - Optional 1/s fold [AWQ translation, section 3.2: the activations are divided by the
-//     channel scales s].  Given s, the helpers turn every x they load into
-//     x' = bf16(x / s) (IEEE division) before staging it, and the CSR term does the same,
-//     so the result is bit-identical to folding x in a separate pass first.
 #include <atomic>
 #include <mutex>
 
@@ -88,11 +84,9 @@ constexpr int kGemvEpilogue = 13;                               // warp 13
 constexpr int kGemvThreads = 32 * 14;
 constexpr int kGemvHG = kGemvUnitGroups / kGemvHelpers;         // groups per helper and unit
 constexpr int kGemvStages = 4;
-constexpr int kGemvSlotFloats = kGemvRows * 16;                 // one partial tile in the workspace
 
 struct GemvArgs {
     const uint16_t* x;
-    const float* s;      // nullptr, or the AWQ channel scales: the kernel uses x' = bf16(x / s)
     const uint16_t* scales;
     const uint32_t* zeros;
     const int32_t* row_ptr;
@@ -156,21 +150,6 @@ __device__ __forceinline__ uint32_t unit_begin(uint32_t p, uint32_t T, uint32_t 
 // The CTA whose unit range contains unit u: the largest p with floor(p*T/P) <= u.
 __device__ __forceinline__ int cta_of_unit(uint32_t u, uint32_t T, uint32_t P) { return (int)(((u + 1) * P - 1) / T); }
 
-// x' = bf16_rne(float(x) / s) with IEEE division: one bf16 value, and the 8 of a 16-byte load
-// (element e in half e % 2 of word e / 2) against the scales of their 8 channels.
-__device__ __forceinline__ uint16_t fold_bf16(uint16_t x, float s) {
-    return float_to_bf16_bits(__fdiv_rn(bf16_bits_to_float(x), s));
-}
-
-__device__ __forceinline__ uint32_t fold_bf16x2(uint32_t v, float s_lo, float s_hi) {
-    return (uint32_t)fold_bf16((uint16_t)(v & 0xFFFFu), s_lo) | ((uint32_t)fold_bf16((uint16_t)(v >> 16), s_hi) << 16);
-}
-
-__device__ __forceinline__ uint4 fold_bf16x8(uint4 v, float4 s0, float4 s1) {
-    return make_uint4(fold_bf16x2(v.x, s0.x, s0.y), fold_bf16x2(v.y, s0.z, s0.w), fold_bf16x2(v.z, s1.x, s1.y),
-                      fold_bf16x2(v.w, s1.z, s1.w));
-}
-
 // y[m][n] for every token m of channel row n: v[m] + the CSR term of row n, rounded once.
 __device__ __forceinline__ void write_row(const GemvArgs& p, int n, float v[16]) {
     if (p.row_ptr != nullptr) {
@@ -185,15 +164,9 @@ __device__ __forceinline__ void write_row(const GemvArgs& p, int n, float v[16])
                     continue;
                 }
                 const float val = fp16_bits_to_float(p.vals[j]);
-                const float sc = p.s != nullptr ? p.s[c] : 1.0f;
 #pragma unroll
                 for (int m = 0; m < 16; ++m)
-                    if (m < p.M) {
-                        const uint16_t xb = p.x[(size_t)m * p.K + c];
-                        const float xm = p.s != nullptr ? bf16_bits_to_float(fold_bf16(xb, sc))
-                                                        : bf16_bits_to_float(xb);
-                        v[m] = fmaf(val, xm, v[m]);
-                    }
+                    if (m < p.M) v[m] = fmaf(val, bf16_bits_to_float(p.x[(size_t)m * p.K + c]), v[m]);
             }
         }
     }
@@ -379,21 +352,6 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                     for (int w = 0; w < 4; ++w)
                         xv[gg][j][w] = m < p.M ? ldg_cached(p.x + (size_t)m * p.K + ((size_t)g << 7) + 32 * t + 8 * w)
                                                : make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
-            if (p.s != nullptr) {
-                // the 1/s fold on the way in: the same conversions as awq_fold_activations
-#pragma unroll
-                for (int gg = 0; gg < kGemvHG; ++gg) {
-                    const float* sg = p.s + ((size_t)(gb * kGemvUnitGroups + kGemvHG * h + gg) << 7) + 32 * t;
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const float4 s0 = __ldg(reinterpret_cast<const float4*>(sg + 8 * w));
-                        const float4 s1 = __ldg(reinterpret_cast<const float4*>(sg + 8 * w) + 1);
-#pragma unroll
-                        for (int j = 0; j < NT; ++j)
-                            if (8 * j + gq < p.M) xv[gg][j][w] = fold_bf16x8(xv[gg][j][w], s0, s1);
-                    }
                 }
             }
             if (s >= S && !__all_sync(0xffffffffu, mbar_wait_bounded(&xempty[slot], ((s / S) - 1) & 1))) {
@@ -850,11 +808,9 @@ bool gemv_fits(int N, int K, int num_sms) {
     return T * (unsigned long long)gemv_ctas(N, K, num_sms) < (1ull << 32);
 }
 
-size_t gemv_workspace_bytes(int N, int num_sms) {
-    const size_t partials = (size_t)2 * num_sms * kGemvSlotFloats * sizeof(float);
-    const size_t counters = (size_t)(N / kGemvRows) * sizeof(unsigned);
-    return partials + ((counters + 255) / 256) * 256;
-}
+size_t gemv_partial_bytes(int num_sms) { return (size_t)2 * num_sms * kGemvSlotFloats * sizeof(float); }
+
+size_t gemv_counter_bytes(int N) { return ((size_t)(N / kGemvRows) * sizeof(unsigned) + 255) / 256 * 256; }
 
 namespace {
 
@@ -943,13 +899,11 @@ GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule) {
 }
 
 cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
-                        const float* s, const uint16_t* scales, const uint32_t* zeros,
-                        const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
-                        uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
-                        cudaStream_t stream) {
+                        const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
+                        const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, float* partials,
+                        unsigned* counters, int M, int N, int K, unsigned* err, cudaStream_t stream) {
     GemvArgs a{};
     a.x = x;
-    a.s = s;
     a.scales = scales;
     a.zeros = zeros;
     a.row_ptr = row_ptr;
@@ -967,9 +921,8 @@ cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ra
     a.ncl = plan.clusters;
     a.err = err;
     if (plan.ctas < 1 || (plan.cluster != 0 && plan.ctas != plan.cluster * plan.clusters)) return cudaErrorInvalidValue;
-    const size_t partial_bytes = (size_t)2 * num_sms * kGemvSlotFloats * sizeof(float);
-    a.partials = static_cast<float*>(workspace);
-    a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + partial_bytes);
+    a.partials = partials;
+    a.counters = counters;
 
     const bool two = M > 8;
     const int smem = two ? GemvSmem<2>::kBytes : GemvSmem<1>::kBytes;

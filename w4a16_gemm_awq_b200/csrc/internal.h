@@ -34,8 +34,14 @@ int gemv_max_k();
 // Whether the GEMV's 32-bit work-unit arithmetic covers this shape (units x CTAs < 2^32).
 bool gemv_fits(int N, int K, int num_sms);
 
-// Bytes of zero-initialised device workspace the GEMV needs for N output channels.
-size_t gemv_workspace_bytes(int N, int num_sms);
+// One fp32 partial tile of the GEMV's workspace: 128 rows x 16 token columns.
+constexpr int kGemvSlotFloats = 128 * 16;
+
+// Device scratch of the GEMV: fp32 partial tiles (gemv_partial_bytes: two per SM, any
+// contents) and one counter per row block (gemv_counter_bytes, 256-byte padded), which must be
+// zero when a call starts; every call that completes leaves them zero.
+size_t gemv_partial_bytes(int num_sms);
+size_t gemv_counter_bytes(int N);
 
 // A GEMV launch: schedule (W4A16_GEMV_STREAM_K or _CLUSTER), CTAs per cluster (0 for
 // stream-K), clusters and CTAs of the grid.  ctas == 0: the requested schedule cannot run.
@@ -50,12 +56,10 @@ struct GemvPlan {
 GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule);
 
 // group_ratio: the quantization group size / 128 (1 for g128; K / 128 for one group per row).
-// s: nullptr, or [K] channel scales that the kernel divides x by as it loads it.
 cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
-                        const float* s, const uint16_t* scales, const uint32_t* zeros,
-                        const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals, long long nnz,
-                        uint16_t* y, void* workspace, int M, int N, int K, int num_sms, unsigned* err,
-                        cudaStream_t stream);
+                        const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
+                        const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, float* partials,
+                        unsigned* counters, int M, int N, int K, unsigned* err, cudaStream_t stream);
 
 // Dense-and-sparse split of W on the GPU (see outliers.cu).  N * K < 2^32, 1 <= nnz <= N * K.
 size_t split_workspace_bytes(int64_t N);

@@ -51,13 +51,37 @@ search_ref_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, f
     }
 }
 
-// x'[m][k] = bf16(float(x[m][k]) / s[k]), IEEE division then round-to-nearest-even.
+// x'[m][k] = bf16(float(x[m][k]) / s[k]), IEEE division then round-to-nearest-even.  A thread
+// converts 8 consecutive channels with 16-byte loads and stores when K % 8 == 0, else one.
+// The kernel lets the next kernel on the stream start at once (programmatic dependent launch):
+// a GEMV that follows it fetches its weights meanwhile and reads x' only after this grid ends.
 __global__ void search_fold_kernel(const uint16_t* __restrict__ x, const float* __restrict__ s,
                                    uint16_t* __restrict__ xs, int M, int K) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int m = blockIdx.y;  // the grid has exactly M rows of blocks
     if (m >= M) return;
-    for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < K; k += gridDim.x * blockDim.x)
-        xs[(size_t)m * K + k] = float_to_bf16_bits(__fdiv_rn(bf16_bits_to_float(x[(size_t)m * K + k]), s[k]));
+    const uint16_t* xr = x + (size_t)m * K;
+    uint16_t* yr = xs + (size_t)m * K;
+    if ((K & 7) == 0) {
+        for (int k = 8 * (blockIdx.x * blockDim.x + threadIdx.x); k < K; k += 8 * gridDim.x * blockDim.x) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
+            const float4 s0 = *reinterpret_cast<const float4*>(s + k);
+            const float4 s1 = *reinterpret_cast<const float4*>(s + k + 4);
+            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t w = u4_get(v, e);
+                const uint32_t lo = float_to_bf16_bits(__fdiv_rn(bf16_bits_to_float((uint16_t)(w & 0xFFFFu)), sv[2 * e]));
+                const uint32_t hi = float_to_bf16_bits(__fdiv_rn(bf16_bits_to_float((uint16_t)(w >> 16)), sv[2 * e + 1]));
+                o[e] = lo | (hi << 16);
+            }
+            *reinterpret_cast<uint4*>(yr + k) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    } else {
+        for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < K; k += gridDim.x * blockDim.x)
+            yr[k] = float_to_bf16_bits(__fdiv_rn(bf16_bits_to_float(xr[k]), s[k]));
+    }
 }
 
 // acc[0] += sum (y_q - y_ref)^2, and when ref2 is given, *ref2 += sum y_ref^2 (double).
@@ -102,7 +126,8 @@ cudaError_t launch_search_ref(const uint16_t* x, const float* W, float* yref, in
 }
 
 cudaError_t launch_search_fold(const uint16_t* x, const float* s, uint16_t* xs, int M, int K, cudaStream_t stream) {
-    dim3 grid((K + 255) / 256, M);
+    const int per = (K & 7) == 0 ? 8 : 1;  // channels per thread
+    dim3 grid((K + 256 * per - 1) / (256 * per), M);
     search_fold_kernel<<<grid, 256, 0, stream>>>(x, s, xs, M, K);
     return cudaGetLastError();
 }
