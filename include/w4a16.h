@@ -16,8 +16,9 @@
  * Conventions for every entry point
  *   - Tensor arguments are DEVICE pointers, allocated and owned by the caller.  So is
  *     the decode path's workspace (see w4a16_workspace_bytes).  The library keeps no
- *     pointer after a call returns.  It allocates no device memory except one static
- *     device status word per GPU, created when the library is loaded.
+ *     pointer after a call returns.  It allocates no device memory at run time: its only
+ *     device memory is static, part of the loaded module on every GPU that loads it (a
+ *     status word, the scratch of w4a16_gemv_noalloc, the self-test's counters).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
  *     stream).  The return value covers argument validation and the kernel launch.
  *     Problems found while a kernel runs are reported later: the kernel records them in
@@ -345,6 +346,18 @@ w4a16_status awq_fold_activations(const uint16_t* x, const float* s, uint16_t* x
  * counterpart.
  */
 w4a16_status w4a16_selftest_timeout(int64_t limit_ns, void* stream);
+
+/*
+ * w4a16_selftest_quotient -- check, on the current GPU, the division the quantizer uses per
+ * weight (Markstein's correction of the product with the correctly rounded reciprocal of the
+ * group's fp16 scale) against the IEEE division, for every 11-bit divisor significand and
+ * every dividend significand, both signs, over the quotient range that decides a 4-bit code.
+ * Synchronous on `stream`.  *mismatches (host) receives the number of differing quotients,
+ * which must be 0; first (host, may be NULL) the bits of the first difference found: divisor,
+ * dividend, result, IEEE result.  The pages have no counterpart: it is the evidence that the
+ * faster division leaves awq_quantize_g128 bit-exact.
+ */
+w4a16_status w4a16_selftest_quotient(uint64_t* mismatches, uint32_t first[4], void* stream);
 
 /*
  * w4a16_check_device_status -- synchronize `stream` and return the first problem that a

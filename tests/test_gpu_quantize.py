@@ -85,3 +85,12 @@ def test_quantize_full_shapes_bit_exact(orc, cfg, i, K, N):
     """The eight layer shapes (Llama-3-8B and 70B) at full size, packing bit-exact."""
     L = workloads.make_layer(workloads.seed_of(cfg, i), K=K, N=N)
     assert_same(orc, L.W, L.act_absmean, workloads.ALPHA, f"{K}x{N}")
+
+
+def test_quantizer_division_matches_ieee_everywhere():
+    """The quantizer divides each weight by its group's fp16 scale with Markstein's correction
+    of w' * RN(1/sf) instead of an IEEE division.  Over every 11-bit divisor significand and
+    every dividend significand (both signs, quotients 2^-4 .. 2^7: all that can change a
+    4-bit code) the quotient must be the IEEE one, bit for bit."""
+    n, first = w4.selftest_quotient()
+    assert n == 0, f"{n} quotients differ; first: b, a, got, want = {[hex(v) for v in first]}"

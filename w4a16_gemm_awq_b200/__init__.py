@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
         L.w4a16_workspace_bytes.restype = ctypes.c_size_t
         L.w4a16_check_device_status.argtypes = [P]
         L.w4a16_selftest_timeout.argtypes = [I64, P]
+        L.w4a16_selftest_quotient.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint32), P]
         L.awq_split_outliers.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P, ctypes.c_size_t, P]
         L.awq_split_outliers_workspace_bytes.argtypes = [I64, I64]
         L.awq_split_outliers_workspace_bytes.restype = ctypes.c_size_t
@@ -95,7 +96,7 @@ def lib() -> ctypes.CDLL:
         L.w4a16_version.argtypes = []
         for name in ("awq_quantize_g128", "awq_quantize", "w4a16_linear_ex", "w4a16_linear", "w4a16_gemv", "w4a16_gemv_ex", "w4a16_gemv_plan",
                      "w4a16_gemm", "w4a16_check_device_status",
-                     "w4a16_selftest_timeout", "awq_split_outliers", "awq_search_alpha", "awq_fold_activations", "w4a16_version"):
+                     "w4a16_selftest_timeout", "w4a16_selftest_quotient", "awq_split_outliers", "awq_search_alpha", "awq_fold_activations", "w4a16_version"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -318,6 +319,15 @@ def selftest_timeout(limit_ns: int, stream=None) -> None:
     _check(lib().w4a16_selftest_timeout(int(limit_ns), s), "selftest_timeout")
 
 
+def selftest_quotient():
+    """(mismatches, first) of the quantizer's division against the IEEE one on its whole
+    domain (w4a16_selftest_quotient); first = (divisor, dividend, got, want) float bits."""
+    n = ctypes.c_uint64(0)
+    first = (ctypes.c_uint32 * 4)()
+    _check(lib().w4a16_selftest_quotient(ctypes.byref(n), first, _stream(torch.device("cuda"))), "selftest_quotient")
+    return int(n.value), tuple(int(v) for v in first)
+
+
 def status_string(code: int) -> str:
     return lib().w4a16_status_string(code).decode()
 
@@ -361,5 +371,6 @@ w4a16_workspace_bytes = workspace_bytes
 w4a16_gemv_plan = gemv_plan
 w4a16_check_device_status = check_device_status
 w4a16_selftest_timeout = selftest_timeout
+w4a16_selftest_quotient = selftest_quotient
 w4a16_status_string = status_string
 w4a16_version = version

@@ -17,6 +17,10 @@ namespace w4a16 {
 // Problems found by kernels while they run (bit set of kErrValue / kErrShape / kErrTimeout).
 __device__ unsigned g_device_status;
 
+// Result of w4a16_selftest_quotient: mismatch count, then the first mismatch (b, a, got, want).
+__device__ unsigned long long g_quotient_mismatches;
+__device__ unsigned g_quotient_first[4];
+
 // Scratch of w4a16_gemv_noalloc: the decode GEMV's row-block counters for N up to
 // kNoallocMaxN, then its fp32 partial tiles for devices with up to kNoallocMaxSms SMs.  It is
 // part of the loaded module: every GPU that loads the library holds it until the process
@@ -302,7 +306,7 @@ w4a16_status awq_quantize(const float* W, const float* act_absmean, float alpha,
     w4a16_status st = device_info(&d);
     if (st != W4A16_OK) return st;
     return from_cuda(launch_awq_quantize(W, act_absmean, alpha, (int)N, (int)K, (int)group_size, qweight, scales,
-                                         zeros, s_out, d->status, static_cast<cudaStream_t>(stream)));
+                                         zeros, s_out, d->num_sms, d->status, static_cast<cudaStream_t>(stream)));
 }
 
 w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
@@ -519,7 +523,8 @@ w4a16_status awq_search_alpha(const float* W, const float* act_absmean, const ui
     if (M <= 16 && cudaMemsetAsync(ws + L.gemv, 0, L.total - L.gemv, s) != cudaSuccess) return W4A16_ERR_CUDA;
     st = from_cuda(launch_search_ref(x_calib, W, yref, (int)M, (int)N, (int)K, s));
     for (int i = 0; i < n_alpha && st == W4A16_OK; ++i) {
-        st = from_cuda(launch_awq_quantize(W, act_absmean, alphas[i], (int)N, (int)K, 128, qw, sc, z, sv, d->status, s));
+        st = from_cuda(launch_awq_quantize(W, act_absmean, alphas[i], (int)N, (int)K, 128, qw, sc, z, sv, d->num_sms,
+                                           d->status, s));
         if (st != W4A16_OK) break;
         st = from_cuda(launch_search_fold(x_calib, sv, xs, (int)M, (int)K, s));
         if (st != W4A16_OK) break;
@@ -562,6 +567,34 @@ w4a16_status awq_fold_activations(const uint16_t* x, const float* s, uint16_t* x
     w4a16_status st = device_info(&d);
     if (st != W4A16_OK) return st;
     return from_cuda(launch_search_fold(x, s, x_out, (int)M, (int)K, static_cast<cudaStream_t>(stream)));
+}
+
+w4a16_status w4a16_selftest_quotient(uint64_t* mismatches, uint32_t first[4], void* stream) {
+    if (!mismatches) return W4A16_ERR_NULL;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    void* cnt = nullptr;
+    void* fst = nullptr;
+    if (cudaGetSymbolAddress(&cnt, g_quotient_mismatches) != cudaSuccess ||
+        cudaGetSymbolAddress(&fst, g_quotient_first) != cudaSuccess)
+        return W4A16_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned long long host_count = 0;
+    unsigned host_first[4] = {0, 0, 0, 0};
+    if (cudaMemsetAsync(cnt, 0, sizeof(unsigned long long), s) != cudaSuccess ||
+        cudaMemsetAsync(fst, 0, sizeof(host_first), s) != cudaSuccess)
+        return W4A16_ERR_CUDA;
+    st = from_cuda(launch_selftest_quotient(static_cast<unsigned long long*>(cnt), static_cast<unsigned*>(fst), s));
+    if (st != W4A16_OK) return st;
+    if (cudaMemcpyAsync(&host_count, cnt, sizeof(host_count), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(host_first, fst, sizeof(host_first), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return W4A16_ERR_CUDA;
+    *mismatches = host_count;
+    if (first)
+        for (int i = 0; i < 4; ++i) first[i] = host_first[i];
+    return W4A16_OK;
 }
 
 w4a16_status w4a16_selftest_timeout(int64_t limit_ns, void* stream) {

@@ -76,6 +76,19 @@ __device__ __forceinline__ uint32_t u4_get(const uint4& v, int i) {
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
+// ------------------------------------------------------------------ division --------
+
+// RN(a / b) by Markstein's method (P. Markstein, "Computation of elementary functions on the
+// IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990), given y = RN(1 / b), the
+// correctly rounded reciprocal: q0 = RN(a y); e = RN(a - b q0), exact with a fused
+// multiply-add; q1 = RN(q0 + e y).  The quantizer divides by fp16 scales (11 significant
+// bits); w4a16_selftest_quotient checks this against the IEEE division on that whole domain.
+__device__ __forceinline__ float quotient_markstein(float a, float b, float y) {
+    const float q0 = __fmul_rn(a, y);
+    const float e = __fmaf_rn(-b, q0, a);
+    return __fmaf_rn(e, y, q0);
+}
+
 // ------------------------------------------------------------------ bf16 helpers -----
 
 // Two bf16 in one register: (lo - hi) subtraction per half, exact for small integers.

@@ -18,8 +18,8 @@ constexpr int kQuantMaxLargeGroup = 32768;
 bool quantize_group_size_ok(int K, int gs);
 
 cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, int gs,
-                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
-                                cudaStream_t stream);
+                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, int num_sms,
+                                unsigned* err, cudaStream_t stream);
 
 // Tensor map the GEMV needs: qweight uint32 [N][K/8] seen as 3-D (16 words of a group,
 // N rows, K/128 groups; strides K/2 and 64 bytes), box 16 x 128 x 4, no swizzle.  One copy
@@ -76,6 +76,10 @@ cudaError_t launch_search_err(const uint16_t* yq, const float* yref, long long c
 // A kernel whose only wait never completes: it gives up after limit_ns and records
 // kErrTimeout (tests the bounded-wait path without any fault).
 cudaError_t launch_selftest_timeout(unsigned long long limit_ns, unsigned* err, cudaStream_t stream);
+
+// The quantizer's division against the IEEE one on its whole domain (see selftest.cu):
+// mismatches and first[4] (b, a, got, want bits of the first mismatch) must start at zero.
+cudaError_t launch_selftest_quotient(unsigned long long* mismatches, unsigned* first, cudaStream_t stream);
 
 // Tensor maps the GEMM needs, encoded by the caller (api.cu) with the driver's encoder.
 struct GemmMaps {

@@ -5,40 +5,81 @@
 //  README, perplexity table row "W4A16 g128": groups of 128 along K; AWQ translation
 //  section 1: TinyChat's 4-bit packing, 8 codes per 32-bit word.]
 //
-// Work decomposition.  A CTA of 8 warps owns a tile of kRowsPerCta rows x 1024 columns
-// (8 groups).  It first computes the 1024 per-channel scales s_k into
-// shared memory (double pow, as the definition states).  Then each warp quantizes one row
-// of the tile at a time: 32 lanes x 16 bytes is exactly one group of 128 fp32 weights,
-// so the row's 8 groups arrive as 8 coalesced 128-bit loads per lane, all issued before
-// the first group is processed.  The group's min/max is a 5-step warp-shuffle reduction.
-// Each lane quantizes its 4 weights.  Lane pairs (2i, 2i+1) merge their nibbles into
-// packed word i with one shuffle.  The fp16 scales and zero points of the tile are collected
-// in shared memory and written group-major at the end (scales[g][n], zeros[g][n/8] with the
-// nibbles of 8 consecutive rows), so those stores are coalesced too.
+// Work decomposition (groups of up to 1024).  A CTA of 8 warps owns a tile of 64 rows x 1024
+// columns (8 slices of 128); a warp quantizes one row at a time.  Lane l owns the 32
+// consecutive weights l*32 .. l*32+31 of the row's chunk: a quarter of slice l/4.  So a group
+// of 128 R weights belongs to 4 R neighbouring lanes: its min/max takes log2(4 R) shuffle
+// rounds, the group's scale, zero point and reciprocal are computed once per lane for 32
+// weights, and the lane's 32 codes are exactly 4 packed words, stored as one 16-byte store
+// (the warp writes the row's 512 bytes of codes contiguously).  The lane's weights arrive as
+// 8 16-byte loads through L1, where the first brings the warp's lines.  The fp16 scales and
+// zero points of the tile are collected in shared memory and written group-major at the end
+// (scales[g][n], zeros[g][n/8] with the nibbles of 8 consecutive rows), so those stores are
+// coalesced too.
 //
 // Bit-exactness: every float step is a single IEEE operation with round-to-nearest-even
 // (__fmul_rn, __fsub_rn, __fdiv_rn, __fadd_rn, __float2half_rn) or an exact equivalent of
 // one.  The build does not use fast-math or flush-to-zero, so any correct implementation of
 // the same steps gives the same bits.
 //
-// Throughput: the quarter-rate XU pipe (reciprocal, rounding, float-to-integer conversion)
-// is the limiting unit, so only the division stays there.  rint(v) is computed as
-// (v + 1.5 * 2^23) - 1.5 * 2^23 on the FMA pipe: for |v| < 2^22 this is exactly
-// round-to-nearest-even, and larger magnitudes end up clamped to 0 or 15 either way.  The
-// integer code of an integral float c in [0, 15] is the low mantissa bits of c + 2^23.
+// Throughput.  The weights stream once from HBM; the arithmetic per weight is kept to a few
+// FMA-pipe and ALU operations, so that HBM rather than instruction issue is the limit:
+//   - s is computed once per call by a small kernel (double pow, as the definition states)
+//     into s_out, and the quantize kernel, launched so that it may start while that kernel
+//     runs, fetches its first rows of W meanwhile.  Without s_out, every CTA computes the s
+//     of its own 1024 columns.
+//   - The per-weight division w' / sf is Markstein's method (P. Markstein, "Computation of
+//     elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+//     1990): with y = RN(1/sf), the correctly rounded reciprocal, computed once per group,
+//     q0 = RN(w' y), e = RN(w' - sf q0) (exact with an FMA), q1 = RN(q0 + e y).  It gives
+//     q1 = RN(w' / sf), the IEEE quotient, for the divisors that occur here (sf has the 11
+//     significant bits of an fp16); a GPU self-test (w4a16_selftest_quotient) compares it
+//     with the IEEE division on every 11-bit divisor significand and every dividend
+//     significand over the quotient range where rounding decides the code.  Groups whose
+//     quotients could exceed 2^20 in magnitude clamp w' first; their codes saturate either
+//     way.
+//   - rint(q) + z and the integer code come from one add of 1.5 * 2^23 (round to nearest
+//     even, exact for |q| < 2^22) and the float's low bits, clamped as integers.
+//   - The group's minimum and maximum use NaN-propagating min/max, so one finiteness test
+//     per group replaces one per weight.
 #include "common.cuh"
 #include "internal.h"
 
 namespace w4a16 {
 
 constexpr int kQuantThreads = 256;
-constexpr int kRowsPerCta = 64;
 
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr float kIntMagic = 8388608.0f;      // 2^23
 
 // round-to-nearest-even to an integral float; exact for |v| < 2^22 (see above)
 __device__ __forceinline__ float round_rne(float v) { return __fsub_rn(__fadd_rn(v, kRoundMagic), kRoundMagic); }
+
+// rint(v) as an integer, for |v| < 2^22: v + 1.5 * 2^23 lies in [2^23, 2^24), where the float's
+// unit is 1, so the addition rounds v to the nearest integer (ties to even) and the low bits
+// hold 2^22 + rint(v).
+__device__ __forceinline__ int rint_int(float v) {
+    return (int)(__float_as_uint(__fadd_rn(v, kRoundMagic)) - 0x4B400000u);
+}
+
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ float min_nan(float a, float b) {
+    float r;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// The 4-bit code of w' in a group with scale sf (y = RN(1/sf)) and integer zero point z:
+// clamp(rint(w' / sf) + z, 0, 15), for |w' / sf| < 2^21.
+__device__ __forceinline__ uint32_t code_of(float w, float sf, float y, int z) {
+    const int t = rint_int(quotient_markstein(w, sf, y)) + z;
+    return (uint32_t)min(max(t, 0), 15);
+}
 
 // the integer value of an integral float in [0, 2^22)
 __device__ __forceinline__ uint32_t int_bits(float c) { return __float_as_uint(__fadd_rn(c, kIntMagic)) & 0x3FFFFFu; }
@@ -53,94 +94,133 @@ __device__ __forceinline__ uint32_t place_nibbles(const float q[4], bool odd) {
     return (q0 << 8) | (q1 << 24) | (q2 << 12) | (q3 << 28);
 }
 
+// s_k = max(float(pow(double(a_k), double(alpha))), 1e-4), once per call.  The next kernel on
+// the stream (the quantizer) may start at once and fetch its first weights meanwhile.
+__global__ void __launch_bounds__(256) awq_scale_kernel(const float* __restrict__ act, float alpha, int K,
+                                                        float* __restrict__ s, unsigned* err) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int k = blockIdx.x * 256 + threadIdx.x;
+    if (k >= K) return;
+    const float a = act[k];
+    const float p = (float)pow((double)a, (double)alpha);
+    if (!(a >= 0.0f) || isinf(a) || !isfinite(p)) record_error(err, kErrValue);
+    s[k] = p > 1e-4f ? p : 1e-4f;
+}
+
+constexpr int kRowsPerCta = 64;
+
+// Nibble position of element e (0..7) of an 8-wide block: ORDER[pos] = e with
+// ORDER = {0,2,4,6,1,3,5,7}.
+__device__ __forceinline__ constexpr int nibble_of(int e) { return (e & 1) ? 4 + (e >> 1) : (e >> 1); }
+
 // Groups of 128 R weights, R in {1, 2, 4, 8}: a 1024-column chunk holds 8 / R whole groups.
+// s_pre: the channel scales computed by awq_scale_kernel just before (read after it has
+// finished), or nullptr: the CTA computes the s of its columns.
 template <int R>
 __global__ void __launch_bounds__(kQuantThreads)
-awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, float alpha, int N, int K,
-                    uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
-                    uint32_t* __restrict__ zeros, float* __restrict__ s_out, unsigned* err) {
+awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, const float* s_pre, float alpha,
+                    int N, int K, uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
+                    uint32_t* __restrict__ zeros, unsigned* err) {
     constexpr int GC = 8 / R;  // groups per chunk
+    constexpr int LG = 4 * R;  // lanes per group
+    // s of the chunk, lane l's 32 values in 8 16-byte pieces, piece c at l*128 + 16 (c ^ (l & 7)),
+    // so that a quarter warp's 16-byte reads hit 8 different bank groups
     __shared__ __align__(16) float s_sm[1024];
     __shared__ __align__(16) uint16_t sc_sm[GC][kRowsPerCta];  // fp16 scale bits per (group, row)
     __shared__ uint8_t zc_sm[GC][kRowsPerCta];                 // zero point per (group, row)
     const int kc = blockIdx.x;                 // 1024-column chunk (groups GC kc .. GC kc + GC - 1)
     const int row0 = blockIdx.y * kRowsPerCta;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sw = lane & 7;                   // this lane's swizzle
 
-    for (int i = threadIdx.x; i < 1024; i += kQuantThreads) {
-        const float a = act[(size_t)kc * 1024 + i];
-        const float p = (float)pow((double)a, (double)alpha);
-        if (!(a >= 0.0f) || isinf(a) || !isfinite(p)) record_error(err, kErrValue);
-        const float s = p > 1e-4f ? p : 1e-4f;
-        s_sm[i] = s;
-        if (s_out != nullptr && blockIdx.y == 0) s_out[(size_t)kc * 1024 + i] = s;
+    // the warp's first row, fetched before s is available
+    float4 v[8];
+    auto load_row = [&](int n) {
+        const float4* wrow = reinterpret_cast<const float4*>(W + (size_t)n * K + (size_t)kc * 1024 + 32 * lane);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 u = ldg_cached(wrow + c);
+            v[c] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+        }
+    };
+    if (row0 + warp < N) load_row(row0 + warp);
+
+    // thread i places s[4 i .. 4 i + 3]: owner lane i / 8, piece i % 8
+    if (s_pre != nullptr) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");  // s was written by the previous kernel
+        const float4 sv = reinterpret_cast<const float4*>(s_pre + (size_t)kc * 1024)[threadIdx.x];
+        const int ol = threadIdx.x >> 3, c = threadIdx.x & 7;
+        reinterpret_cast<float4*>(s_sm)[ol * 8 + (c ^ (ol & 7))] = sv;
+    } else {
+        float sv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float a = act[(size_t)kc * 1024 + 4 * threadIdx.x + e];
+            const float p = (float)pow((double)a, (double)alpha);
+            if (!(a >= 0.0f) || isinf(a) || !isfinite(p)) record_error(err, kErrValue);
+            sv[e] = p > 1e-4f ? p : 1e-4f;
+        }
+        const int ol = threadIdx.x >> 3, c = threadIdx.x & 7;
+        reinterpret_cast<float4*>(s_sm)[ol * 8 + (c ^ (ol & 7))] = make_float4(sv[0], sv[1], sv[2], sv[3]);
     }
     __syncthreads();
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool odd = lane & 1;
     for (int r = warp; r < kRowsPerCta; r += kQuantThreads / 32) {
         const int n = row0 + r;
         if (n >= N) break;  // warp-uniform
-        const float* wrow = W + (size_t)n * K + (size_t)kc * 1024 + 4 * lane;
-        float4 v[8];
+        if (r != warp) load_row(n);
+        float w[32];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            uint4 u = ldg_stream(wrow + c * 128);
-            v[c] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
-                               __uint_as_float(u.w));
+            const float4 s4 = reinterpret_cast<const float4*>(s_sm)[lane * 8 + (c ^ sw)];  // s of these 4 columns
+            w[4 * c] = __fmul_rn(v[c].x, s4.x);
+            w[4 * c + 1] = __fmul_rn(v[c].y, s4.y);
+            w[4 * c + 2] = __fmul_rn(v[c].z, s4.z);
+            w[4 * c + 3] = __fmul_rn(v[c].w, s4.w);
         }
-        bool bad = false;
+        float mx = w[0], mn = w[0];
 #pragma unroll
-        for (int gi = 0; gi < GC; ++gi) {
-            // the group's R slices of 128: this lane's 4 scaled weights of each
-            float w[R][4];
-            float mx = 0.0f, mn = 0.0f;
-#pragma unroll
-            for (int c = 0; c < R; ++c) {
-                const int sl = gi * R + c;
-                const float4 sv = *reinterpret_cast<const float4*>(&s_sm[sl * 128 + 4 * lane]);
-                w[c][0] = __fmul_rn(v[sl].x, sv.x);
-                w[c][1] = __fmul_rn(v[sl].y, sv.y);
-                w[c][2] = __fmul_rn(v[sl].z, sv.z);
-                w[c][3] = __fmul_rn(v[sl].w, sv.w);
-                if (c == 0) mx = mn = w[0][0];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    bad |= !isfinite(w[c][i]);
-                    mx = fmaxf(mx, w[c][i]);
-                    mn = fminf(mn, w[c][i]);
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            }
-            float scale32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-            if (scale32 < 1e-5f) scale32 = 1e-5f;
-            const __half h = __float2half_rn(scale32);
-            const float sf = __half2float(h);
-            bad |= isinf(scale32) || isinf(sf);
-            float zf = rintf(__fdiv_rn(-mn, sf));
-            zf = fminf(fmaxf(zf, 0.0f), 15.0f);
-#pragma unroll
-            for (int c = 0; c < R; ++c) {
-                float q[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float t = __fadd_rn(round_rne(__fdiv_rn(w[c][i], sf)), zf);
-                    q[i] = fminf(fmaxf(t, 0.0f), 15.0f);
-                }
-                uint32_t part = place_nibbles(q, odd);
-                part |= __shfl_xor_sync(0xffffffffu, part, 1);
-                if (!odd) qweight[(size_t)n * (K >> 3) + (size_t)kc * 128 + (gi * R + c) * 16 + (lane >> 1)] = part;
-            }
-            if (lane == 0) {
-                sc_sm[gi][r] = __half_as_ushort(h);
-                zc_sm[gi][r] = (uint8_t)int_bits(zf);
-            }
+        for (int i = 1; i < 32; ++i) {
+            mx = max_nan(mx, w[i]);
+            mn = min_nan(mn, w[i]);
         }
-        if (bad) record_error(err, kErrValue);
+#pragma unroll
+        for (int o = 1; o < LG; o <<= 1) {
+            mx = max_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            mn = min_nan(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        }
+        const bool bad_range = !isfinite(mx) || !isfinite(mn);  // NaN or Inf anywhere in the group
+        float scale32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+        if (scale32 < 1e-5f) scale32 = 1e-5f;
+        const __half h = __float2half_rn(scale32);
+        const float sf = __half2float(h);
+        const bool bad = bad_range || isinf(scale32) || isinf(sf);
+        float zf = rintf(__fdiv_rn(-mn, sf));
+        zf = fminf(fmaxf(zf, 0.0f), 15.0f);
+        const int zi = (int)int_bits(zf);
+        const float y = __frcp_rn(sf);
+        // |w' / sf| < 2^20 for the whole group: no clamp before dividing
+        const bool small = __fmul_rn(fmaxf(fabsf(mx), fabsf(mn)), y) < 1048576.0f;
+        if (!small) {
+            const float lim = __fmul_rn(sf, 1048576.0f);  // exact: sf times a power of two
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = fminf(fmaxf(w[i], -lim), lim);
+        }
+        uint32_t word[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            uint32_t acc = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc |= code_of(w[8 * b + e], sf, y, zi) << (4 * nibble_of(e));
+            word[b] = acc;
+        }
+        *reinterpret_cast<uint4*>(qweight + (size_t)n * (K >> 3) + (size_t)kc * 128 + 4 * lane) =
+            make_uint4(word[0], word[1], word[2], word[3]);
+        if ((lane & (LG - 1)) == 0) {
+            sc_sm[lane / LG][r] = __half_as_ushort(h);
+            zc_sm[lane / LG][r] = (uint8_t)zi;
+        }
+        if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(err, kErrValue);
     }
     __syncthreads();
 
@@ -154,12 +234,12 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
             *reinterpret_cast<uint32_t*>(scales + ((size_t)kc * GC + g) * N + row0 + r) = pair;
         }
         if (threadIdx.x < 64) {
-            const int gz = threadIdx.x >> 3, w = threadIdx.x & 7;
-            if (gz < GC && row0 + 8 * w < N) {
+            const int gz = threadIdx.x >> 3, w8 = threadIdx.x & 7;
+            if (gz < GC && row0 + 8 * w8 < N) {
                 uint32_t word = 0;
 #pragma unroll
-                for (int b = 0; b < 8; ++b) word |= (uint32_t)(zc_sm[gz][8 * w + b] & 15u) << (4 * b);
-                zeros[((size_t)kc * GC + gz) * (N >> 3) + (row0 >> 3) + w] = word;
+                for (int b = 0; b < 8; ++b) word |= (uint32_t)(zc_sm[gz][8 * w8 + b] & 15u) << (4 * b);
+                zeros[((size_t)kc * GC + gz) * (N >> 3) + (row0 >> 3) + w8] = word;
             }
         }
     }
@@ -270,8 +350,8 @@ bool quantize_group_size_ok(int K, int gs) {
 }
 
 cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, int gs,
-                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, unsigned* err,
-                                cudaStream_t stream) {
+                                uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, int num_sms,
+                                unsigned* err, cudaStream_t stream) {
     if (!quantize_group_size_ok(K, gs)) return cudaErrorInvalidValue;
     if (gs > 1024) {
         const int smem = gs * 4;
@@ -283,13 +363,31 @@ cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, i
                                                                          zeros, s_out, err);
         return cudaGetLastError();
     }
-    dim3 grid(K / 1024, (N + kRowsPerCta - 1) / kRowsPerCta);
     auto* kernel = gs == 128 ? awq_quantize_kernel<1>
                  : gs == 256 ? awq_quantize_kernel<2>
                  : gs == 512 ? awq_quantize_kernel<4>
                              : awq_quantize_kernel<8>;
-    kernel<<<grid, kQuantThreads, 0, stream>>>(W, act, alpha, N, K, qweight, scales, zeros, s_out, err);
-    return cudaGetLastError();
+    const dim3 grid(K / 1024, (N + kRowsPerCta - 1) / kRowsPerCta);
+    (void)num_sms;
+    if (s_out == nullptr) {
+        kernel<<<grid, kQuantThreads, 0, stream>>>(W, act, nullptr, alpha, N, K, qweight, scales, zeros, err);
+        return cudaGetLastError();
+    }
+    // s once into s_out, then the quantizer, which streams its weights while s is computed
+    awq_scale_kernel<<<(K + 255) / 256, 256, 0, stream>>>(act, alpha, K, s_out, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kQuantThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, W, act, (const float*)s_out, alpha, N, K, qweight, scales, zeros, err);
 }
 
 }  // namespace w4a16
