@@ -275,6 +275,43 @@ def build_gemv_workload(torch, w4):
     return calls, quant
 
 
+STEPS_PER_GRAPH = 8
+
+
+def capture_steps(torch, fn, n):
+    """A CUDA graph of n consecutive calls of fn (fn has run eagerly before)."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        for _ in range(n):
+            fn()
+    return g
+
+
+def time_steps(torch, fn, steps, warmup):
+    """ms per call of fn, replayed as graphs of STEPS_PER_GRAPH calls (plus single ones)."""
+    fn()
+    torch.cuda.synchronize()
+    g_many, g_one = capture_steps(torch, fn, STEPS_PER_GRAPH), capture_steps(torch, fn, 1)
+    for _ in range(warmup):
+        g_one.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps // STEPS_PER_GRAPH):
+        g_many.replay()
+    for _ in range(steps % STEPS_PER_GRAPH):
+        g_one.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g_many, g_one
+    return e0.elapsed_time(e1) / steps
+
+
 def time_graph(torch, fn, steps, warmup):
     """Capture fn() once, replay warmup + steps times; CUDA-event ms per replay."""
     fn()
@@ -319,16 +356,12 @@ def run_gpu(args, world, rank, local):
     for _ in range(max(args.warmup, 3)):
         step()
     w4.check_device_status()
-    g = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream()
-    cap.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(cap):
-        step()
-    torch.cuda.current_stream().wait_stream(cap)
-    with torch.cuda.graph(g):
-        step()
+    # Graphs of STEPS_PER_GRAPH steps (and of one step for the remainder), so that the gap
+    # between graph launches is paid once per several steps, as in a decode loop; exactly
+    # args.steps steps run inside the timed region.
+    g_many, g_one = capture_steps(torch, step, STEPS_PER_GRAPH), capture_steps(torch, step, 1)
     for _ in range(args.warmup):
-        g.replay()
+        g_one.replay()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
     stream = torch.cuda.current_stream()
@@ -338,8 +371,10 @@ def run_gpu(args, world, rank, local):
     sampler.start()
     time.sleep(0.3)
     e0.record(stream)
-    for _ in range(args.steps):
-        g.replay()
+    for _ in range(args.steps // STEPS_PER_GRAPH):
+        g_many.replay()
+    for _ in range(args.steps % STEPS_PER_GRAPH):
+        g_one.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -347,7 +382,7 @@ def run_gpu(args, world, rank, local):
     w4.check_device_status()
     ms_local = e0.elapsed_time(e1) / args.steps
     ms, gbs = aggregate(ms_local, step_bytes, world)
-    del g
+    del g_many, g_one
 
     # End to end through the public API with host buffers: the step's activations go from one
     # pinned host buffer to the device in one copy, the 16 GEMVs run, and their outputs come
@@ -373,8 +408,7 @@ def run_gpu(args, world, rank, local):
         hy_all.copy_(dy_all, non_blocking=True)
 
     e2e_steps = max(1, min(args.steps, 2000))
-    ms_e2e, ge = time_graph(torch, e2e_step, e2e_steps, max(args.warmup, 3))
-    del ge
+    ms_e2e = time_steps(torch, e2e_step, e2e_steps, max(args.warmup, 3))
     ms_e2e = reduce_max(ms_e2e, world)
     h2d = dx_all.numel() * 2
     d2h = dy_all.numel() * 2
@@ -402,10 +436,8 @@ def run_gpu(args, world, rank, local):
                 w4.awq_fold_activations(c["x"], s_of[c["K"]], out=xb)
                 w4.w4a16_gemv(xb, qw, sc, z, out=c["y"], workspace=ws)
 
-        ms_f, gf = time_graph(torch, fused_step, 500, 5)
-        del gf
-        ms_s, gs_ = time_graph(torch, separate_step, 500, 5)
-        del gs_
+        ms_f = time_steps(torch, fused_step, 400, 5)
+        ms_s = time_steps(torch, separate_step, 400, 5)
         w4.check_device_status()
         finfo = {"fused": {"value": step_bytes / (ms_f * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_f},
                  "separate": {"value": step_bytes / (ms_s * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_s},
@@ -537,6 +569,10 @@ def run_gpu(args, world, rank, local):
                               "workload": "awq_quantize with group size K on the four Llama-3-8B layers"}}
         del rcalls
 
+    cinfo = None
+    if not args.skip_configs:
+        cinfo = run_configs(torch, w4, pk, pk_kind, quant)
+
     if rank != 0:
         return
     cpu = None
@@ -566,8 +602,145 @@ def run_gpu(args, world, rank, local):
         "alpha_search": ainfo,
         "per_row_groups": rinfo,
         "fold_in_gemv": finfo,
+        "configs": cinfo,
     }
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ the other configs -------
+
+L2_BYTES = 126e6
+
+
+def _copies(nbytes: float) -> int:
+    """Weight copies a timed loop cycles through so that its weights do not stay in L2."""
+    return max(1, int(np.ceil(2.5 * L2_BYTES / nbytes)))
+
+
+def _gpu_layer(torch, seed: int, K: int, N: int):
+    """(W fp32 [N][K], act_absmean [K], mult [K]) on the device: the workloads recipe, with W
+    drawn on the device (N(0, 0.02^2), seeded) for layers too large to draw on the host."""
+    mult, act = workloads.make_act_absmean(seed, K)
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    W = torch.randn(N, K, device="cuda", generator=g) * 0.02
+    return W, torch.from_numpy(act).cuda(), mult
+
+
+def _x(torch, seed: int, M: int, mult):
+    return torch.from_numpy(workloads.make_activations(seed, M, mult).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _rate(nbytes=None, flops=None, ms=None, pk=None, pk_kind=""):
+    out = {"us": round(ms * 1e3, 2)}
+    if nbytes is not None:
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out.update({"GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4)})
+    if flops is not None:
+        tf = flops / (ms * 1e-3) / 1e12
+        out.update({"TFLOP/s": round(tf, 1), "frac_of_bf16": round(tf / pk["bf16_tflops"], 4)})
+    return out
+
+
+def _time_calls(torch, calls, reps=20):
+    """ms per call: the calls in order inside one graph, replayed reps times."""
+    ms = time_steps(torch, lambda: [c() for c in calls], reps, 3)
+    return ms / len(calls)
+
+
+def run_configs(torch, w4, pk, pk_kind, quant8b):
+    """Every workload config besides the headline sweep and the prefill GEMM: the single layer
+    (config 0), the dense-and-sparse 13B layers (config 3), the 70B layers (config 4) and the
+    quantize pass over all eight layers (config 4's C4q).  GEMV timings cycle weight copies
+    (> 2x L2); GEMM timings reuse one copy (compute-bound)."""
+    out = {}
+    # ---- config 0: single layer 4096x4096, M = 1: quantize, then the GEMV
+    L = workloads.make_layer(workloads.seed_of(0, 0), K=4096, N=4096)
+    W, act = torch.from_numpy(L.W).cuda(), torch.from_numpy(L.act_absmean).cuda()
+    ms_q = _time_calls(torch, [lambda: w4.awq_quantize_g128(W, act, workloads.ALPHA)], 10)
+    qw, sc, z, _ = w4.awq_quantize_g128(W, act, workloads.ALPHA)
+    packs = [(qw, sc, z)] + [(qw.clone(), sc.clone(), z.clone()) for _ in range(_copies(workloads.packed_bytes(4096, 4096)) - 1)]
+    x = _x(torch, workloads.seed_of(0, 0), 1, L.mult)
+    y = torch.empty(1, 4096, dtype=torch.bfloat16, device="cuda")
+    ms_g = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p, out=y) for p in packs])
+    out["config0_single_layer"] = {
+        "workload": "4096x4096, M=1: awq_quantize_g128 then w4a16_gemv",
+        "quantize": _rate(nbytes=4096 * 4096 * 4 + workloads.packed_bytes(4096, 4096) + 4096 * 4, ms=ms_q, pk=pk),
+        "gemv": _rate(nbytes=gemv_bytes(4096, 4096, 1), ms=ms_g, pk=pk)}
+    del W, act, packs
+
+    # ---- config 3: dense-and-sparse 13B layers, the CSR term against nnz = 0
+    rows = []
+    for si, (name, K, N) in enumerate(workloads.DENSE_SPARSE_13B["shapes"]):
+        L = workloads.make_layer(workloads.seed_of(3, si), K=K, N=N)
+        W, act = torch.from_numpy(L.W).cuda(), torch.from_numpy(L.act_absmean).cuda()
+        nnz = workloads.outlier_nnz(N, K)
+        Wd, (rp, ci, vals) = w4.awq_split_outliers(W, act, workloads.ALPHA, nnz)
+        qw, sc, z, _ = w4.awq_quantize_g128(Wd, act, workloads.ALPHA)
+        w4.check_device_status()
+        nc = _copies(workloads.packed_bytes(N, K))
+        packs = [(qw, sc, z, (rp, ci, vals))] + [(qw.clone(), sc.clone(), z.clone(), (rp.clone(), ci.clone(), vals.clone()))
+                                                 for _ in range(nc - 1)]
+        csr_bytes = 6 * nnz + 4 * (N + 1)
+        for M in workloads.DENSE_SPARSE_13B["Ms"]:
+            x = _x(torch, workloads.seed_of(3, si), M, L.mult)
+            y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            if M <= 16:
+                ms_c = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p[:3], csr=p[3], out=y) for p in packs])
+                ms_0 = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p[:3], out=y) for p in packs])
+                b0 = gemv_bytes(N, K, M)
+                rows.append({"K": K, "N": N, "M": M, "nnz": nnz, "kernel": "gemv",
+                             "csr": _rate(nbytes=b0 + csr_bytes, ms=ms_c, pk=pk), "no_csr": _rate(nbytes=b0, ms=ms_0, pk=pk),
+                             "csr_cost": round(ms_c / ms_0 - 1.0, 4)})
+            else:
+                p = packs[0]
+                ms_c = _time_calls(torch, [lambda: w4.w4a16_gemm(x, *p[:3], csr=p[3], out=y)])
+                ms_0 = _time_calls(torch, [lambda: w4.w4a16_gemm(x, *p[:3], out=y)])
+                f0 = 2.0 * M * N * K
+                rows.append({"K": K, "N": N, "M": M, "nnz": nnz, "kernel": "gemm",
+                             "csr": _rate(flops=f0 + 2.0 * M * nnz, ms=ms_c, pk=pk), "no_csr": _rate(flops=f0, ms=ms_0, pk=pk),
+                             "csr_cost": round(ms_c / ms_0 - 1.0, 4)})
+        del W, act, Wd, packs
+    out["config3_dense_sparse_13b"] = {"workload": "Llama-2-13B layers with the 0.45% fp16 CSR, M in {1, 16, 1024}",
+                                       "per_call": rows}
+
+    # ---- config 4: 70B layers at M = 1, 64, 4096; the quantize pass over all eight layers
+    rows, qb, qms = [], 0.0, 0.0
+    for W8, act8, N8, K8 in quant8b:
+        qms += _time_calls(torch, [lambda: w4.awq_quantize_g128(W8, act8, workloads.ALPHA)], 5)
+        qb += N8 * K8 * 4 + workloads.packed_bytes(N8, K8) + K8 * 4
+    for si, (name, K, N) in enumerate(workloads.LLAMA2_70B):
+        W, act, mult = _gpu_layer(torch, workloads.seed_of(4, si), K, N)
+        qms += _time_calls(torch, [lambda: w4.awq_quantize_g128(W, act, workloads.ALPHA)], 5)
+        qb += N * K * 4 + workloads.packed_bytes(N, K) + K * 4
+        qw, sc, z, _ = w4.awq_quantize_g128(W, act, workloads.ALPHA)
+        w4.check_device_status()
+        del W
+        nb = workloads.packed_bytes(N, K)
+        packs = [(qw, sc, z)] + [(qw.clone(), sc.clone(), z.clone()) for _ in range(_copies(nb) - 1)]
+        for M in workloads.LARGE_LAYERS_70B["Ms"]:
+            x = _x(torch, workloads.seed_of(4, si), M, mult)
+            y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            if M <= 16:
+                ms = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p, out=y) for p in packs])
+                rows.append({"K": K, "N": N, "M": M, "kernel": "gemv", **_rate(nbytes=gemv_bytes(N, K, M), ms=ms, pk=pk)})
+            else:
+                use = packs if M <= 256 else packs[:1]  # the ridge point streams its weights: cycle copies
+                ms = _time_calls(torch, [lambda p=p: w4.w4a16_linear(x, *p, out=y) for p in use], 10)
+                r = {"K": K, "N": N, "M": M, "kernel": "gemm"}
+                if M <= 256:  # near the ridge: both rooflines
+                    r.update(_rate(nbytes=gemv_bytes(N, K, M), flops=2.0 * M * N * K, ms=ms, pk=pk))
+                else:
+                    r.update(_rate(flops=2.0 * M * N * K, ms=ms, pk=pk))
+                rows.append(r)
+        del packs, qw, sc, z
+    out["config4_large_70b"] = {"workload": "Llama-2-70B layers (W drawn on the device), M in {1, 64, 4096}",
+                                "per_call": rows}
+    out["c4q_quantize_eight_layers"] = {
+        "workload": "awq_quantize_g128 over the four Llama-3-8B and the four Llama-2-70B layers (1.074 G weights)",
+        "value": qb / (qms * 1e-3) / 1e9, "unit": "GB/s", "frac_of_hbm": qb / (qms * 1e-3) / 1e9 / pk["hbm_gbs"],
+        "algorithmic_bytes": qb, "ms": round(qms, 3)}
+    w4.check_device_status()
+    return out
 
 
 GEMV_SOURCE = os.path.join(ROOT, "w4a16_gemm_awq_b200", "csrc", "gemv.cu")
@@ -681,6 +854,7 @@ def main():
     ap.add_argument("--skip-search", action="store_true")
     ap.add_argument("--skip-groups", action="store_true")
     ap.add_argument("--skip-fold", action="store_true")
+    ap.add_argument("--skip-configs", action="store_true")
     ap.add_argument("--case", choices=["gemv", "gemm", "quantize"], help="time one kernel on one layer (ncu)")
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=28672)

@@ -107,17 +107,20 @@ __global__ void __launch_bounds__(256) awq_scale_kernel(const float* __restrict_
     s[k] = p > 1e-4f ? p : 1e-4f;
 }
 
-constexpr int kRowsPerCta = 64;
+// CTAs of the g128 kernel resident per SM (the register budget per thread follows from it).
+#ifndef W4A16_QUANT_CTAS_PER_SM
+#define W4A16_QUANT_CTAS_PER_SM 4
+#endif
 
 // Nibble position of element e (0..7) of an 8-wide block: ORDER[pos] = e with
 // ORDER = {0,2,4,6,1,3,5,7}.
 __device__ __forceinline__ constexpr int nibble_of(int e) { return (e & 1) ? 4 + (e >> 1) : (e >> 1); }
 
 // Groups of 128 R weights, R in {1, 2, 4, 8}: a 1024-column chunk holds 8 / R whole groups.
-// s_pre: the channel scales computed by awq_scale_kernel just before (read after it has
-// finished), or nullptr: the CTA computes the s of its columns.
-template <int R>
-__global__ void __launch_bounds__(kQuantThreads)
+// A CTA takes ROWS (32 or 64) rows.  s_pre: the channel scales computed by awq_scale_kernel
+// just before (read after it has finished), or nullptr: the CTA computes the s of its columns.
+template <int R, int ROWS>
+__global__ void __launch_bounds__(kQuantThreads, W4A16_QUANT_CTAS_PER_SM)
 awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, const float* s_pre, float alpha,
                     int N, int K, uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
                     uint32_t* __restrict__ zeros, unsigned* err) {
@@ -126,21 +129,25 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
     // s of the chunk, lane l's 32 values in 8 16-byte pieces, piece c at l*128 + 16 (c ^ (l & 7)),
     // so that a quarter warp's 16-byte reads hit 8 different bank groups
     __shared__ __align__(16) float s_sm[1024];
-    __shared__ __align__(16) uint16_t sc_sm[GC][kRowsPerCta];  // fp16 scale bits per (group, row)
-    __shared__ uint8_t zc_sm[GC][kRowsPerCta];                 // zero point per (group, row)
+    __shared__ __align__(16) uint16_t sc_sm[GC][ROWS];  // fp16 scale bits per (group, row)
+    __shared__ uint8_t zc_sm[GC][ROWS];                 // zero point per (group, row)
     const int kc = blockIdx.x;                 // 1024-column chunk (groups GC kc .. GC kc + GC - 1)
-    const int row0 = blockIdx.y * kRowsPerCta;
+    const int row0 = blockIdx.y * ROWS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sw = lane & 7;                   // this lane's swizzle
 
-    // the warp's first row, fetched before s is available
-    float4 v[8];
+    // the warp's first row, fetched before s is available; w holds the row's weights, then
+    // the scaled weights in place
+    float w[32];
     auto load_row = [&](int n) {
         const float4* wrow = reinterpret_cast<const float4*>(W + (size_t)n * K + (size_t)kc * 1024 + 32 * lane);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const uint4 u = ldg_cached(wrow + c);
-            v[c] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+            w[4 * c] = __uint_as_float(u.x);
+            w[4 * c + 1] = __uint_as_float(u.y);
+            w[4 * c + 2] = __uint_as_float(u.z);
+            w[4 * c + 3] = __uint_as_float(u.w);
         }
     };
     if (row0 + warp < N) load_row(row0 + warp);
@@ -165,18 +172,17 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
     }
     __syncthreads();
 
-    for (int r = warp; r < kRowsPerCta; r += kQuantThreads / 32) {
+    for (int r = warp; r < ROWS; r += kQuantThreads / 32) {
         const int n = row0 + r;
         if (n >= N) break;  // warp-uniform
         if (r != warp) load_row(n);
-        float w[32];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const float4 s4 = reinterpret_cast<const float4*>(s_sm)[lane * 8 + (c ^ sw)];  // s of these 4 columns
-            w[4 * c] = __fmul_rn(v[c].x, s4.x);
-            w[4 * c + 1] = __fmul_rn(v[c].y, s4.y);
-            w[4 * c + 2] = __fmul_rn(v[c].z, s4.z);
-            w[4 * c + 3] = __fmul_rn(v[c].w, s4.w);
+            w[4 * c] = __fmul_rn(w[4 * c], s4.x);
+            w[4 * c + 1] = __fmul_rn(w[4 * c + 1], s4.y);
+            w[4 * c + 2] = __fmul_rn(w[4 * c + 2], s4.z);
+            w[4 * c + 3] = __fmul_rn(w[4 * c + 3], s4.w);
         }
         float mx = w[0], mn = w[0];
 #pragma unroll
@@ -229,12 +235,12 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
     {
         const int g = threadIdx.x >> 5, j = threadIdx.x & 31;  // up to 8 groups x 32 row pairs
         const int r = 2 * j;
-        if (g < GC && row0 + r < N) {
+        if (g < GC && r < ROWS && row0 + r < N) {
             const uint32_t pair = (uint32_t)sc_sm[g][r] | ((uint32_t)sc_sm[g][r + 1] << 16);
             *reinterpret_cast<uint32_t*>(scales + ((size_t)kc * GC + g) * N + row0 + r) = pair;
         }
-        if (threadIdx.x < 64) {
-            const int gz = threadIdx.x >> 3, w8 = threadIdx.x & 7;
+        if (threadIdx.x < 8 * (ROWS / 8)) {
+            const int gz = threadIdx.x / (ROWS / 8), w8 = threadIdx.x % (ROWS / 8);
             if (gz < GC && row0 + 8 * w8 < N) {
                 uint32_t word = 0;
 #pragma unroll
@@ -363,12 +369,14 @@ cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, i
                                                                          zeros, s_out, err);
         return cudaGetLastError();
     }
-    auto* kernel = gs == 128 ? awq_quantize_kernel<1>
-                 : gs == 256 ? awq_quantize_kernel<2>
-                 : gs == 512 ? awq_quantize_kernel<4>
-                             : awq_quantize_kernel<8>;
-    const dim3 grid(K / 1024, (N + kRowsPerCta - 1) / kRowsPerCta);
-    (void)num_sms;
+    // 64-row tiles, or 32-row ones when 64-row tiles would not fill the resident CTA slots twice
+    const bool small = (long long)(K / 1024) * ((N + 63) / 64) < 2LL * W4A16_QUANT_CTAS_PER_SM * num_sms;
+    const int rows = small ? 32 : 64;
+    auto* kernel = small ? (gs == 128 ? awq_quantize_kernel<1, 32> : gs == 256 ? awq_quantize_kernel<2, 32>
+                            : gs == 512 ? awq_quantize_kernel<4, 32> : awq_quantize_kernel<8, 32>)
+                         : (gs == 128 ? awq_quantize_kernel<1, 64> : gs == 256 ? awq_quantize_kernel<2, 64>
+                            : gs == 512 ? awq_quantize_kernel<4, 64> : awq_quantize_kernel<8, 64>);
+    const dim3 grid(K / 1024, (N + rows - 1) / rows);
     if (s_out == nullptr) {
         kernel<<<grid, kQuantThreads, 0, stream>>>(W, act, nullptr, alpha, N, K, qweight, scales, zeros, err);
         return cudaGetLastError();

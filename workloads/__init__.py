@@ -88,6 +88,22 @@ def make_layer(seed: int, K: int, N: int, calib_rows: int = CALIB_ROWS) -> Layer
     return Layer(K=K, N=N, W=W, mult=mult.astype(np.float32), act_absmean=act, seed=seed)
 
 
+def make_act_absmean(seed: int, K: int, calib_rows: int = CALIB_ROWS):
+    """(mult, act_absmean) of make_layer(seed, K, N) without drawing W (for layers too large to
+    draw on the host; the same substreams, so the values equal make_layer's)."""
+    _, rm, ro, rc, _ = _streams(seed)
+    mult = np.exp(rm.standard_normal(K)).astype(np.float64)
+    idx = ro.choice(K, size=min(N_OUTLIER_CHANNELS, K), replace=False)
+    mult[idx] *= OUTLIER_CHANNEL_GAIN
+    acc = np.zeros(K, np.float64)
+    done = 0
+    while done < calib_rows:
+        r = min(64, calib_rows - done)
+        acc += np.abs(rc.standard_normal((r, K)) * mult).sum(axis=0)
+        done += r
+    return mult.astype(np.float32), (acc / calib_rows).astype(np.float32)
+
+
 def _f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round fp32 to bf16 (nearest-even) via torch's conversion; returns uint16 bits."""
     import torch
