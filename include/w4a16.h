@@ -134,8 +134,8 @@ w4a16_status awq_quantize(const float* W, const float* act_absmean, float alpha,
  *   - After a call reports W4A16_ERR_TIMEOUT, zero the workspace again before reusing it.
  * w4a16_workspace_bytes returns the size for the CURRENT device (it depends on the number
  * of SMs), or 0 when the call with these sizes needs no workspace (M > 16) or the sizes
- * are invalid.  It is 128 KiB of counters, 16 KiB of partial tiles per SM, and M x K bf16
- * for the folded activations (rounded up to 256 bytes); it does not depend on N.
+ * are invalid.  It is 128 KiB of counters, 16 KiB of partial tiles per SM, M x K bf16 for
+ * the folded activations and N x M fp32 for the CSR term (each rounded up to 256 bytes).
  */
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -150,6 +150,9 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   y        [M][N] bf16 bits, device, output.  It must not overlap any input.
  *   workspace, workspace_bytes: see above.  Required when M <= 16; ignored otherwise.
  *   M >= 1.  M <= 16 runs the decode GEMV; larger M runs the tensor-core GEMM.
+ *   Decode path with a CSR: a small kernel first writes the sparse term x . W_sparse^T in
+ *   fp32 to the workspace (fp16 values times bf16 activations, fp32 sums), while the GEMV
+ *   already streams its weights; the GEMV adds it to each output before the one rounding.
  *   Errors: NULL, SHAPE, ALIGN and UNSUPPORTED when called (SHAPE also for a workspace that
  *   is too small).  Later: SHAPE if a CSR index is out of range (that entry is skipped),
  *   TIMEOUT if a pipeline wait runs out.
@@ -257,7 +260,8 @@ w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16
  * callback, where calling cudaMalloc would re-enter the allocator.
  *   - Arguments, result and limits are those of w4a16_gemv, minus the workspace.
  *     N <= 131072 and at most 160 SMs on the device; otherwise W4A16_ERR_UNSUPPORTED.
- *   - Its scratch is a static device array of about 5 MiB inside the library.  Every GPU
+ *   - With a CSR term, N x M <= 262144 as well (UNSUPPORTED otherwise).
+ *   - Its scratch is a static device array of about 3.6 MiB inside the library.  Every GPU
  *     that loads the library holds one until the process exits.  The call allocates
  *     nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - The first call on a device looks up the array's device address

@@ -28,8 +28,9 @@ __device__ unsigned g_quotient_first[4];
 constexpr int kNoallocMaxSms = 160;
 constexpr int kNoallocMaxN = 131072;
 constexpr size_t kNoallocCounterBytes = (size_t)(kNoallocMaxN / 128) * sizeof(unsigned);
-constexpr size_t kNoallocScratchBytes =
-    kNoallocCounterBytes + (size_t)2 * kNoallocMaxSms * kGemvSlotFloats * sizeof(float);
+constexpr size_t kNoallocCsrMax = 262144;  // N x M of a call with a CSR term
+constexpr size_t kNoallocPartialBytes = (size_t)2 * kNoallocMaxSms * kGemvSlotFloats * sizeof(float);
+constexpr size_t kNoallocScratchBytes = kNoallocCounterBytes + kNoallocPartialBytes + kNoallocCsrMax * sizeof(float);
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 namespace {
@@ -127,6 +128,7 @@ struct LinearArgs {
     int group_ratio = 1;  // group size / 128
     float* partials = nullptr;   // the GEMV's scratch (gemv_partial_bytes)
     unsigned* counters = nullptr;  // zero when the call starts (gemv_counter_bytes)
+    float* ysp = nullptr;          // the GEMV's CSR term, [N][M] fp32 (only with a CSR)
 };
 
 w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -188,21 +190,31 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4A16_ERR_CUDA;
     }
-    return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals,
-                                 a.nnz, a.y, a.partials, a.counters, (int)a.M, (int)a.N, (int)a.K, d->status,
-                                 stream));
+    const float* ysp = nullptr;
+    if (a.row_ptr != nullptr) {
+        // the sparse term first, into the workspace; the GEMV streams its weights meanwhile
+        if (a.ysp == nullptr) return W4A16_ERR_NULL;
+        st = from_cuda(launch_csr_rows(a.x, a.row_ptr, a.col_idx, a.vals, a.nnz, (int)a.M, (int)a.N, (int)a.K, a.ysp,
+                                       d->status, stream));
+        if (st != W4A16_OK) return st;
+        ysp = a.ysp;
+    }
+    return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.scales, a.zeros, ysp, a.y, a.partials,
+                                 a.counters, (int)a.M, (int)a.N, (int)a.K, d->status, stream));
 }
 
 // The decode workspace of the public entry points:
 //   [0, kCounterRegionBytes)   the GEMV's row-block counters (zero between calls);
 //   then gemv_partial_bytes    its fp32 partial tiles;
-//   then M x K bf16            x / s of w4a16_gemv_folded, rounded up to 256 bytes.
-// Only the last part depends on the call's sizes, and it lies after everything else, so one
-// zeroed workspace serves calls of any sizes in stream order.
+//   then M x K bf16            x / s of w4a16_gemv_folded, rounded up to 256 bytes;
+//   then N x M fp32            the CSR term, rounded up to 256 bytes.
+// Only the last two parts depend on the call's sizes, and they lie after everything that must
+// stay zero, so one zeroed workspace serves calls of any sizes in stream order.
 size_t fold_region_bytes(int64_t M, int64_t K) { return ((size_t)M * (size_t)K * 2 + 255) / 256 * 256; }
+size_t csr_region_bytes(int64_t M, int64_t N) { return ((size_t)M * (size_t)N * 4 + 255) / 256 * 256; }
 
-size_t decode_workspace_bytes(int64_t M, int64_t K, int num_sms) {
-    return kCounterRegionBytes + gemv_partial_bytes(num_sms) + fold_region_bytes(M, K);
+size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+    return kCounterRegionBytes + gemv_partial_bytes(num_sms) + fold_region_bytes(M, K) + csr_region_bytes(M, N);
 }
 
 // Checks the caller's decode workspace and points a at its parts; *fold = the x / s region.
@@ -212,11 +224,13 @@ w4a16_status take_decode_workspace(LinearArgs* a, void* workspace, size_t worksp
     if (st != W4A16_OK) return st;
     if (workspace == nullptr) return W4A16_ERR_NULL;
     if (!aligned(workspace, 16)) return W4A16_ERR_ALIGN;
-    if (workspace_bytes < decode_workspace_bytes(a->M, a->K, d->num_sms)) return W4A16_ERR_SHAPE;
+    if (workspace_bytes < decode_workspace_bytes(a->M, a->N, a->K, d->num_sms)) return W4A16_ERR_SHAPE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const size_t fold_off = kCounterRegionBytes + gemv_partial_bytes(d->num_sms);
     a->counters = reinterpret_cast<unsigned*>(ws);
     a->partials = reinterpret_cast<float*>(ws + kCounterRegionBytes);
-    if (fold) *fold = reinterpret_cast<uint16_t*>(ws + kCounterRegionBytes + gemv_partial_bytes(d->num_sms));
+    if (fold) *fold = reinterpret_cast<uint16_t*>(ws + fold_off);
+    a->ysp = reinterpret_cast<float*>(ws + fold_off + fold_region_bytes(a->M, a->K));
     return W4A16_OK;
 }
 
@@ -319,7 +333,7 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
         return 0;
     DeviceInfo* d = nullptr;
     if (device_info(&d) != W4A16_OK) return 0;
-    return decode_workspace_bytes(M, K, d->num_sms);
+    return decode_workspace_bytes(M, N, K, d->num_sms);
 }
 
 w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
@@ -438,6 +452,7 @@ w4a16_status w4a16_gemv_noalloc(const uint16_t* x, const uint32_t* qweight, cons
     if (st != W4A16_OK) return st;
     if (M > 16) return W4A16_ERR_SHAPE;
     if (N > kNoallocMaxN) return W4A16_ERR_UNSUPPORTED;
+    if (a.row_ptr != nullptr && (size_t)(N * M) > kNoallocCsrMax) return W4A16_ERR_UNSUPPORTED;
     DeviceInfo* d = nullptr;
     st = device_info(&d);
     if (st != W4A16_OK) return st;
@@ -451,6 +466,7 @@ w4a16_status w4a16_gemv_noalloc(const uint16_t* x, const uint32_t* qweight, cons
     if (cudaMemsetAsync(scratch, 0, (size_t)(N / 128) * sizeof(unsigned), s) != cudaSuccess) return W4A16_ERR_CUDA;
     a.counters = static_cast<unsigned*>(scratch);
     a.partials = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kNoallocCounterBytes);
+    a.ysp = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kNoallocCounterBytes + kNoallocPartialBytes);
     return run_gemv(a, s);
 }
 

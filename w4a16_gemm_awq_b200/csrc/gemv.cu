@@ -89,10 +89,7 @@ struct GemvArgs {
     const uint16_t* x;
     const uint16_t* scales;
     const uint32_t* zeros;
-    const int32_t* row_ptr;
-    const int32_t* col_idx;
-    const uint16_t* vals;
-    long long nnz;
+    const float* ysp;    // nullptr, or the CSR term [N][M] fp32 (csr_rows_kernel, the previous kernel)
     uint16_t* y;
     float* partials;     // workspace: [2P][128][16] fp32 (stream-K)
     unsigned* counters;  // workspace: [N/128], zero between calls (stream-K)
@@ -150,25 +147,15 @@ __device__ __forceinline__ uint32_t unit_begin(uint32_t p, uint32_t T, uint32_t 
 // The CTA whose unit range contains unit u: the largest p with floor(p*T/P) <= u.
 __device__ __forceinline__ int cta_of_unit(uint32_t u, uint32_t T, uint32_t P) { return (int)(((u + 1) * P - 1) / T); }
 
-// y[m][n] for every token m of channel row n: v[m] + the CSR term of row n, rounded once.
-__device__ __forceinline__ void write_row(const GemvArgs& p, int n, float v[16]) {
-    if (p.row_ptr != nullptr) {
-        const int j0 = p.row_ptr[n], j1 = p.row_ptr[n + 1];
-        if (j0 < 0 || j1 < j0 || (long long)j1 > p.nnz) {
-            record_error(p.err, kErrShape);
-        } else {
-            for (int j = j0; j < j1; ++j) {
-                const int c = p.col_idx[j];
-                if ((unsigned)c >= (unsigned)p.K) {
-                    record_error(p.err, kErrShape);
-                    continue;
-                }
-                const float val = fp16_bits_to_float(p.vals[j]);
+// y[m][n] for every token m of channel row n: v[m] + the CSR term of row n (computed by
+// csr_rows_kernel into ysp[n][m] before this kernel reads it), rounded once.
+__device__ __forceinline__ void write_row(const GemvArgs& p, int n, const float v[16]) {
+    if (p.ysp != nullptr) {
+        const float* sp = p.ysp + (size_t)n * p.M;
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    if (m < p.M) v[m] = fmaf(val, bf16_bits_to_float(p.x[(size_t)m * p.K + c]), v[m]);
-            }
-        }
+        for (int m = 0; m < 16; ++m)
+            if (m < p.M) p.y[(size_t)m * p.N + n] = float_to_bf16_bits(v[m] + __ldcg(sp + m));
+        return;
     }
 #pragma unroll
     for (int m = 0; m < 16; ++m)
@@ -899,17 +886,14 @@ GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule) {
 }
 
 cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
-                        const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
-                        const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, float* partials,
-                        unsigned* counters, int M, int N, int K, unsigned* err, cudaStream_t stream) {
+                        const uint16_t* scales, const uint32_t* zeros, const float* ysp, uint16_t* y,
+                        float* partials, unsigned* counters, int M, int N, int K, unsigned* err,
+                        cudaStream_t stream) {
     GemvArgs a{};
     a.x = x;
     a.scales = scales;
     a.zeros = zeros;
-    a.row_ptr = row_ptr;
-    a.col_idx = col_idx;
-    a.vals = vals;
-    a.nnz = nnz;
+    a.ysp = ysp;
     a.y = y;
     a.M = M;
     a.N = N;

@@ -56,10 +56,18 @@ struct GemvPlan {
 GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule);
 
 // group_ratio: the quantization group size / 128 (1 for g128; K / 128 for one group per row).
+// ysp: nullptr, or the CSR term [N][M] fp32 written by launch_csr_rows just before (the GEMV
+// adds it to each output before rounding, after the previous kernel has finished).
 cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
-                        const uint16_t* scales, const uint32_t* zeros, const int32_t* row_ptr,
-                        const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, float* partials,
-                        unsigned* counters, int M, int N, int K, unsigned* err, cudaStream_t stream);
+                        const uint16_t* scales, const uint32_t* zeros, const float* ysp, uint16_t* y,
+                        float* partials, unsigned* counters, int M, int N, int K, unsigned* err,
+                        cudaStream_t stream);
+
+// The CSR term of the decode path: ysp[n][m] = sum_j float(val_j) * float(x[m][col_j]) over
+// row n's entries, in fp32 (see csr.cu).  1 <= M <= 16.  The next kernel on the stream may
+// start while it runs (programmatic dependent launch) and must wait for it before reading ysp.
+cudaError_t launch_csr_rows(const uint16_t* x, const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals,
+                            long long nnz, int M, int N, int K, float* ysp, unsigned* err, cudaStream_t stream);
 
 // Dense-and-sparse split of W on the GPU (see outliers.cu).  N * K < 2^32, 1 <= nnz <= N * K.
 size_t split_workspace_bytes(int64_t N);
