@@ -265,7 +265,9 @@ w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16
  *     that loads the library holds one until the process exits.  The call allocates
  *     nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress).  Make that first call before any stream capture.
+ *     (cudaGetSymbolAddress); the first call with M <= 8 and the first with M > 8 also
+ *     cache the device's properties, the driver's tensor-map encoder and the occupancy of
+ *     that kernel instance.  Make one call of each kind before any stream capture.
  *   - Each call clears the scratch's counters with cudaMemsetAsync on `stream`, and then
  *     runs the GEMV.
  *   - All calls on a device share the one array, which keeps the last call's contents.

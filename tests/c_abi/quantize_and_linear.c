@@ -1,6 +1,8 @@
 /*
  * A plain C99 user of libw4a16: quantize a seeded 4096 x 1024 layer on the GPU, fold 1/s
- * into 4 tokens of activations, run the W4A16 linear and check the device status.
+ * into 4 tokens of activations, run the W4A16 linear and check the device status.  Given a
+ * directory argument, it also writes its inputs and output there as raw little-endian files
+ * (W.f32 [N][K], act.f32 [K], x.bf16 [M][K], y.bf16 [M][N]) for a checker to compare.
  *
  * The tests compile and link it on any machine (the header must be valid C and every
  * entry point it uses must resolve); run it on an sm_100 GPU to see the library work:
@@ -50,7 +52,22 @@ static float from_bf16(uint16_t h) {
     return f;
 }
 
-int main(void) {
+static int dump(const char* dir, const char* name, const void* data, size_t bytes) {
+    char path[4096];
+    FILE* f;
+    size_t w;
+    if (snprintf(path, sizeof path, "%s/%s", dir, name) >= (int)sizeof path) return 0;
+    f = fopen(path, "wb");
+    if (!f) {
+        fprintf(stderr, "cannot write %s\n", path);
+        return 0;
+    }
+    w = fwrite(data, 1, bytes, f);
+    fclose(f);
+    return w == bytes;
+}
+
+int main(int argc, char** argv) {
     const size_t nw = (size_t)N_OUT * K_IN, nx = (size_t)M_TOK * K_IN, ny = (size_t)M_TOK * N_OUT;
     const size_t groups = K_IN / 128;
     float* hW = malloc(nw * sizeof(float));
@@ -91,6 +108,9 @@ int main(void) {
                       "w4a16_linear");
     ok = ok && lib_ok(w4a16_check_device_status(NULL), "device status");
     ok = ok && cuda_ok(cudaMemcpy(hy, dy, ny * sizeof(uint16_t), cudaMemcpyDeviceToHost), "copy y");
+    if (ok && argc > 1)
+        ok = dump(argv[1], "W.f32", hW, nw * sizeof(float)) && dump(argv[1], "act.f32", ha, K_IN * sizeof(float)) &&
+             dump(argv[1], "x.bf16", hx, nx * sizeof(uint16_t)) && dump(argv[1], "y.bf16", hy, ny * sizeof(uint16_t));
     if (ok)
         printf("y[0][0..3] = %g %g %g %g\nok\n", from_bf16(hy[0]), from_bf16(hy[1]), from_bf16(hy[2]),
                from_bf16(hy[3]));

@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import w4a16_gemm_awq_b200 as w4
 
@@ -190,3 +191,27 @@ def test_binding_has_every_entry_point_by_name():
     assert w4.awq_split_outliers_workspace_bytes(256, 1024) == want
     assert w4.w4a16_version() == w4.version()
     assert w4.w4a16_status_string(w4.ERR_SHAPE) == w4.status_string(w4.ERR_SHAPE)
+
+
+def test_linear_shape_checks_before_any_launch():
+    """Mismatched operands are refused by the binding with ValueError (CPU tensors suffice:
+    the shapes are checked before the device)."""
+    M, N, K = 3, 256, 2048
+    x = torch.zeros(M, K, dtype=torch.bfloat16)
+    qw = torch.zeros(N, K // 8, dtype=torch.int32)
+    sc = torch.zeros(K // 128, N, dtype=torch.int16)
+    z = torch.zeros(K // 128, N // 8, dtype=torch.int32)
+    w4.check_linear_shapes(x, qw, sc, z)
+    bad = [
+        (x, qw[:, :-1], sc, z, None, None),                    # qweight too short for K
+        (x, qw, sc[:, :-8], z, None, None),                    # scales for fewer rows
+        (x, qw, sc, z[:-1], None, None),                       # zeros for fewer groups
+        (x, qw, sc, z, (torch.zeros(N, dtype=torch.int32), None, None), None),  # row_ptr of N entries
+        (x, qw, sc, z, None, torch.zeros(M, N - 128, dtype=torch.bfloat16)),    # out of the wrong shape
+    ]
+    for args in bad:
+        with pytest.raises(ValueError):
+            w4.check_linear_shapes(*args)
+    for fn in (w4.w4a16_gemv_noalloc, w4.w4a16_gemv):
+        with pytest.raises(ValueError):
+            fn(x, qw[:, :-1], sc, z)

@@ -121,6 +121,32 @@ def _need(t, dtype, ndim, name):
                          f"{t.dtype} {tuple(t.shape)} on {t.device}")
 
 
+def check_linear_shapes(x, qweight, scales, zeros, csr=None, out=None, group_size: int = 128):
+    """Raise ValueError unless the operands of a linear call agree: x [M][K], qweight [N][K/8],
+    scales [K/gs][N], zeros [K/gs][N/8], csr row_ptr [N+1], out [M][N] bf16.  Shapes only, so
+    a mismatch is reported before anything reaches the library."""
+    if x.dim() != 2 or qweight.dim() != 2:
+        raise ValueError("x and qweight must be matrices")
+    M, K = x.shape
+    N = qweight.shape[0]
+    gs = int(group_size)
+    if qweight.shape[1] * 8 != K:
+        raise ValueError(f"qweight {tuple(qweight.shape)} does not match K = {K}")
+    if gs < 1 or K % gs != 0:
+        raise ValueError(f"group size {gs} does not divide K = {K}")
+    if tuple(scales.shape) != (K // gs, N):
+        raise ValueError(f"scales {tuple(scales.shape)}: expected ({K // gs}, {N})")
+    if tuple(zeros.shape) != (K // gs, N // 8):
+        raise ValueError(f"zeros {tuple(zeros.shape)}: expected ({K // gs}, {N // 8})")
+    if csr is not None and csr[0].numel() != N + 1:
+        raise ValueError(f"CSR row_ptr has {csr[0].numel()} entries, expected N + 1 = {N + 1}")
+    if out is not None:
+        if tuple(out.shape) != (M, N) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+            raise ValueError(f"out: expected a contiguous bf16 ({M}, {N}) tensor, got {out.dtype} {tuple(out.shape)}")
+        if out.device != x.device:
+            raise ValueError("out is on another device than x")
+
+
 def awq_quantize(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, group_size: int, out=None):
     """awq_quantize_g128 with groups of group_size along K -> (qweight int32 [N][K/8],
     scales int16 [K/gs][N], zeros int32 [K/gs][N/8], s fp32 [K])."""
@@ -183,6 +209,7 @@ def workspace_bytes(M: int, N: int, K: int) -> int:
 
 def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, schedule=None, group_size=None,
             fold=False, s=None):
+    check_linear_shapes(x, qweight, scales, zeros, csr, out, 128 if group_size is None else group_size)
     _need(x, torch.bfloat16, 2, "x")
     if s is not None:
         _need(s, torch.float32, 1, "s")
@@ -340,6 +367,7 @@ def version() -> int:
 
 def w4a16_gemv_noalloc(x, qweight, scales, zeros, csr=None, out=None):
     """The decode GEMV without a caller workspace (the library's static scratch)."""
+    check_linear_shapes(x, qweight, scales, zeros, csr, out)
     _need(x, torch.bfloat16, 2, "x")
     _need(qweight, torch.int32, 2, "qweight")
     _need(scales, torch.int16, 2, "scales")
