@@ -450,13 +450,16 @@ def run_gpu(args, world, rank, local):
     if not args.skip_gemm:
         flops, t_ms = 0.0, 0.0
         per = []
+        # one zeroed workspace for the split-K partial tiles and counters of every call
+        wsg = torch.zeros(max(w4.workspace_bytes(M, c["N"], c["K"], csr=False) for c in calls for M in GEMM_MS),
+                          dtype=torch.uint8, device="cuda")
         for ci in range(0, len(calls), len(GEMV_MS)):
             c = calls[ci]
             qw, sc, z = c["w"]
             for M in GEMM_MS:
                 x = torch.randn(M, c["K"], device="cuda").to(torch.bfloat16)
                 y = torch.empty(M, c["N"], dtype=torch.bfloat16, device="cuda")
-                ms1, gg = time_graph(torch, lambda: w4.w4a16_gemm(x, qw, sc, z, out=y), 20, 3)
+                ms1, gg = time_graph(torch, lambda: w4.w4a16_gemm(x, qw, sc, z, out=y, workspace=wsg), 20, 3)
                 del gg
                 f = 2.0 * M * c["N"] * c["K"]
                 flops += f
@@ -653,6 +656,14 @@ def run_configs(torch, w4, pk, pk_kind, quant8b):
     quantize pass over all eight layers (config 4's C4q).  GEMV timings cycle weight copies
     (> 2x L2); GEMM timings reuse one copy (compute-bound)."""
     out = {}
+    # one zeroed workspace, created before any graph capture, for every call below (each call
+    # leaves its counters zero): the largest need of configs 0, 3 and 4
+    need = [w4.workspace_bytes(1, 4096, 4096)]
+    need += [w4.workspace_bytes(M, N, K) for _, K, N in workloads.DENSE_SPARSE_13B["shapes"]
+             for M in workloads.DENSE_SPARSE_13B["Ms"]]
+    need += [w4.workspace_bytes(M, N, K, csr=False) for _, K, N in workloads.LLAMA2_70B
+             for M in workloads.LARGE_LAYERS_70B["Ms"]]
+    ws = torch.zeros(max(need), dtype=torch.uint8, device="cuda")
     # ---- config 0: single layer 4096x4096, M = 1: quantize, then the GEMV
     L = workloads.make_layer(workloads.seed_of(0, 0), K=4096, N=4096)
     W, act = torch.from_numpy(L.W).cuda(), torch.from_numpy(L.act_absmean).cuda()
@@ -661,7 +672,7 @@ def run_configs(torch, w4, pk, pk_kind, quant8b):
     packs = [(qw, sc, z)] + [(qw.clone(), sc.clone(), z.clone()) for _ in range(_copies(workloads.packed_bytes(4096, 4096)) - 1)]
     x = _x(torch, workloads.seed_of(0, 0), 1, L.mult)
     y = torch.empty(1, 4096, dtype=torch.bfloat16, device="cuda")
-    ms_g = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p, out=y) for p in packs])
+    ms_g = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p, out=y, workspace=ws) for p in packs])
     out["config0_single_layer"] = {
         "workload": "4096x4096, M=1: awq_quantize_g128 then w4a16_gemv",
         "quantize": _rate(nbytes=4096 * 4096 * 4 + workloads.packed_bytes(4096, 4096) + 4096 * 4, ms=ms_q, pk=pk),
@@ -685,16 +696,17 @@ def run_configs(torch, w4, pk, pk_kind, quant8b):
             x = _x(torch, workloads.seed_of(3, si), M, L.mult)
             y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
             if M <= 16:
-                ms_c = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p[:3], csr=p[3], out=y) for p in packs])
-                ms_0 = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p[:3], out=y) for p in packs])
+                ms_c = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p[:3], csr=p[3], out=y, workspace=ws)
+                                           for p in packs])
+                ms_0 = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p[:3], out=y, workspace=ws) for p in packs])
                 b0 = gemv_bytes(N, K, M)
                 rows.append({"K": K, "N": N, "M": M, "nnz": nnz, "kernel": "gemv",
                              "csr": _rate(nbytes=b0 + csr_bytes, ms=ms_c, pk=pk), "no_csr": _rate(nbytes=b0, ms=ms_0, pk=pk),
                              "csr_cost": round(ms_c / ms_0 - 1.0, 4)})
             else:
                 p = packs[0]
-                ms_c = _time_calls(torch, [lambda: w4.w4a16_gemm(x, *p[:3], csr=p[3], out=y)])
-                ms_0 = _time_calls(torch, [lambda: w4.w4a16_gemm(x, *p[:3], out=y)])
+                ms_c = _time_calls(torch, [lambda: w4.w4a16_gemm(x, *p[:3], csr=p[3], out=y, workspace=ws)])
+                ms_0 = _time_calls(torch, [lambda: w4.w4a16_gemm(x, *p[:3], out=y, workspace=ws)])
                 f0 = 2.0 * M * N * K
                 rows.append({"K": K, "N": N, "M": M, "nnz": nnz, "kernel": "gemm",
                              "csr": _rate(flops=f0 + 2.0 * M * nnz, ms=ms_c, pk=pk), "no_csr": _rate(flops=f0, ms=ms_0, pk=pk),
@@ -721,11 +733,11 @@ def run_configs(torch, w4, pk, pk_kind, quant8b):
             x = _x(torch, workloads.seed_of(4, si), M, mult)
             y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
             if M <= 16:
-                ms = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p, out=y) for p in packs])
+                ms = _time_calls(torch, [lambda p=p: w4.w4a16_gemv(x, *p, out=y, workspace=ws) for p in packs])
                 rows.append({"K": K, "N": N, "M": M, "kernel": "gemv", **_rate(nbytes=gemv_bytes(N, K, M), ms=ms, pk=pk)})
             else:
                 use = packs if M <= 256 else packs[:1]  # the ridge point streams its weights: cycle copies
-                ms = _time_calls(torch, [lambda p=p: w4.w4a16_linear(x, *p, out=y) for p in use], 10)
+                ms = _time_calls(torch, [lambda p=p: w4.w4a16_linear(x, *p, out=y, workspace=ws) for p in use], 10)
                 r = {"K": K, "N": N, "M": M, "kernel": "gemm"}
                 if M <= 256:  # near the ridge: both rooflines
                     r.update(_rate(nbytes=gemv_bytes(N, K, M), flops=2.0 * M * N * K, ms=ms, pk=pk))
@@ -807,7 +819,7 @@ def run_case(args):
     y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     sched = {"auto": w4.GEMV_AUTO, "stream_k": w4.GEMV_STREAM_K, "cluster": w4.GEMV_CLUSTER}[args.schedule]
     fn = {"gemv": lambda *a, **k: w4.w4a16_gemv_ex(*a, **k, schedule=sched), "gemm": w4.w4a16_gemm}.get(args.case)
-    ws = torch.zeros(max(256, w4.workspace_bytes(min(M, 16), N, K)), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(256, w4.workspace_bytes(M, N, K, csr=False)), dtype=torch.uint8, device="cuda")
 
     def once(i):
         if args.case == "quantize":

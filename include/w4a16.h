@@ -121,23 +121,33 @@ w4a16_status awq_quantize(const float* W, const float* act_absmean, float alpha,
                           float* s_out, void* stream);
 
 /*
- * Workspace of the decode path.  The GEMV splits the output row blocks evenly over a
- * persistent grid.  Row blocks shared by two or more CTAs are combined through fp32
- * partial tiles and per-row-block counters, which live in a caller-provided device
- * workspace; w4a16_gemv_folded also writes its x / s there.
- *   - It must hold at least w4a16_workspace_bytes(M, N, K) bytes and be 16-byte aligned.
+ * Workspace.  A caller-provided device buffer holds the library's scratch:
+ *   - Decode path (M <= 16).  The GEMV splits the output row blocks evenly over a
+ *     persistent grid.  Row blocks shared by two or more CTAs are combined through fp32
+ *     partial tiles and per-row-block counters; w4a16_gemv_folded also writes its x / s
+ *     there, and a CSR term goes there as N x M fp32.
+ *   - Prefill path (the GEMM).  When the output tiles alone would leave SMs idle, the GEMM
+ *     splits K over several CTAs per tile; their fp32 partial tiles and per-tile counters
+ *     live in the workspace.  With a CSR term, x transposed (K x M' bf16) and the term
+ *     itself (N x M' fp32) go there too, M' = M rounded up to a multiple of 8.
+ *   - It must hold at least w4a16_workspace_bytes_ex(M, N, K, with_csr) bytes (with_csr: 1
+ *     when a CSR term is passed) and be 16-byte aligned.  w4a16_workspace_bytes(M, N, K) is
+ *     the size with a CSR term, enough either way.
  *   - It must be zero-filled before its first use.  Every call that completes leaves the
  *     parts that must start at zero zero-filled again, whatever its sizes, so one workspace
  *     of the largest size needed serves any number of calls of any sizes in stream order.
  *   - Calls that may run at the same time (on different streams without ordering between
  *     them) need different workspaces.
  *   - After a call reports W4A16_ERR_TIMEOUT, zero the workspace again before reusing it.
- * w4a16_workspace_bytes returns the size for the CURRENT device (it depends on the number
- * of SMs), or 0 when the call with these sizes needs no workspace (M > 16) or the sizes
- * are invalid.  It is 128 KiB of counters, 16 KiB of partial tiles per SM, M x K bf16 for
- * the folded activations and N x M fp32 for the CSR term (each rounded up to 256 bytes).
+ * Both functions return the size for the CURRENT device (it depends on the number of SMs),
+ * or 0 for invalid sizes.  Decode: 128 KiB of counters, 16 KiB of partial tiles per SM,
+ * M x K bf16 for the folded activations and N x M fp32 for the CSR term.  Prefill: 128 KiB
+ * of counters, the split-K partial tiles (none for grids that fill the GPU, else about
+ * splits x M x N x 4 bytes, at most 64 MiB), then the CSR parts above.  Each part is
+ * rounded up to 256 bytes.
  */
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+size_t w4a16_workspace_bytes_ex(int64_t M, int64_t N, int64_t K, int with_csr);
 
 /*
  * w4a16_linear -- y = bf16_rne( x . dequant(Q)^T + x . W_sparse^T ), fp32 accumulation.
@@ -148,11 +158,13 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   outliers host pointer to a w4a16_csr whose arrays are on the device, or NULL when
  *            there is no sparse term.  nnz may be 0.
  *   y        [M][N] bf16 bits, device, output.  It must not overlap any input.
- *   workspace, workspace_bytes: see above.  Required when M <= 16; ignored otherwise.
+ *   workspace, workspace_bytes: see above.  Required when M <= 16 or when a CSR is given.
+ *            Otherwise it may be NULL, and the GEMM then does not split K.
  *   M >= 1.  M <= 16 runs the decode GEMV; larger M runs the tensor-core GEMM.
- *   Decode path with a CSR: a small kernel first writes the sparse term x . W_sparse^T in
- *   fp32 to the workspace (fp16 values times bf16 activations, fp32 sums), while the GEMV
- *   already streams its weights; the GEMV adds it to each output before the one rounding.
+ *   With a CSR, small kernels first write the sparse term x . W_sparse^T in fp32 to the
+ *   workspace (fp16 values times bf16 activations, fp32 sums, entries in CSR order), while
+ *   the GEMV or GEMM already runs its main loop; its epilogue adds the term to each fp32
+ *   output before the one rounding to bf16.
  *   Errors: NULL, SHAPE, ALIGN and UNSUPPORTED when called (SHAPE also for a workspace that
  *   is too small).  Later: SHAPE if a CSR index is out of range (that entry is skipped),
  *   TIMEOUT if a pipeline wait runs out.
@@ -243,9 +255,12 @@ w4a16_status w4a16_gemv_folded(const uint16_t* x, const float* s, const uint32_t
                                size_t workspace_bytes, int schedule, void* stream);
 
 /* w4a16_gemm -- the tcgen05 tensor-core path of w4a16_linear, for any M >= 1.  Arguments
- * and result are as for w4a16_linear.  The workspace is not used (NULL and 0 are fine).
- * Weights are dequantized to bf16 inside the kernel.  When a CSR is given, its values are
- * added to those weights before the bf16 rounding that feeds the tensor cores. */
+ * and result are as for w4a16_linear, with the prefill workspace (see above): required with
+ * a CSR, optional without (NULL: one CTA per output tile).  Weights are dequantized to bf16
+ * inside the kernel; the sum over K is fp32 and, with split-K, its partial sums are added
+ * in a fixed order, so the result does not depend on which CTA finishes first.
+ * Launch overlap with a CSR: the GEMM may start its main loop while the CSR kernels run and
+ * waits for them only before it adds the sparse term. */
 w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
                         const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y,
                         int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,

@@ -118,7 +118,7 @@ def test_gemv_workspace_contract(orc):
     c = Case(orc, seed=13, K=4096, N=512, M=3)
     d = c.device()
     need = w4.workspace_bytes(3, c.N, c.K)
-    assert need > 0 and w4.workspace_bytes(17, c.N, c.K) == 0
+    assert need > 0 and w4.workspace_bytes(17, c.N, c.K, csr=False) >= 128 * 1024  # prefill: counters at least
     with pytest.raises(w4.W4A16Error) as e:
         w4.w4a16_gemv(d["x"], d["qweight"], d["scales"], d["zeros"],
                       workspace=torch.zeros(need - 256, dtype=torch.uint8, device="cuda"))

@@ -12,7 +12,7 @@ mirror the C ABI in include/w4a16.h:
   w4a16_linear_ex(..., group_size, schedule)    -> y      (weights from awq_quantize with that group size)
   gemv_plan(M, N, K, schedule)                  -> (schedule, cluster size, CTAs) the call would launch
   w4a16_gemm(...)                               -> y      (tcgen05 path, any M)
-  workspace_bytes(M, N, K)                      -> bytes of zeroed device workspace a decode call needs
+  workspace_bytes(M, N, K, csr=True)            -> bytes of zeroed device workspace a call needs
   check_device_status()                         -> raises W4A16Error on a recorded problem
 
 Bit containers: qweight [N][K/8] and zeros [K/128][N/8] are int32 tensors holding uint32
@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.w4a16_gemv_plan.argtypes = [I64, I64, I64, ctypes.c_int, PI, PI, PI]
         L.w4a16_workspace_bytes.argtypes = [I64, I64, I64]
         L.w4a16_workspace_bytes.restype = ctypes.c_size_t
+        L.w4a16_workspace_bytes_ex.argtypes = [I64, I64, I64, ctypes.c_int]
+        L.w4a16_workspace_bytes_ex.restype = ctypes.c_size_t
         L.w4a16_check_device_status.argtypes = [P]
         L.w4a16_selftest_timeout.argtypes = [I64, P]
         L.w4a16_selftest_quotient.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint32), P]
@@ -203,8 +205,9 @@ def workspace(device: torch.device, nbytes: int, stream=None) -> torch.Tensor:
     return ws
 
 
-def workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(lib().w4a16_workspace_bytes(M, N, K))
+def workspace_bytes(M: int, N: int, K: int, csr: bool = True) -> int:
+    """Bytes of workspace a call with these sizes needs (csr: whether it passes a CSR term)."""
+    return int(lib().w4a16_workspace_bytes_ex(M, N, K, 1 if csr else 0))
 
 
 def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, schedule=None, group_size=None,
@@ -229,7 +232,7 @@ def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, s
         _need(rp, torch.int32, 1, "row_ptr")
         cs = Csr(rp.data_ptr(), ci.data_ptr() if ci.numel() else None, v.data_ptr() if v.numel() else None,
                  int(ci.numel()))
-    need = workspace_bytes(M, N, K) if name != "w4a16_gemm" else 0
+    need = workspace_bytes(M, N, K, csr is not None)
     if ws is None and need > 0:
         ws = workspace(x.device, need)
     args = [_ptr(x)] + ([_ptr(s)] if fold else []) + [
@@ -396,6 +399,12 @@ def awq_search_alpha_workspace_bytes(M: int, N: int, K: int, n_alpha: int) -> in
 
 
 w4a16_workspace_bytes = workspace_bytes
+
+
+def w4a16_workspace_bytes_ex(M: int, N: int, K: int, with_csr: int) -> int:
+    return workspace_bytes(M, N, K, bool(with_csr))
+
+
 w4a16_gemv_plan = gemv_plan
 w4a16_check_device_status = check_device_status
 w4a16_selftest_timeout = selftest_timeout

@@ -128,7 +128,8 @@ struct LinearArgs {
     int group_ratio = 1;  // group size / 128
     float* partials = nullptr;   // the GEMV's scratch (gemv_partial_bytes)
     unsigned* counters = nullptr;  // zero when the call starts (gemv_counter_bytes)
-    float* ysp = nullptr;          // the GEMV's CSR term, [N][M] fp32 (only with a CSR)
+    float* ysp = nullptr;          // the CSR term: decode [N][M], prefill [N][ld] fp32 (only with a CSR)
+    uint16_t* xT = nullptr;        // prefill with a CSR: x transposed, [K][ld] bf16
 };
 
 w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -234,21 +235,48 @@ w4a16_status take_decode_workspace(LinearArgs* a, void* workspace, size_t worksp
     return W4A16_OK;
 }
 
-int pick_bn(int64_t M) {
-    if (M <= 32) return 32;
-    if (M <= 64) return 64;
-    if (M <= 128) return 128;
-    return 256;
+// The prefill workspace (M > 16):
+//   [0, kCounterRegionBytes)   the split-K tile counters (zero between calls; shared with the
+//                              decode layout, which keeps its counters there too);
+//   then plan.partial_bytes    fp32 partial tiles of split-K, rounded up to 256 bytes;
+//   then K x ld bf16           x transposed (only with a CSR), rounded up to 256 bytes;
+//   then N x ld fp32           the CSR term (only with a CSR); ld = csr_token_stride(M).
+size_t up256(size_t b) { return (b + 255) / 256 * 256; }
+
+size_t prefill_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms, bool csr) {
+    const GemmPlan g = gemm_plan(M, N, K, num_sms);
+    size_t b = kCounterRegionBytes + up256(g.partial_bytes);
+    if (csr) {
+        const size_t ld = (size_t)csr_token_stride(M);
+        b += up256((size_t)K * ld * 2) + up256((size_t)N * ld * 4);
+    }
+    return b;
 }
 
-w4a16_status run_gemm(const LinearArgs& a, cudaStream_t stream) {
+// The prefill GEMM.  workspace may be nullptr when there is no CSR term: the GEMM then runs
+// without split-K.
+w4a16_status run_gemm(const LinearArgs& a, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
     DeviceInfo* d = nullptr;
     w4a16_status st = device_info(&d);
     if (st != W4A16_OK) return st;
     EncodeTiledFn enc = nullptr;
     st = encoder(&enc);
     if (st != W4A16_OK) return st;
-    const int bn = pick_bn(a.M);
+    const bool csr = a.row_ptr != nullptr;
+    GemmPlan plan = gemm_plan(a.M, a.N, a.K, d->num_sms);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (ws == nullptr) {
+        if (csr) return W4A16_ERR_NULL;
+        plan = GemmPlan{plan.bn, 1, (int)(a.K / 128), 0};
+    } else {
+        if (!aligned(ws, 16)) return W4A16_ERR_ALIGN;
+        if (workspace_bytes < prefill_workspace_bytes(a.M, a.N, a.K, d->num_sms, csr)) return W4A16_ERR_SHAPE;
+    }
+    const int bn = plan.bn;
+    if ((a.M + bn - 1) / bn > 65535) return W4A16_ERR_UNSUPPORTED;  // grid y limit
+    if (csr && ((int64_t)csr_token_stride(a.M) / 32 + 1 > 65535 ||
+                a.N * ((a.M + 255) / 256) * 32 >= ((int64_t)1 << 31)))
+        return W4A16_ERR_UNSUPPORTED;  // launch limits of the CSR kernels
     GemmMaps maps;
     {   // x: bf16 [M][K]; box 64 k (128 bytes) x bn tokens; 128-byte swizzle
         cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
@@ -270,8 +298,21 @@ w4a16_status run_gemm(const LinearArgs& a, cudaStream_t stream) {
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4A16_ERR_CUDA;
     }
-    return from_cuda(launch_gemm(maps, a.group_ratio, a.scales, a.zeros, a.row_ptr, a.col_idx, a.vals, a.nnz, a.y,
-                                 (int)a.M, (int)a.N, (int)a.K, bn, d->num_sms, d->status, stream));
+    unsigned* counters = ws != nullptr ? reinterpret_cast<unsigned*>(ws) : nullptr;
+    float* partials = ws != nullptr ? reinterpret_cast<float*>(ws + kCounterRegionBytes) : nullptr;
+    const float* ysp = nullptr;
+    const int ld = csr_token_stride(a.M);
+    if (csr) {
+        uint8_t* base = ws + kCounterRegionBytes + up256(plan.partial_bytes);
+        uint16_t* xT = reinterpret_cast<uint16_t*>(base);
+        float* yspw = reinterpret_cast<float*>(base + up256((size_t)a.K * ld * 2));
+        st = from_cuda(launch_csr_prefill(a.x, a.row_ptr, a.col_idx, a.vals, a.nnz, (int)a.M, (int)a.N, (int)a.K, xT,
+                                          yspw, d->status, stream));
+        if (st != W4A16_OK) return st;
+        ysp = yspw;
+    }
+    return from_cuda(launch_gemm(maps, plan, a.group_ratio, a.scales, a.zeros, ysp, ld, a.y, partials, counters,
+                                 (int)a.M, (int)a.N, (int)a.K, d->status, stream));
 }
 
 // ---------------------------------------------------------------------------------------
@@ -328,13 +369,16 @@ w4a16_status awq_quantize_g128(const float* W, const float* act_absmean, float a
     return awq_quantize(W, act_absmean, alpha, N, K, 128, qweight, scales, zeros, s_out, stream);
 }
 
-size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    if (M < 1 || M > 16 || N < 128 || N % 128 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > gemv_max_k())
+size_t w4a16_workspace_bytes_ex(int64_t M, int64_t N, int64_t K, int with_csr) {
+    if (M < 1 || M > kMaxM || N < 128 || N % 128 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK)
         return 0;
     DeviceInfo* d = nullptr;
     if (device_info(&d) != W4A16_OK) return 0;
-    return decode_workspace_bytes(M, N, K, d->num_sms);
+    if (M <= 16 && K <= gemv_max_k()) return decode_workspace_bytes(M, N, K, d->num_sms);
+    return prefill_workspace_bytes(M, N, K, d->num_sms, with_csr != 0);
 }
+
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) { return w4a16_workspace_bytes_ex(M, N, K, 1); }
 
 w4a16_status w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
                         const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
@@ -406,12 +450,10 @@ w4a16_status w4a16_gemv_plan(int64_t M, int64_t N, int64_t K, int schedule, int*
 w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint32_t* zeros,
                         const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
                         size_t workspace_bytes, void* stream) {
-    (void)workspace;
-    (void)workspace_bytes;
     LinearArgs a;
     w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
     if (st != W4A16_OK) return st;
-    return run_gemm(a, static_cast<cudaStream_t>(stream));
+    return run_gemm(a, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 w4a16_status w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -421,7 +463,7 @@ w4a16_status w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint
     w4a16_status st = validate_linear(x, qweight, scales, zeros, outliers, y, M, N, K, &a);
     if (st != W4A16_OK) return st;
     const bool decode = M <= 16 && K <= gemv_max_k();
-    if (!decode) return run_gemm(a, static_cast<cudaStream_t>(stream));
+    if (!decode) return run_gemm(a, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
     st = take_decode_workspace(&a, workspace, workspace_bytes, nullptr);
     if (st != W4A16_OK) return st;
     return run_gemv(a, static_cast<cudaStream_t>(stream));
@@ -438,7 +480,7 @@ w4a16_status w4a16_linear_ex(const uint16_t* x, const uint32_t* qweight, const u
     if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
     a.group_ratio = (int)(group_size / 128);
     const bool decode = M <= 16 && K <= gemv_max_k();
-    if (!decode) return run_gemm(a, static_cast<cudaStream_t>(stream));
+    if (!decode) return run_gemm(a, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
     st = take_decode_workspace(&a, workspace, workspace_bytes, nullptr);
     if (st != W4A16_OK) return st;
     return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);
@@ -552,7 +594,7 @@ w4a16_status awq_search_alpha(const float* W, const float* act_absmean, const ui
             a.partials = reinterpret_cast<float*>(ws + L.gemv + gemv_counter_bytes((int)N));
             st = run_gemv(a, s);
         } else {
-            st = run_gemm(a, s);
+            st = run_gemm(a, nullptr, 0, s);
         }
         if (st != W4A16_OK) break;
         st = from_cuda(launch_search_err(yq, yref, (long long)(M * N), acc + 1 + i, i == 0 ? acc : nullptr,

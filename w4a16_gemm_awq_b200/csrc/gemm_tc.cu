@@ -1,6 +1,6 @@
 // gemm_tc.cu -- prefill W4A16 GEMM on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
 //
-// y[m][n] = bf16( sum_k x[m][k] * w~[n][k] ),  w~ = bf16((q - z) * scale) (+ CSR value)
+// y[m][n] = bf16( sum_k x[m][k] * w~[n][k]  (+ ysp[n][m]) ),  w~ = bf16((q - z) * scale)
 //
 // [AWQ (MLSys 2024) translation, section 1: TinyChat dequantizes the packed 4-bit weights on
 //  the fly inside the linear-layer kernel; SqueezeLLM article, section 2.3: W x = W_dense x +
@@ -22,10 +22,15 @@
 //   - Warp roles: warp 0 issues the TMA, warp 1 issues tcgen05.mma from one thread, and
 //     warps 2..5 dequantize and then run the epilogue.  There are four smem stages and
 //     four TMEM A-stages, linked by mbarriers; tcgen05.commit releases the stages.
-//   - CSR outlier term: each dequant thread walks its row of the CSR.  It adds each value
-//     (fp32) to the dequantized weight at that column before the bf16 rounding.  The
-//     sparse product therefore rides on the same tensor-core contraction, with no gather
-//     of x and no extra pass.
+//   - Split-K for small grids: when the output tiles alone would leave SMs idle, the grid's
+//     z dimension splits K into equal runs of whole 128-k slices.  Every CTA of a tile writes
+//     its fp32 partial tile to the workspace and counts itself in the tile's counter; the CTA
+//     that arrives last adds the partials in split order (its own from TMEM), so the sum's
+//     order, and every bit of y, is the same whichever CTA finishes last.  It then resets the
+//     counter to zero.  No CTA waits for another.
+//   - CSR outlier term: the kernels of csr.cu compute ysp[n][m] = x . W_sparse^T in fp32
+//     just before this kernel, which may start meanwhile (programmatic dependent launch).
+//     The epilogue waits for them and adds ysp to the fp32 sum before the one rounding.
 //   - Every mbarrier wait is bounded.  On timeout the CTA records kErrTimeout, stops its
 //     loops, drains its own TMA and MMA work with bounded waits, and frees its TMEM.
 #include "common.cuh"
@@ -43,13 +48,15 @@ constexpr uint32_t kACols = kBK / 2;             // TMEM columns per A-stage (bf
 struct GemmArgs {
     const uint16_t* scales;
     const uint32_t* zeros;
-    const int32_t* row_ptr;
-    const int32_t* col_idx;
-    const uint16_t* vals;
-    long long nnz;
+    const float* ysp;  // the CSR term [N][ysp_ld] fp32, or nullptr
+    int ysp_ld;
     uint16_t* y;
+    float* partials;    // split-K: fp32 tiles [tile][split][128][BN]
+    unsigned* counters; // split-K: one per tile, zero between calls
     int M, N, K;
-    int gr;  // quantization group size / 128: scales and zeros of 128-slice g are those of group g / gr
+    int gr;      // quantization group size / 128: scales and zeros of 128-slice g are those of group g / gr
+    int splits;  // CTAs per output tile along K (gridDim.z)
+    int slices;  // 128-k slices per split
     unsigned* err;
 };
 
@@ -84,11 +91,8 @@ __device__ __forceinline__ constexpr uint32_t idesc_bf16_m128() {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-__device__ __forceinline__ uint32_t patch_bf16x2(uint32_t v, int hi, float add) {
-    const float old = __uint_as_float(hi ? (v & 0xFFFF0000u) : (v << 16));
-    const uint32_t nb = float_to_bf16_bits(old + add);
-    return hi ? ((v & 0x0000FFFFu) | (nb << 16)) : ((v & 0xFFFF0000u) | nb);
-}
+// Barrier 1 among the four epilogue warps (warps 2..5).
+__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -104,10 +108,14 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     uint64_t* accfull = aempty + kAStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN;
-    const int nK = p.K / kBK;
+    // this CTA's stages: [s0, s0 + nK), whole 128-k slices (a slice's first stage brings its
+    // scales and zero points)
+    const int s0 = (int)blockIdx.z * p.slices * 2;
+    const int nK = min(p.slices * 2, p.K / kBK - s0);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -152,14 +160,15 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     fail();
                     break;
                 }
-                // a stage that starts a group also brings the group's 128 scales and 16 zero words
-                const bool first_half = (s & 1) == 0;
+                // a stage that starts a slice also brings the slice's 128 scales and 16 zero words
+                const int sg = s0 + s;  // stage index along K
+                const bool first_half = (sg & 1) == 0;
                 mbar_arrive_expect_tx(&full[slot],
                                       (uint32_t)(L::kXStageBytes + kWStageBytes + (first_half ? 256 + 64 : 0)));
-                tma_load_2d(smem + L::kXOff + slot * L::kXStageBytes, &map_x, &full[slot], s * kBK, m0);
-                tma_load_2d(smem + L::kWOff + slot * kWStageBytes, &map_w, &full[slot], s * (kBK / 8), n0);
+                tma_load_2d(smem + L::kXOff + slot * L::kXStageBytes, &map_x, &full[slot], sg * kBK, m0);
+                tma_load_2d(smem + L::kWOff + slot * kWStageBytes, &map_w, &full[slot], sg * (kBK / 8), n0);
                 if (first_half) {
-                    const int g = (s >> 1) / p.gr;  // the quantization group of this 128-slice
+                    const int g = (sg >> 1) / p.gr;  // the quantization group of this 128-slice
                     uint8_t* par = smem + L::kParOff + slot * 512;
                     bulk_load(par, p.scales + (size_t)g * p.N + n0, 256, &full[slot]);
                     bulk_load(par + 256, p.zeros + (size_t)g * (p.N >> 3) + (n0 >> 3), 64, &full[slot]);
@@ -203,22 +212,6 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
         uint32_t sb = 0, zb = 0;
 
-        // CSR walk for this row: next entry's column and value
-        int jc = 0, jend = 0, ccol = 0x7FFFFFFF;
-        float cval = 0.0f;
-        if (p.row_ptr != nullptr) {
-            jc = p.row_ptr[n];
-            jend = p.row_ptr[n + 1];
-            if (jc < 0 || jend < jc || (long long)jend > p.nnz) {
-                record_error(p.err, kErrShape);
-                jend = jc;
-            }
-            if (jc < jend) {
-                ccol = p.col_idx[jc];
-                cval = fp16_bits_to_float(p.vals[jc]);
-            }
-        }
-
         // waits and abort checks are made warp-uniform: tcgen05.st/ld are .sync.aligned
         auto warp_wait = [&](uint64_t* bar, uint32_t parity) {
             const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
@@ -236,7 +229,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             const int sw = (row >> 2) & 1;
             const uint4 wa = *reinterpret_cast<const uint4*>(wrow + ((0 ^ sw) << 4));
             const uint4 wb = *reinterpret_cast<const uint4*>(wrow + ((1 ^ sw) << 4));
-            if ((s & 1) == 0) {  // a new group of 128 k: its scale and zero point from the stage
+            if (((s0 + s) & 1) == 0) {  // a new slice of 128 k: its scale and zero point from the stage
                 const uint8_t* par = smem + L::kParOff + slot * 512;
                 const uint16_t sbits = reinterpret_cast<const uint16_t*>(par)[row];
                 const uint32_t z = (reinterpret_cast<const uint32_t*>(par + 256)[row >> 3] >> (4 * (row & 7))) & 15u;
@@ -260,26 +253,6 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 }
             }
 
-            // CSR values of this row that fall in the stage's 64 columns
-            const int kend = (s + 1) * kBK;
-            while (ccol < kend) {
-                const int pos = ccol - s * kBK;
-                if (pos >= 0 && ccol < p.K) {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (c == (pos >> 1)) v[c] = patch_bf16x2(v[c], pos & 1, cval);
-                } else {
-                    record_error(p.err, kErrShape);  // unsorted or out-of-range column
-                }
-                ++jc;
-                if (jc < jend) {
-                    ccol = p.col_idx[jc];
-                    cval = fp16_bits_to_float(p.vals[jc]);
-                } else {
-                    ccol = 0x7FFFFFFF;
-                }
-            }
-
             if (s >= kAStages && !warp_wait(&aempty[as], ((s / kAStages) - 1) & 1)) break;
             tc_fence_after();
             tmem_st_32x32b_x32(tmem + t_lane + a_col0 + (uint32_t)as * kACols, v);
@@ -289,12 +262,41 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             if (lane == 0) mbar_arrive(&afull[as]);
         }
         const bool aborted = warp_abort();
-        if (jc < jend && !aborted) record_error(p.err, kErrShape);  // entries past column K
 
-        // epilogue: TMEM -> registers -> bf16 -> y[m][n]
-        if (!aborted) {
-            if (warp_wait(accfull, 0)) {
-                tc_fence_after();
+        // epilogue: TMEM -> registers (-> split-K reduction) (+ CSR term) -> bf16 -> y[m][n]
+        if (!aborted && warp_wait(accfull, 0)) {
+            tc_fence_after();
+            const size_t tile = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+            const int z = (int)blockIdx.z;
+            bool last = true;
+            if (p.splits > 1) {
+                // this CTA's partial tile, row by row: thread `row` writes BN contiguous floats
+                float* mine = p.partials + ((tile * p.splits + z) * 128 + row) * BN;
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c0, r);
+                    tmem_ld_wait();
+                    float4* dst = reinterpret_cast<float4*>(mine + c0);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                             __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                }
+                __threadfence();
+                epilogue_sync();
+                if (warp == 2 && lane == 0) {
+                    const unsigned before = atomicAdd(p.counters + tile, 1u);
+                    const bool is_last = before == (unsigned)(p.splits - 1);
+                    if (is_last) p.counters[tile] = 0u;  // every split has counted itself
+                    *last_flag = is_last ? 1 : 0;
+                }
+                epilogue_sync();
+                last = *last_flag != 0;
+                if (last) __threadfence();
+            }
+            if (p.splits == 1 && p.ysp == nullptr) {
+                // the common case, kept minimal: one TMEM chunk at a time straight to y
 #pragma unroll 1
                 for (int c0 = 0; c0 < BN; c0 += 32) {
                     uint32_t r[32];
@@ -305,6 +307,56 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     for (int j = 0; j < 32; ++j) {
                         const int m = m0 + c0 + j;
                         if (m < p.M) p.y[(size_t)m * p.N + n] = float_to_bf16_bits(__uint_as_float(r[j]));
+                    }
+                }
+            } else if (last) {
+                const float* ysr = nullptr;
+                if (p.ysp != nullptr) {
+                    asm volatile("griddepcontrol.wait;" ::: "memory");  // ysp is complete
+                    ysr = p.ysp + (size_t)n * p.ysp_ld;
+                }
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c0, r);
+                    tmem_ld_wait();
+                    if (m0 + c0 >= p.M) break;
+                    float acc[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(r[j]);
+                    if (p.splits > 1) {
+                        // sum of the partial tiles in split order; this CTA's own is in acc
+                        float own[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) own[j] = acc[j];
+#pragma unroll 1
+                        for (int zz = 0; zz < p.splits; ++zz) {
+                            float v[32];
+                            if (zz == z) {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) v[j] = own[j];
+                            } else {
+                                const float4* src = reinterpret_cast<const float4*>(
+                                    p.partials + ((tile * p.splits + zz) * 128 + row) * BN + c0);
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) {
+                                    const float4 f = __ldcg(src + q);
+                                    v[4 * q] = f.x, v[4 * q + 1] = f.y, v[4 * q + 2] = f.z, v[4 * q + 3] = f.w;
+                                }
+                            }
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) acc[j] = zz == 0 ? v[j] : acc[j] + v[j];
+                        }
+                    }
+                    if (ysr != nullptr) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (m0 + c0 + j < p.M) acc[j] += __ldcg(ysr + m0 + c0 + j);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = m0 + c0 + j;
+                        if (m < p.M) p.y[(size_t)m * p.N + n] = float_to_bf16_bits(acc[j]);
                     }
                 }
             }
@@ -320,7 +372,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
 }
 
 template <int BN>
-static cudaError_t launch_bn(const GemmMaps& maps, const GemmArgs& a, cudaStream_t stream) {
+static cudaError_t launch_bn(const GemmMaps& maps, const GemmArgs& a, bool after_csr, cudaStream_t stream) {
     using L = GemmSmem<BN>;
     // At most 512 / kTmemCols CTAs may share an SM, or a tcgen05.alloc would have to wait for
     // another CTA's TMEM: the shared-memory request enforces that bound.
@@ -328,21 +380,62 @@ static cudaError_t launch_bn(const GemmMaps& maps, const GemmArgs& a, cudaStream
     const int smem = (L::kBytes + 1024) > kMinSmem ? (L::kBytes + 1024) : kMinSmem;
     cudaError_t e = cudaFuncSetAttribute(gemm_w4a16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.N / 128, (a.M + BN - 1) / BN);
-    gemm_w4a16_tc_kernel<BN><<<grid, kGemmThreads, smem, stream>>>(maps.x, maps.qw, a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.N / 128, (a.M + BN - 1) / BN, a.splits);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_csr ? 1 : 0;  // overlap the CSR kernels; otherwise plain stream order
+    return cudaLaunchKernelEx(&cfg, gemm_w4a16_tc_kernel<BN>, maps.x, maps.qw, a);
 }
 
-cudaError_t launch_gemm(const GemmMaps& maps, int group_ratio, const uint16_t* scales, const uint32_t* zeros,
-                        const int32_t* row_ptr,
-                        const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, int M, int N,
-                        int K, int bn, int /*num_sms*/, unsigned* err, cudaStream_t stream) {
-    GemmArgs a{scales, zeros, row_ptr, col_idx, vals, nnz, y, M, N, K, group_ratio, err};
-    switch (bn) {
-        case 32: return launch_bn<32>(maps, a, stream);
-        case 64: return launch_bn<64>(maps, a, stream);
-        case 128: return launch_bn<128>(maps, a, stream);
-        case 256: return launch_bn<256>(maps, a, stream);
+GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
+    GemmPlan g{};
+    g.bn = M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    const int64_t tiles = (N / 128) * ((M + g.bn - 1) / g.bn);
+    const int64_t nslices = K / 128;
+    g.splits = 1;
+    g.slices = (int)nslices;
+    // Time model in slices: waves x slices per CTA, plus about one slice per extra partial tile
+    // of 256 tokens that the last CTA reads back.  Only grids of under two waves are split
+    // (larger ones lose little to their last wave), only while the partial tiles stay within
+    // kMaxGemmPartialBytes, and only into runs of at least min_per slices: measured on
+    // B200, wide token tiles (whose CTAs each stream a large x tile) gained nothing from runs
+    // shorter than 32 slices (4096 x 4096 at M = 512), narrow ones gained down to runs of 8.
+    const int64_t min_per = g.bn == 256 ? 32 : g.bn == 128 ? 16 : 4;
+    if (tiles < 2 * (int64_t)num_sms && tiles <= kMaxGemmTiles) {
+        double best = (double)nslices;
+        for (int S = 2; S <= kMaxGemmSplits; ++S) {
+            const int64_t per = (nslices + S - 1) / S;
+            const int64_t used = (nslices + per - 1) / per;  // no empty split
+            if (used != S || per < min_per || (size_t)tiles * S * 128 * g.bn * 4 > kMaxGemmPartialBytes) continue;
+            const int64_t waves = (tiles * S + num_sms - 1) / num_sms;
+            const double cost = (double)(waves * per) + (double)(S - 1) * g.bn / 256.0;
+            if (cost < best - 0.5) {
+                best = cost;
+                g.splits = S;
+                g.slices = (int)per;
+            }
+        }
+    }
+    g.partial_bytes = g.splits > 1 ? (size_t)tiles * g.splits * 128 * g.bn * 4 : 0;
+    return g;
+}
+
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmPlan& plan, int group_ratio, const uint16_t* scales,
+                        const uint32_t* zeros, const float* ysp, int ysp_ld, uint16_t* y, float* partials,
+                        unsigned* counters, int M, int N, int K, unsigned* err, cudaStream_t stream) {
+    GemmArgs a{scales, zeros, ysp, ysp_ld, y, partials, counters, M, N, K, group_ratio, plan.splits, plan.slices, err};
+    const bool after_csr = ysp != nullptr;
+    switch (plan.bn) {
+        case 32: return launch_bn<32>(maps, a, after_csr, stream);
+        case 64: return launch_bn<64>(maps, a, after_csr, stream);
+        case 128: return launch_bn<128>(maps, a, after_csr, stream);
+        case 256: return launch_bn<256>(maps, a, after_csr, stream);
         default: return cudaErrorInvalidValue;
     }
 }

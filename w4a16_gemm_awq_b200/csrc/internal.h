@@ -69,6 +69,14 @@ cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ra
 cudaError_t launch_csr_rows(const uint16_t* x, const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals,
                             long long nnz, int M, int N, int K, float* ysp, unsigned* err, cudaStream_t stream);
 
+// The CSR term of the prefill path (see csr.cu): x is transposed into xT [K][ld] bf16, then
+// ysp[n][m] (row stride ld) is computed from it.  ld = csr_token_stride(M).  The GEMM launched
+// next may start while these run and waits for them before it reads ysp.
+inline int csr_token_stride(int64_t M) { return (int)((M + 7) / 8 * 8); }
+cudaError_t launch_csr_prefill(const uint16_t* x, const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals,
+                               long long nnz, int M, int N, int K, uint16_t* xT, float* ysp, unsigned* err,
+                               cudaStream_t stream);
+
 // Dense-and-sparse split of W on the GPU (see outliers.cu).  N * K < 2^32, 1 <= nnz <= N * K.
 size_t split_workspace_bytes(int64_t N);
 cudaError_t launch_split_outliers(const float* W, const float* act, float alpha, uint32_t N, uint32_t K, uint32_t nnz,
@@ -95,9 +103,26 @@ struct GemmMaps {
     CUtensorMap qw;  // uint32 [N][K/8], box 16 words (one group) x 128 rows, 64-byte swizzle
 };
 
-cudaError_t launch_gemm(const GemmMaps& maps, int group_ratio, const uint16_t* scales, const uint32_t* zeros,
-                        const int32_t* row_ptr,
-                        const int32_t* col_idx, const uint16_t* vals, long long nnz, uint16_t* y, int M, int N,
-                        int K, int bn, int num_sms, unsigned* err, cudaStream_t stream);
+// A GEMM launch: token tile BN (32, 64, 128 or 256), CTAs per output tile along K (splits,
+// each over `slices` 128-k slices) and the bytes of fp32 partial tiles that split-K needs.
+// Splitting is limited to kMaxGemmTiles tiles (their counters live in the workspace's counter
+// region), kMaxGemmSplits CTAs per tile and kMaxGemmPartialBytes of partial tiles.
+constexpr int kMaxGemmTiles = 4096;
+constexpr int kMaxGemmSplits = 8;
+constexpr size_t kMaxGemmPartialBytes = size_t(64) << 20;
+struct GemmPlan {
+    int bn;
+    int splits;
+    int slices;
+    size_t partial_bytes;
+};
+GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K, int num_sms);
+
+// partials and counters: the workspace's split-K parts (unused when plan.splits == 1; the
+// counters must be zero and are left zero).  ysp: nullptr or the CSR term from
+// launch_csr_prefill, row stride ysp_ld.
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmPlan& plan, int group_ratio, const uint16_t* scales,
+                        const uint32_t* zeros, const float* ysp, int ysp_ld, uint16_t* y, float* partials,
+                        unsigned* counters, int M, int N, int K, unsigned* err, cudaStream_t stream);
 
 }  // namespace w4a16
