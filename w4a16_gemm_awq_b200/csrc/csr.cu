@@ -11,12 +11,13 @@
 // finishes and reads x after it; the GEMV streams its weights meanwhile and reads ysp only
 // after this kernel has finished.
 //
-// Work split: 4 lanes per (row n, token m); lane q takes the row's entries j0 + q, j0 + q + 4,
-// ... and accumulates val * x[m][col] in fp32 from -0 (the additive identity, so an empty row
-// adds nothing to the dense sum's bits); the 4 partial sums are then combined as
-// (p0 + p1) + (p2 + p3) by two shuffle steps.  The order is fixed, so every call gives the
-// same bits.  Entries are independent within a lane, so their loads overlap; with many rows in
-// flight across the GPU the gathers of x (small, L2-resident) are latency-, not bandwidth-bound.
+// Work split: one warp per row n.  Lane l takes the row's entries j0 + l, j0 + l + 32, ...
+// (its column and value are read once for all tokens) and keeps one fp32 partial sum per token,
+// accumulated from -0 (the additive identity, so an empty row adds nothing to the dense sum's
+// bits).  The 32 partial sums of each token are then added by a butterfly (xor 16, 8, 4, 2, 1),
+// whose order is fixed, so every call gives the same bits.  Lane m writes token m.  CTAs are
+// 4 warps, small enough in registers that many fit beside each other and the whole grid
+// starts at once.
 //
 // Prefill (M > 16): the same term for many tokens.  Gathering x[m][col] for a fixed column
 // over many tokens would touch one 32-byte sector per token, so x is first transposed into
@@ -24,76 +25,72 @@
 // tokens: lane l owns tokens m0 + 8l .. m0 + 8l + 7, reads them with one 16-byte load per
 // entry (a warp reads 512 contiguous bytes of xT per entry) and accumulates in fp32 from -0,
 // entry after entry in CSR order.  ysp[n][m] has the same padded token stride, so the GEMM's
-// epilogue reads a row's tokens contiguously.
+// epilogue reads a row's tokens contiguously.  (A persistent grid of two CTAs per SM, so that
+// the GEMM could start beside it, was measured slower: the two slowed each other.  Batching
+// four entries' loads per step did not help either.)
 #include "common.cuh"
 #include "internal.h"
 
 namespace w4a16 {
 
-constexpr int kCsrLanes = 4;  // lanes per (row, token)
-constexpr int kCsrAhead = 8;  // entries per lane fetched before waiting for the previous kernel
+constexpr int kCsrWarps = 4;  // warps (rows) per CTA of the decode kernel
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(32 * kCsrWarps)
 csr_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
                 const uint16_t* __restrict__ vals, long long nnz, int M, int N, int K, float* __restrict__ ysp,
                 unsigned* err) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const int q = (int)(t % kCsrLanes);
-    const long long rm = t / kCsrLanes;  // (row, token) index, token fastest
-    const bool live = rm < (long long)N * M;
-    const int n = live ? (int)(rm / M) : 0, m = live ? (int)(rm % M) : 0;
+    const int lane = threadIdx.x & 31;
+    const int n = blockIdx.x * kCsrWarps + (threadIdx.x >> 5);
+    if (n >= N) return;
     // The CSR arrays do not come from the previous kernel (as for the weights): this lane's
-    // first kCsrAhead entries are fetched before waiting for it; x after.
-    int j0 = 0, j1 = 0;
-    if (live) {
-        j0 = row_ptr[n];
-        j1 = row_ptr[n + 1];
-        if (j0 < 0 || j1 < j0 || (long long)j1 > nnz) {
-            if (q == 0) record_error(err, kErrShape);
-            j1 = j0;
-        }
+    // first entry is fetched before waiting for it; x after.
+    int j0 = row_ptr[n], j1 = row_ptr[n + 1];
+    if (j0 < 0 || j1 < j0 || (long long)j1 > nnz) {
+        if (lane == 0) record_error(err, kErrShape);
+        j1 = j0;
     }
-    int c[kCsrAhead];
-    float v[kCsrAhead];
-#pragma unroll
-    for (int e = 0; e < kCsrAhead; ++e) {
-        const int j = j0 + q + kCsrLanes * e;
-        c[e] = j < j1 ? __ldg(col_idx + j) : -1;
-        v[e] = j < j1 ? fp16_bits_to_float(__ldg(vals + j)) : 0.0f;
+    int c = -1;
+    float v = 0.0f;
+    if (j0 + lane < j1) {
+        c = __ldg(col_idx + j0 + lane);
+        v = fp16_bits_to_float(__ldg(vals + j0 + lane));
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x belongs to the stream order
-    float acc = -0.0f;
-    const uint16_t* xr = x + (size_t)m * K;
+    float acc[16];
 #pragma unroll
-    for (int e = 0; e < kCsrAhead; ++e) {
-        const int j = j0 + q + kCsrLanes * e;
-        if (j < j1) {
-            if ((unsigned)c[e] >= (unsigned)K) record_error(err, kErrShape);  // the entry is skipped
-            else acc = fmaf(v[e], bf16_bits_to_float(__ldcg(xr + c[e])), acc);
+    for (int m = 0; m < 16; ++m) acc[m] = -0.0f;
+    for (int j = j0 + lane; j < j1; j += 32) {
+        if (j != j0 + lane) {
+            c = __ldg(col_idx + j);
+            v = fp16_bits_to_float(__ldg(vals + j));
         }
-    }
-#pragma unroll 4
-    for (int j = j0 + q + kCsrLanes * kCsrAhead; j < j1; j += kCsrLanes) {
-        const int cj = __ldg(col_idx + j);
-        if ((unsigned)cj >= (unsigned)K) {
+        if ((unsigned)c >= (unsigned)K) {  // the entry is skipped
             record_error(err, kErrShape);
             continue;
         }
-        acc = fmaf(fp16_bits_to_float(__ldg(vals + j)), bf16_bits_to_float(__ldcg(xr + cj)), acc);
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+            if (m < M) acc[m] = fmaf(v, bf16_bits_to_float(__ldg(x + (size_t)m * K + c)), acc[m]);
     }
-    // (p0 + p1) + (p2 + p3); the 4 lanes of a (row, token) are adjacent and in one warp
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (live && q == 0) ysp[(size_t)n * M + m] = acc;
+    float mine = 0.0f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        if (m < M) {
+            float t = acc[m];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+            if (lane == m) mine = t;
+        }
+    }
+    if (lane < M) ysp[(size_t)n * M + lane] = mine;
 }
 
 cudaError_t launch_csr_rows(const uint16_t* x, const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals,
                             long long nnz, int M, int N, int K, float* ysp, unsigned* err, cudaStream_t stream) {
-    const long long threads = (long long)N * M * kCsrLanes;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((threads + 255) / 256), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.gridDim = dim3((unsigned)((N + kCsrWarps - 1) / kCsrWarps), 1, 1);
+    cfg.blockDim = dim3(32 * kCsrWarps, 1, 1);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
