@@ -572,6 +572,42 @@ def run_gpu(args, world, rank, local):
                               "workload": "awq_quantize with group size K on the four Llama-3-8B layers"}}
         del rcalls
 
+    # 3-bit codes [SqueezeLLM article, sections 2.1-2.2]: quantize the four layers with eight
+    # levels, then the decode sweep's 16 calls through w3a16_gemv (own weights per call)
+    tinfo = None
+    if not args.skip_3bit:
+        tq_b, tq_ms = 0.0, 0.0
+        tcalls = []
+        for W, act, N, K in quant:
+            ms1, gq = time_graph(torch, lambda: w4.awq_quantize3(W, act, workloads.ALPHA, 128), 5, 2)
+            del gq
+            pb = N * (3 * K // 32) * 4 + (K // 128) * N * 2 + (K // 128) * (N // 8) * 4
+            tq_b += N * K * 4 + pb + K * 4
+            tq_ms += ms1
+            qw, sc, z, _ = w4.awq_quantize3(W, act, workloads.ALPHA, 128)
+            for j, M in enumerate(GEMV_MS):
+                packed = (qw, sc, z) if j == 0 else (qw.clone(), sc.clone(), z.clone())
+                x = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+                tcalls.append((x, packed, torch.empty(M, N, dtype=torch.bfloat16, device="cuda"),
+                               pb + 2 * M * K + 2 * M * N))
+        w4.check_device_status()
+
+        def tstep():
+            for x, (qw, sc, z), y, _ in tcalls:
+                w4.w3a16_gemv(x, qw, sc, z, out=y, workspace=ws)
+
+        ms_t, gt = time_graph(torch, tstep, 200, 5)
+        del gt
+        w4.check_device_status()
+        tb = sum(c[3] for c in tcalls)
+        tinfo = {"gemv": {"value": tb / (ms_t * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_t,
+                          "frac_of_hbm": tb / (ms_t * 1e-3) / 1e9 / pk["hbm_gbs"],
+                          "workload": "the decode sweep (4 Llama-3-8B shapes x M in {1, 4, 8, 16}) on 3-bit "
+                                      "codes (w3a16_gemv), own weights per call"},
+                 "quantize": {"value": tq_b / tq_ms / 1e6, "unit": "GB/s",
+                              "workload": "awq_quantize3 (g128) on the four Llama-3-8B layers"}}
+        del tcalls
+
     cinfo = None
     if not args.skip_configs:
         cinfo = run_configs(torch, w4, pk, pk_kind, quant)
@@ -604,6 +640,7 @@ def run_gpu(args, world, rank, local):
         "outlier_split": sinfo,
         "alpha_search": ainfo,
         "per_row_groups": rinfo,
+        "three_bit": tinfo,
         "fold_in_gemv": finfo,
         "configs": cinfo,
     }
@@ -865,6 +902,7 @@ def main():
     ap.add_argument("--skip-split", action="store_true")
     ap.add_argument("--skip-search", action="store_true")
     ap.add_argument("--skip-groups", action="store_true")
+    ap.add_argument("--skip-3bit", action="store_true")
     ap.add_argument("--skip-fold", action="store_true")
     ap.add_argument("--skip-configs", action="store_true")
     ap.add_argument("--case", choices=["gemv", "gemm", "quantize"], help="time one kernel on one layer (ncu)")

@@ -233,6 +233,38 @@ w4a16_status w4a16_linear_ex(const uint16_t* x, const uint32_t* qweight, const u
                              int64_t M, int64_t N, int64_t K, int64_t group_size, void* workspace,
                              size_t workspace_bytes, int schedule, void* stream);
 
+/*
+ * 3-bit codes [SqueezeLLM article, 2.1-2.2: once its few sensitive weights are split off, the
+ * dense part takes uniform quantization with as few as eight levels; 4.1 / 5.3: 3-bit runs].
+ *
+ * awq_quantize3 -- awq_quantize with codes 0..7: the same activation-aware scaling, groups,
+ *   scale and zero-point rules with 2^3 - 1 steps (scale = fp16(max((max - min) / 7, 1e-5)),
+ *   z = clamp(rint(-min / scale), 0, 7), q = clamp(rint(w' / scale) + z, 0, 7)).
+ *   qweight3 [N][3K/32] uint32: the 32 codes of k = 32b .. 32b + 31 of row n sit in the three
+ *            words qweight3[n][3b + w], w = 0..2: bits 4j .. 4j+2 of word w hold the code of
+ *            element 8w + ORDER[j]; bit 4j + 3 of word w holds bit w of the code of element
+ *            24 + ORDER[j] (ORDER as for 4-bit codes).
+ *   scales   [K/group_size][N] fp16 bits; zeros [K/group_size][N/8] (nibbles, values 0..7).
+ *   group_size  128, 256, 512 or 1024.  Everything else as awq_quantize.
+ */
+w4a16_status awq_quantize3(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                           int64_t group_size, uint32_t* qweight3, uint16_t* scales, uint32_t* zeros,
+                           float* s_out, void* stream);
+
+/*
+ * w3a16_gemv -- the decode GEMV (1 <= M <= 16) on 3-bit codes laid out as awq_quantize3
+ *   writes them, with the optional CSR term: y = bf16_rne(x . dequant3(Q)^T + x . W_sparse^T).
+ *   The kernel is the 4-bit GEMV's with 24 KB units (12 words a row and group); codes 0..7
+ *   enter the MMA as the exact bf16 values 128 + q, so the arithmetic and the error bound are
+ *   those of w4a16_gemv_ex.  group_size: a multiple of 128 dividing K.  workspace: as for
+ *   w4a16_gemv (w4a16_workspace_bytes).  schedule: as w4a16_gemv_ex.  Errors as w4a16_gemv_ex.
+ *   The prefill GEMM has no 3-bit form (M > 16: W4A16_ERR_SHAPE).
+ */
+w4a16_status w3a16_gemv(const uint16_t* x, const uint32_t* qweight3, const uint16_t* scales,
+                        const uint32_t* zeros, const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N,
+                        int64_t K, int64_t group_size, void* workspace, size_t workspace_bytes, int schedule,
+                        void* stream);
+
 /* w4a16_gemv_folded -- the decode GEMV on the layer input BEFORE the AWQ scaling, as one call.
  * [AWQ translation, 3.2: the weights are multiplied by s and the activations divided by it.]
  *   x   [M][K] bf16 bits, device: the raw layer input.

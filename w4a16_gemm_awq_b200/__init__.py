@@ -6,6 +6,8 @@ mirror the C ABI in include/w4a16.h:
 
   awq_quantize_g128(W, act_absmean, alpha)      -> (qweight, scales, zeros, s)
   awq_quantize(W, act_absmean, alpha, gs)       -> the same with groups of gs along K (gs = K: per row)
+  awq_quantize3(W, act_absmean, alpha, gs=128)  -> the same with 3-bit codes (qweight3 [N][3K/32])
+  w3a16_gemv(x, qweight3, scales, zeros, csr)   -> y      (1 <= M <= 16, 3-bit codes)
   w4a16_linear(x, qweight, scales, zeros, csr)  -> y      (any M)
   w4a16_gemv(...)                               -> y      (1 <= M <= 16)
   w4a16_gemv_ex(..., schedule)                  -> y      (GEMV_AUTO, GEMV_STREAM_K or GEMV_CLUSTER)
@@ -67,6 +69,9 @@ def lib() -> ctypes.CDLL:
         P, I64, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
         L.awq_quantize_g128.argtypes = [P, P, F, I64, I64, P, P, P, P, P]
         L.awq_quantize.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P]
+        L.awq_quantize3.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P]
+        L.w3a16_gemv.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, I64, P, ctypes.c_size_t,
+                                 ctypes.c_int, P]
         L.w4a16_linear_ex.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, I64, P, ctypes.c_size_t,
                                       ctypes.c_int, P]
         for name in ("w4a16_linear", "w4a16_gemv", "w4a16_gemm"):
@@ -123,17 +128,17 @@ def _need(t, dtype, ndim, name):
                          f"{t.dtype} {tuple(t.shape)} on {t.device}")
 
 
-def check_linear_shapes(x, qweight, scales, zeros, csr=None, out=None, group_size: int = 128):
-    """Raise ValueError unless the operands of a linear call agree: x [M][K], qweight [N][K/8],
-    scales [K/gs][N], zeros [K/gs][N/8], csr row_ptr [N+1], out [M][N] bf16.  Shapes only, so
-    a mismatch is reported before anything reaches the library."""
+def check_linear_shapes(x, qweight, scales, zeros, csr=None, out=None, group_size: int = 128, bits: int = 4):
+    """Raise ValueError unless the operands of a linear call agree: x [M][K], qweight [N][K/8]
+    ([N][3K/32] for 3-bit codes), scales [K/gs][N], zeros [K/gs][N/8], csr row_ptr [N+1], out
+    [M][N] bf16.  Shapes only, so a mismatch is reported before anything reaches the library."""
     if x.dim() != 2 or qweight.dim() != 2:
         raise ValueError("x and qweight must be matrices")
     M, K = x.shape
     N = qweight.shape[0]
     gs = int(group_size)
-    if qweight.shape[1] * 8 != K:
-        raise ValueError(f"qweight {tuple(qweight.shape)} does not match K = {K}")
+    if (qweight.shape[1] * 8 != K) if bits == 4 else (qweight.shape[1] * 32 != 3 * K):
+        raise ValueError(f"qweight {tuple(qweight.shape)} does not match K = {K} ({bits}-bit codes)")
     if gs < 1 or K % gs != 0:
         raise ValueError(f"group size {gs} does not divide K = {K}")
     if tuple(scales.shape) != (K // gs, N):
@@ -166,6 +171,26 @@ def awq_quantize(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, group
     code = lib().awq_quantize(_ptr(W), _ptr(act_absmean), ctypes.c_float(alpha), N, K, int(group_size), _ptr(qw),
                               _ptr(sc), _ptr(z), _ptr(s), _stream(dev))
     _check(code, "awq_quantize")
+    return qw, sc, z, s
+
+
+def awq_quantize3(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, group_size: int = 128, out=None):
+    """awq_quantize with 3-bit codes -> (qweight3 int32 [N][3K/32], scales int16 [K/gs][N],
+    zeros int32 [K/gs][N/8] (values 0..7), s fp32 [K])."""
+    _need(W, torch.float32, 2, "W")
+    _need(act_absmean, torch.float32, 1, "act_absmean")
+    N, K = W.shape
+    dev = W.device
+    G = max(K // max(group_size, 1), 1)
+    if out is None:
+        out = (torch.empty(N, max(3 * K // 32, 1), dtype=torch.int32, device=dev),
+               torch.empty(G, N, dtype=torch.int16, device=dev),
+               torch.empty(G, max(N // 8, 1), dtype=torch.int32, device=dev),
+               torch.empty(K, dtype=torch.float32, device=dev))
+    qw, sc, z, s = out
+    code = lib().awq_quantize3(_ptr(W), _ptr(act_absmean), ctypes.c_float(alpha), N, K, int(group_size), _ptr(qw),
+                               _ptr(sc), _ptr(z), _ptr(s), _stream(dev))
+    _check(code, "awq_quantize3")
     return qw, sc, z, s
 
 
@@ -211,8 +236,8 @@ def workspace_bytes(M: int, N: int, K: int, csr: bool = True) -> int:
 
 
 def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, schedule=None, group_size=None,
-            fold=False, s=None):
-    check_linear_shapes(x, qweight, scales, zeros, csr, out, 128 if group_size is None else group_size)
+            fold=False, s=None, bits=4):
+    check_linear_shapes(x, qweight, scales, zeros, csr, out, 128 if group_size is None else group_size, bits)
     _need(x, torch.bfloat16, 2, "x")
     if s is not None:
         _need(s, torch.float32, 1, "s")
@@ -221,8 +246,6 @@ def _linear(name: str, x, qweight, scales, zeros, csr=None, out=None, ws=None, s
     _need(zeros, torch.int32, 2, "zeros")
     M, K = x.shape
     N = qweight.shape[0]
-    if qweight.shape[1] * 8 != K:
-        raise ValueError(f"qweight {tuple(qweight.shape)} does not match K = {K}")
     if s is not None and s.numel() != K:
         raise ValueError(f"s has {s.numel()} entries, K = {K}")
     y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
@@ -264,6 +287,11 @@ def w4a16_linear_ex(x, qweight, scales, zeros, csr=None, out=None, workspace=Non
                     schedule=GEMV_AUTO):
     """w4a16_linear for weights quantized in groups of group_size along K."""
     return _linear("w4a16_linear_ex", x, qweight, scales, zeros, csr, out, workspace, schedule, group_size)
+
+
+def w3a16_gemv(x, qweight3, scales, zeros, csr=None, out=None, workspace=None, group_size=128, schedule=GEMV_AUTO):
+    """The decode GEMV (M <= 16) on 3-bit codes as awq_quantize3 writes them."""
+    return _linear("w3a16_gemv", x, qweight3, scales, zeros, csr, out, workspace, schedule, group_size, bits=3)
 
 
 def w4a16_gemv_folded(x, s, qweight, scales, zeros, csr=None, out=None, workspace=None, group_size=128,

@@ -126,6 +126,7 @@ struct LinearArgs {
     uint16_t* y;
     int64_t M, N, K;
     int group_ratio = 1;  // group size / 128
+    int bits = 4;         // code width: 4, or 3 (qweight [N][3K/32], decode GEMV only)
     float* partials = nullptr;   // the GEMV's scratch (gemv_partial_bytes)
     unsigned* counters = nullptr;  // zero when the call starts (gemv_counter_bytes)
     float* ysp = nullptr;          // the CSR term: decode [N][M], prefill [N][ld] fp32 (only with a CSR)
@@ -181,10 +182,11 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
         EncodeTiledFn enc = nullptr;
         st = encoder(&enc);
         if (st != W4A16_OK) return st;
-        // qweight: 16 words of a group x 128 rows x 4 groups per copy
-        cuuint64_t dims[3] = {16, (cuuint64_t)a.N, (cuuint64_t)(a.K / 128)};
-        cuuint64_t strides[2] = {(cuuint64_t)(a.K / 2), 64};
-        cuuint32_t box[3] = {16, 128, 4};
+        // qweight: the words of a group (16 for 4-bit codes, 12 for 3-bit) x 128 rows x 4 groups
+        const cuuint64_t gw = a.bits == 3 ? 12 : 16;  // words per row and group
+        cuuint64_t dims[3] = {gw, (cuuint64_t)a.N, (cuuint64_t)(a.K / 128)};
+        cuuint64_t strides[2] = {(cuuint64_t)(a.K / 128) * gw * 4, gw * 4};
+        cuuint32_t box[3] = {(cuuint32_t)gw, 128, 4};
         cuuint32_t estr[3] = {1, 1, 1};
         if (enc(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(a.qweight), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -201,7 +203,7 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
         ysp = a.ysp;
     }
     return from_cuda(launch_gemv(maps, plan, a.group_ratio, a.x, a.scales, a.zeros, ysp, a.y, a.partials,
-                                 a.counters, (int)a.M, (int)a.N, (int)a.K, d->status, stream));
+                                 a.counters, (int)a.M, (int)a.N, (int)a.K, d->status, stream, a.bits));
 }
 
 // The decode workspace of the public entry points:
@@ -400,6 +402,39 @@ w4a16_status w4a16_gemv_ex(const uint16_t* x, const uint32_t* qweight, const uin
     if (st != W4A16_OK) return st;
     if (M > 16) return W4A16_ERR_SHAPE;
     if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
+    st = take_decode_workspace(&a, workspace, workspace_bytes, nullptr);
+    if (st != W4A16_OK) return st;
+    return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);
+}
+
+w4a16_status awq_quantize3(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                           int64_t group_size, uint32_t* qweight3, uint16_t* scales, uint32_t* zeros, float* s_out,
+                           void* stream) {
+    if (!W || !act_absmean || !qweight3 || !scales || !zeros) return W4A16_ERR_NULL;
+    if (N < 8 || N % 8 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK) return W4A16_ERR_SHAPE;
+    if (group_size != 128 && group_size != 256 && group_size != 512 && group_size != 1024) return W4A16_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(act_absmean, 16) || !aligned(qweight3, 16) || !aligned(scales, 16) ||
+        !aligned(zeros, 16) || (s_out && !aligned(s_out, 16)))
+        return W4A16_ERR_ALIGN;
+    if (!std::isfinite(alpha)) return W4A16_ERR_VALUE;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    return from_cuda(launch_awq_quantize(W, act_absmean, alpha, (int)N, (int)K, (int)group_size, qweight3, scales,
+                                         zeros, s_out, d->num_sms, d->status, static_cast<cudaStream_t>(stream), 3));
+}
+
+w4a16_status w3a16_gemv(const uint16_t* x, const uint32_t* qweight3, const uint16_t* scales, const uint32_t* zeros,
+                        const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t group_size,
+                        void* workspace, size_t workspace_bytes, int schedule, void* stream) {
+    LinearArgs a;
+    w4a16_status st = validate_linear(x, qweight3, scales, zeros, outliers, y, M, N, K, &a);
+    if (st != W4A16_OK) return st;
+    if (M > 16 || K > gemv_max_k()) return W4A16_ERR_SHAPE;
+    if (group_size < 128 || group_size % 128 != 0 || group_size > K || K % group_size != 0) return W4A16_ERR_SHAPE;
+    if (!valid_schedule(schedule)) return W4A16_ERR_VALUE;
+    a.group_ratio = (int)(group_size / 128);
+    a.bits = 3;
     st = take_decode_workspace(&a, workspace, workspace_bytes, nullptr);
     if (st != W4A16_OK) return st;
     return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);

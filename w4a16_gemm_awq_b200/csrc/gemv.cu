@@ -74,8 +74,15 @@ namespace w4a16 {
 
 constexpr int kGemvRows = 128;                                  // output channels per row block
 constexpr int kGemvUnitGroups = 4;                              // groups of 128 k per work unit
-constexpr int kGemvGroupBytes = kGemvRows * 64;                 // one group of packed weights, 128 rows
-constexpr int kGemvWBytes = kGemvUnitGroups * kGemvGroupBytes;  // 32 KB per unit
+// Packed weights of a unit in shared memory, [4 groups][128 rows][row bytes]: 64 bytes a row
+// and group for 4-bit codes (32 KB a unit), 48 for 3-bit codes (24 KB).
+template <int BITS>
+struct GemvW {
+    static_assert(BITS == 4 || BITS == 3, "4- or 3-bit codes");
+    static constexpr int kRowBytes = 16 * BITS;
+    static constexpr int kGroupBytes = kGemvRows * kRowBytes;
+    static constexpr int kWBytes = kGemvUnitGroups * kGroupBytes;
+};
 constexpr int kGemvConsumers = 8;                               // warps 0..7
 constexpr int kGemvProducer = 12;                               // warp 12
 constexpr int kGemvHelper0 = 8;                                 // warps 8..11, one per SMSP
@@ -102,13 +109,13 @@ struct GemvArgs {
     unsigned* err;
 };
 
-template <int NT>
+template <int NT, int BITS = 4>
 struct GemvSmem {
     static constexpr int kCols = 8 * NT;                                    // token columns
     static constexpr int kXBytes = kGemvUnitGroups * NT * 4 * 32 * 16;      // B fragments of a unit
     static constexpr int kParBytes = kGemvUnitGroups * kGemvRows * 8;       // (s, -(128+z)) per group, row
     static constexpr int kSumBytes = kGemvUnitGroups * 16 * 4;              // X_g per group, token
-    static constexpr int kXOff = kGemvStages * kGemvWBytes;
+    static constexpr int kXOff = kGemvStages * GemvW<BITS>::kWBytes;
     static constexpr int kParOff = kXOff + kGemvStages * kXBytes;
     static constexpr int kSumOff = kParOff + kGemvStages * kParBytes;
     static constexpr int kPartOff = kSumOff + kGemvStages * kSumBytes;      // [128 rows][kCols]
@@ -129,6 +136,32 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t out[4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(out[i]) : "r"(w >> (4 * i)), "r"(0x000F000Fu), "r"(0x43004300u));
+}
+
+// The bf16 pairs of "word" w (0..3) of a thread's 32 codes: for 4-bit codes v holds the 4
+// packed words.  For 3-bit codes v holds the 3 words of the 32 codes: pairs of words 0..2 are
+// their nibbles' low 3 bits, and "word" 3 gathers the bit-3 planes: bit 4i + 3 of word b is
+// bit b of the codes of nibbles i and i + 4 of the fourth 8-code block.
+template <int BITS>
+__device__ __forceinline__ void unpack_codes(const uint4& v, int w, uint32_t out[4]) {
+    if constexpr (BITS == 4) {
+        unpack_word(u4_get(v, w), out);
+    } else if (w < 3) {
+        const uint32_t word = u4_get(v, w);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(out[i]) : "r"(word >> (4 * i)), "r"(0x00070007u),
+                "r"(0x43004300u));
+    } else {
+        // gather the three bit-3 planes into one word whose nibble j is the code of element
+        // 24 + ORDER[j], then unpack it like a 4-bit word: 6 operations for the planes and 2
+        // per pair, instead of 7 per pair
+        uint32_t p;
+        asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(p) : "r"(v.x >> 3), "r"(0x11111111u),
+            "r"((v.y >> 2) & 0x22222222u));
+        asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(p) : "r"(v.z >> 1), "r"(0x44444444u), "r"(p));
+        unpack_word(p, out);
+    }
 }
 
 // Next unit of a CTA's walk: gb runs over [kb, ke) within a row block, then the walk moves
@@ -199,10 +232,11 @@ __device__ __forceinline__ bool gather_other(const GemvArgs& p, int rb, int GB, 
     return true;
 }
 
-template <int NT>
+template <int NT, int BITS>
 __global__ void __launch_bounds__(kGemvThreads, 1)
 gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
-    using L = GemvSmem<NT>;
+    using L = GemvSmem<NT, BITS>;
+    constexpr int kWBytes = GemvW<BITS>::kWBytes;
     constexpr int S = kGemvStages;
     constexpr int C = L::kCols;
     // Pointers into shared memory derive from the array itself (no integer round trip), so the
@@ -262,8 +296,8 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
         fence_mbarrier_init();
         fence_proxy_async_smem();
         for (; pre < S && pre < n; ++pre, walk_next(prb, pgb, kb, ke, step)) {
-            mbar_arrive_expect_tx(&wfull[pre], (uint32_t)kGemvWBytes);
-            tma_load_3d(smem + pre * kGemvWBytes, &map_w, &wfull[pre], 0, prb * kGemvRows, pgb * kGemvUnitGroups);
+            mbar_arrive_expect_tx(&wfull[pre], (uint32_t)kWBytes);
+            tma_load_3d(smem + pre * kWBytes, &map_w, &wfull[pre], 0, prb * kGemvRows, pgb * kGemvUnitGroups);
         }
     }
     // the other barriers, one per thread, so that the prologue is short
@@ -297,8 +331,8 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                     record_error(p.err, kErrTimeout);
                     break;
                 }
-                mbar_arrive_expect_tx(&wfull[slot], (uint32_t)kGemvWBytes);
-                tma_load_3d(smem + slot * kGemvWBytes, &map_w, &wfull[slot], 0, prb * kGemvRows, pgb * kGemvUnitGroups);
+                mbar_arrive_expect_tx(&wfull[slot], (uint32_t)kWBytes);
+                tma_load_3d(smem + slot * kWBytes, &map_w, &wfull[slot], 0, prb * kGemvRows, pgb * kGemvUnitGroups);
                 ++issued;
             }
             // the copies this CTA started must land before it may exit
@@ -417,16 +451,23 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
                 if (lane == 0) record_error(p.err, kErrTimeout);
                 break;
             }
-            const uint8_t* ws = smem + slot * kGemvWBytes;
+            const uint8_t* ws = smem + slot * kWBytes;
             uint4 wv[2][2][2];  // [group][tile i][row half hh]
 #pragma unroll
             for (int gg = 0; gg < 2; ++gg)
 #pragma unroll
                 for (int i = 0; i < 2; ++i)
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
-                        wv[gg][i][hh] = *reinterpret_cast<const uint4*>(
-                            ws + (2 * half + gg) * kGemvGroupBytes + (rbase + 16 * i + 8 * hh) * 64 + 16 * t);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint8_t* src = ws + (2 * half + gg) * GemvW<BITS>::kGroupBytes +
+                                             (rbase + 16 * i + 8 * hh) * GemvW<BITS>::kRowBytes;
+                        if constexpr (BITS == 4) {
+                            wv[gg][i][hh] = *reinterpret_cast<const uint4*>(src + 16 * t);
+                        } else {  // the thread's 3 words of 32 codes
+                            const uint32_t* s3 = reinterpret_cast<const uint32_t*>(src + 12 * t);
+                            wv[gg][i][hh] = make_uint4(s3[0], s3[1], s3[2], 0u);
+                        }
+                    }
             __syncwarp();
             if (lane == 0) mbar_arrive(&wempty[slot]);
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(&xfull[slot], (s / S) & 1))) {
@@ -458,8 +499,8 @@ gemv_w4a16_kernel(const __grid_constant__ CUtensorMap map_w, const GemvArgs p) {
 #pragma unroll
                         for (int i = 0; i < 2; ++i) {
                             uint32_t pa0[4], pa1[4];
-                            unpack_word(u4_get(wv[pass * GI + g2][i][0], w), pa0);
-                            unpack_word(u4_get(wv[pass * GI + g2][i][1], w), pa1);
+                            unpack_codes<BITS>(wv[pass * GI + g2][i][0], w, pa0);
+                            unpack_codes<BITS>(wv[pass * GI + g2][i][1], w, pa1);
 #pragma unroll
                             for (int hh = 0; hh < 2; ++hh) {
                                 const uint32_t A[4] = {pa0[2 * hh], pa1[2 * hh], pa0[2 * hh + 1], pa1[2 * hh + 1]};
@@ -829,8 +870,9 @@ int max_active_clusters(bool two, int cl) {
     std::atomic<int>& slot = cache[dev][two ? 1 : 0][cl];
     int v = slot.load(std::memory_order_relaxed);
     if (v >= 0) return v;
-    const int smem = two ? GemvSmem<2>::kBytes : GemvSmem<1>::kBytes;
-    const void* fn = two ? (const void*)gemv_w4a16_kernel<2> : (const void*)gemv_w4a16_kernel<1>;
+    // the 4-bit kernel's figures; the 3-bit one needs less shared memory, so they hold for it too
+    const int smem = two ? GemvSmem<2, 4>::kBytes : GemvSmem<1, 4>::kBytes;
+    const void* fn = two ? (const void*)gemv_w4a16_kernel<2, 4> : (const void*)gemv_w4a16_kernel<1, 4>;
     v = 0;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
@@ -885,10 +927,33 @@ GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule) {
     return best;
 }
 
+template <int NT, int BITS>
+static cudaError_t launch_gemv_kernel(const GemvMaps& maps, const GemvPlan& plan, const GemvArgs& a,
+                                      cudaStream_t stream) {
+    const int smem = GemvSmem<NT, BITS>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(gemv_w4a16_kernel<NT, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.P, 1, 1);
+    cfg.blockDim = dim3(kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = plan.cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = plan.cluster != 0 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<NT, BITS>, maps.w, a);
+}
+
 cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
                         const uint16_t* scales, const uint32_t* zeros, const float* ysp, uint16_t* y,
                         float* partials, unsigned* counters, int M, int N, int K, unsigned* err,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, int bits) {
     GemvArgs a{};
     a.x = x;
     a.scales = scales;
@@ -909,26 +974,9 @@ cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ra
     a.counters = counters;
 
     const bool two = M > 8;
-    const int smem = two ? GemvSmem<2>::kBytes : GemvSmem<1>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(two ? gemv_w4a16_kernel<2> : gemv_w4a16_kernel<1>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.P, 1, 1);
-    cfg.blockDim = dim3(kGemvThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = plan.cluster;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = plan.cluster != 0 ? 2 : 1;
-    if (two) return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<2>, maps.w, a);
-    return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<1>, maps.w, a);
+    if (bits == 3) return two ? launch_gemv_kernel<2, 3>(maps, plan, a, stream) : launch_gemv_kernel<1, 3>(maps, plan, a, stream);
+    if (bits != 4) return cudaErrorInvalidValue;
+    return two ? launch_gemv_kernel<2, 4>(maps, plan, a, stream) : launch_gemv_kernel<1, 4>(maps, plan, a, stream);
 }
 
 }  // namespace w4a16

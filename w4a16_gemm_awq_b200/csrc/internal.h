@@ -17,13 +17,16 @@ enum : unsigned { kErrValue = 1u, kErrShape = 2u, kErrTimeout = 4u };
 constexpr int kQuantMaxLargeGroup = 32768;
 bool quantize_group_size_ok(int K, int gs);
 
+// bits: 4 (qweight [N][K/8]) or 3 (qweight [N][3K/32], group sizes up to 1024; see quantize.cu).
 cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, int gs,
                                 uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, int num_sms,
-                                unsigned* err, cudaStream_t stream);
+                                unsigned* err, cudaStream_t stream, int bits = 4);
 
 // Tensor map the GEMV needs: qweight uint32 [N][K/8] seen as 3-D (16 words of a group,
 // N rows, K/128 groups; strides K/2 and 64 bytes), box 16 x 128 x 4, no swizzle.  One copy
 // brings 4 groups of 128 rows and lays them out group by group: [4][128 rows][64 bytes].
+// For 3-bit codes: qweight [N][3K/32] as (12 words, N, K/128; strides 3K/8 and 48 bytes),
+// box 12 x 128 x 4: [4][128 rows][48 bytes].
 struct GemvMaps {
     CUtensorMap w;
 };
@@ -58,10 +61,11 @@ GemvPlan gemv_plan(int M, int N, int K, int num_sms, int schedule);
 // group_ratio: the quantization group size / 128 (1 for g128; K / 128 for one group per row).
 // ysp: nullptr, or the CSR term [N][M] fp32 written by launch_csr_rows just before (the GEMV
 // adds it to each output before rounding, after the previous kernel has finished).
+// bits: 4, or 3 for 3-bit codes (qweight [N][3K/32], the map's inner extent 12 words a group).
 cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ratio, const uint16_t* x,
                         const uint16_t* scales, const uint32_t* zeros, const float* ysp, uint16_t* y,
                         float* partials, unsigned* counters, int M, int N, int K, unsigned* err,
-                        cudaStream_t stream);
+                        cudaStream_t stream, int bits = 4);
 
 // The CSR term of the decode path: ysp[n][m] = sum_j float(val_j) * float(x[m][col_j]) over
 // row n's entries, in fp32 (see csr.cu).  1 <= M <= 16.  The next kernel on the stream may

@@ -74,11 +74,12 @@ __device__ __forceinline__ float min_nan(float a, float b) {
     return r;
 }
 
-// The 4-bit code of w' in a group with scale sf (y = RN(1/sf)) and integer zero point z:
-// clamp(rint(w' / sf) + z, 0, 15), for |w' / sf| < 2^21.
+// The code of w' in a group with scale sf (y = RN(1/sf)) and integer zero point z:
+// clamp(rint(w' / sf) + z, 0, qmax), for |w' / sf| < 2^21 (qmax = 15 for 4-bit codes, 7 for 3-bit).
+template <int QMAX>
 __device__ __forceinline__ uint32_t code_of(float w, float sf, float y, int z) {
     const int t = rint_int(quotient_markstein(w, sf, y)) + z;
-    return (uint32_t)min(max(t, 0), 15);
+    return (uint32_t)min(max(t, 0), QMAX);
 }
 
 // the integer value of an integral float in [0, 2^22)
@@ -119,13 +120,19 @@ __device__ __forceinline__ constexpr int nibble_of(int e) { return (e & 1) ? 4 +
 // Groups of 128 R weights, R in {1, 2, 4, 8}: a 1024-column chunk holds 8 / R whole groups.
 // A CTA takes ROWS (32 or 64) rows.  s_pre: the channel scales computed by awq_scale_kernel
 // just before (read after it has finished), or nullptr: the CTA computes the s of its columns.
-template <int R, int ROWS>
+// BITS = 4: codes 0..15, 8 per word, qweight [N][K/8].  BITS = 3 (SqueezeLLM article,
+// sections 2.1-2.2: eight levels): codes 0..7, the 32 codes of k = 32b .. 32b + 31 in the
+// three words qweight[n][3b + w]: bits 4j .. 4j+2 of word w hold element 8w + ORDER[j], bit
+// 4j + 3 holds bit w of element 24 + ORDER[j]; qweight [N][3K/32].
+template <int R, int ROWS, int BITS>
 __global__ void __launch_bounds__(kQuantThreads, W4A16_QUANT_CTAS_PER_SM)
 awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, const float* s_pre, float alpha,
                     int N, int K, uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales,
                     uint32_t* __restrict__ zeros, unsigned* err) {
     constexpr int GC = 8 / R;  // groups per chunk
     constexpr int LG = 4 * R;  // lanes per group
+    constexpr int QMAX = BITS == 4 ? 15 : 7;
+    static_assert(BITS == 4 || BITS == 3, "4- or 3-bit codes");
     // s of the chunk, lane l's 32 values in 8 16-byte pieces, piece c at l*128 + 16 (c ^ (l & 7)),
     // so that a quarter warp's 16-byte reads hit 8 different bank groups
     __shared__ __align__(16) float s_sm[1024];
@@ -196,13 +203,13 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
             mn = min_nan(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         }
         const bool bad_range = !isfinite(mx) || !isfinite(mn);  // NaN or Inf anywhere in the group
-        float scale32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+        float scale32 = __fdiv_rn(__fsub_rn(mx, mn), (float)QMAX);
         if (scale32 < 1e-5f) scale32 = 1e-5f;
         const __half h = __float2half_rn(scale32);
         const float sf = __half2float(h);
         const bool bad = bad_range || isinf(scale32) || isinf(sf);
         float zf = rintf(__fdiv_rn(-mn, sf));
-        zf = fminf(fmaxf(zf, 0.0f), 15.0f);
+        zf = fminf(fmaxf(zf, 0.0f), (float)QMAX);
         const int zi = (int)int_bits(zf);
         const float y = __frcp_rn(sf);
         // |w' / sf| < 2^20 for the whole group: no clamp before dividing
@@ -212,16 +219,32 @@ awq_quantize_kernel(const float* __restrict__ W, const float* __restrict__ act, 
 #pragma unroll
             for (int i = 0; i < 32; ++i) w[i] = fminf(fmaxf(w[i], -lim), lim);
         }
-        uint32_t word[4];
+        if constexpr (BITS == 4) {
+            uint32_t word[4];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            uint32_t acc = 0;
+            for (int b = 0; b < 4; ++b) {
+                uint32_t acc = 0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc |= code_of(w[8 * b + e], sf, y, zi) << (4 * nibble_of(e));
-            word[b] = acc;
+                for (int e = 0; e < 8; ++e) acc |= code_of<QMAX>(w[8 * b + e], sf, y, zi) << (4 * nibble_of(e));
+                word[b] = acc;
+            }
+            *reinterpret_cast<uint4*>(qweight + (size_t)n * (K >> 3) + (size_t)kc * 128 + 4 * lane) =
+                make_uint4(word[0], word[1], word[2], word[3]);
+        } else {
+            uint32_t word[3] = {0u, 0u, 0u};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int j = nibble_of(e);
+                const uint32_t hi = code_of<QMAX>(w[24 + e], sf, y, zi);  // its 3 bits go to the 3 words
+#pragma unroll
+                for (int b = 0; b < 3; ++b)
+                    word[b] |= (code_of<QMAX>(w[8 * b + e], sf, y, zi) | (((hi >> b) & 1u) << 3)) << (4 * j);
+            }
+            uint32_t* dst = qweight + (size_t)n * (3 * (K >> 5)) + (size_t)kc * 96 + 3 * lane;
+            dst[0] = word[0];
+            dst[1] = word[1];
+            dst[2] = word[2];
         }
-        *reinterpret_cast<uint4*>(qweight + (size_t)n * (K >> 3) + (size_t)kc * 128 + 4 * lane) =
-            make_uint4(word[0], word[1], word[2], word[3]);
         if ((lane & (LG - 1)) == 0) {
             sc_sm[lane / LG][r] = __half_as_ushort(h);
             zc_sm[lane / LG][r] = (uint8_t)zi;
@@ -357,8 +380,9 @@ bool quantize_group_size_ok(int K, int gs) {
 
 cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, int N, int K, int gs,
                                 uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, int num_sms,
-                                unsigned* err, cudaStream_t stream) {
-    if (!quantize_group_size_ok(K, gs)) return cudaErrorInvalidValue;
+                                unsigned* err, cudaStream_t stream, int bits) {
+    if (!quantize_group_size_ok(K, gs) || (bits != 4 && bits != 3) || (bits == 3 && gs > 1024))
+        return cudaErrorInvalidValue;
     if (gs > 1024) {
         const int smem = gs * 4;
         cudaError_t e = cudaFuncSetAttribute(awq_quantize_large_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -372,10 +396,20 @@ cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, i
     // 64-row tiles, or 32-row ones when 64-row tiles would not fill the resident CTA slots twice
     const bool small = (long long)(K / 1024) * ((N + 63) / 64) < 2LL * W4A16_QUANT_CTAS_PER_SM * num_sms;
     const int rows = small ? 32 : 64;
-    auto* kernel = small ? (gs == 128 ? awq_quantize_kernel<1, 32> : gs == 256 ? awq_quantize_kernel<2, 32>
-                            : gs == 512 ? awq_quantize_kernel<4, 32> : awq_quantize_kernel<8, 32>)
-                         : (gs == 128 ? awq_quantize_kernel<1, 64> : gs == 256 ? awq_quantize_kernel<2, 64>
-                            : gs == 512 ? awq_quantize_kernel<4, 64> : awq_quantize_kernel<8, 64>);
+    using Kernel = void (*)(const float*, const float*, const float*, float, int, int, uint32_t*, uint16_t*,
+                            uint32_t*, unsigned*);
+    static const Kernel k4[2][4] = {
+        {awq_quantize_kernel<1, 64, 4>, awq_quantize_kernel<2, 64, 4>, awq_quantize_kernel<4, 64, 4>,
+         awq_quantize_kernel<8, 64, 4>},
+        {awq_quantize_kernel<1, 32, 4>, awq_quantize_kernel<2, 32, 4>, awq_quantize_kernel<4, 32, 4>,
+         awq_quantize_kernel<8, 32, 4>}};
+    static const Kernel k3[2][4] = {
+        {awq_quantize_kernel<1, 64, 3>, awq_quantize_kernel<2, 64, 3>, awq_quantize_kernel<4, 64, 3>,
+         awq_quantize_kernel<8, 64, 3>},
+        {awq_quantize_kernel<1, 32, 3>, awq_quantize_kernel<2, 32, 3>, awq_quantize_kernel<4, 32, 3>,
+         awq_quantize_kernel<8, 32, 3>}};
+    const int ri = gs == 128 ? 0 : gs == 256 ? 1 : gs == 512 ? 2 : 3;
+    const Kernel kernel = (bits == 4 ? k4 : k3)[small ? 1 : 0][ri];
     const dim3 grid(K / 1024, (N + rows - 1) / rows);
     if (s_out == nullptr) {
         kernel<<<grid, kQuantThreads, 0, stream>>>(W, act, nullptr, alpha, N, K, qweight, scales, zeros, err);
