@@ -33,6 +33,8 @@
 //     The epilogue waits for them and adds ysp to the fp32 sum before the one rounding.
 //   - Every mbarrier wait is bounded.  On timeout the CTA records kErrTimeout, stops its
 //     loops, drains its own TMA and MMA work with bounded waits, and frees its TMEM.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -51,7 +53,7 @@ struct GemmArgs {
     const float* ysp;  // the CSR term [N][ysp_ld] fp32, or nullptr
     int ysp_ld;
     uint16_t* y;
-    float* partials;    // split-K: fp32 tiles [tile][split][128][BN]
+    float* partials;    // split-K: fp32 tiles [tile][split][BN tokens][128 rows]
     unsigned* counters; // split-K: one per tile, zero between calls
     int M, N, K;
     int gr;      // quantization group size / 128: scales and zeros of 128-slice g are those of group g / gr
@@ -270,18 +272,16 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             const int z = (int)blockIdx.z;
             bool last = true;
             if (p.splits > 1) {
-                // this CTA's partial tile, row by row: thread `row` writes BN contiguous floats
-                float* mine = p.partials + ((tile * p.splits + z) * 128 + row) * BN;
+                // this CTA's partial tile, token-major ([BN][128]): for each token the 32 lanes of a
+                // warp write 32 consecutive floats, so every store is one coalesced 128-byte line
+                float* mine = p.partials + (tile * p.splits + z) * 128 * BN + row;
 #pragma unroll 1
                 for (int c0 = 0; c0 < BN; c0 += 32) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tmem + t_lane + (uint32_t)c0, r);
                     tmem_ld_wait();
-                    float4* dst = reinterpret_cast<float4*>(mine + c0);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                             __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                    for (int j = 0; j < 32; ++j) __stcg(mine + (c0 + j) * 128, __uint_as_float(r[j]));
                 }
                 __threadfence();
                 epilogue_sync();
@@ -336,13 +336,9 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
 #pragma unroll
                                 for (int j = 0; j < 32; ++j) v[j] = own[j];
                             } else {
-                                const float4* src = reinterpret_cast<const float4*>(
-                                    p.partials + ((tile * p.splits + zz) * 128 + row) * BN + c0);
+                                const float* src = p.partials + (tile * p.splits + zz) * 128 * BN + c0 * 128 + row;
 #pragma unroll
-                                for (int q = 0; q < 8; ++q) {
-                                    const float4 f = __ldcg(src + q);
-                                    v[4 * q] = f.x, v[4 * q + 1] = f.y, v[4 * q + 2] = f.z, v[4 * q + 3] = f.w;
-                                }
+                                for (int j = 0; j < 32; ++j) v[j] = __ldcg(src + j * 128);
                             }
 #pragma unroll
                             for (int j = 0; j < 32; ++j) acc[j] = zz == 0 ? v[j] : acc[j] + v[j];
@@ -400,21 +396,22 @@ GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
     const int64_t nslices = K / 128;
     g.splits = 1;
     g.slices = (int)nslices;
-    // Time model in slices: waves x slices per CTA, plus about one slice per extra partial tile
-    // of 256 tokens that the last CTA reads back.  Only grids of under two waves are split
-    // (larger ones lose little to their last wave), only while the partial tiles stay within
-    // kMaxGemmPartialBytes, and only into runs of at least min_per slices: measured on
-    // B200, wide token tiles (whose CTAs each stream a large x tile) gained nothing from runs
-    // shorter than 32 slices (4096 x 4096 at M = 512), narrow ones gained down to runs of 8.
-    const int64_t min_per = g.bn == 256 ? 32 : g.bn == 128 ? 16 : 4;
+    // Time model in slices: the longer of one CTA's run and the grid's total work spread over
+    // the SMs, plus the split's own cost (partial tiles written and read back), about half a
+    // slice per extra split and 64 tokens.  Only grids of under two waves are split, and only
+    // while the partial tiles stay within kMaxGemmPartialBytes.  Measured on B200, 256-token
+    // tiles lose when the split grid needs a second wave (their CTAs' partial tiles, 128 KB
+    // each, cost several microseconds to write and read back), so those split only within
+    // one wave.
     if (tiles < 2 * (int64_t)num_sms && tiles <= kMaxGemmTiles) {
-        double best = (double)nslices;
+        const double sms = (double)num_sms;
+        double best = std::max((double)nslices, (double)(tiles * nslices) / sms);
         for (int S = 2; S <= kMaxGemmSplits; ++S) {
             const int64_t per = (nslices + S - 1) / S;
             const int64_t used = (nslices + per - 1) / per;  // no empty split
-            if (used != S || per < min_per || (size_t)tiles * S * 128 * g.bn * 4 > kMaxGemmPartialBytes) continue;
-            const int64_t waves = (tiles * S + num_sms - 1) / num_sms;
-            const double cost = (double)(waves * per) + (double)(S - 1) * g.bn / 256.0;
+            if (used != S || per < 4 || (size_t)tiles * S * 128 * g.bn * 4 > kMaxGemmPartialBytes) continue;
+            if (g.bn == 256 && tiles * S > num_sms) continue;
+            const double cost = std::max((double)per, (double)(tiles * S * per) / sms) + 0.5 * (S - 1) * g.bn / 64.0;
             if (cost < best - 0.5) {
                 best = cost;
                 g.splits = S;
