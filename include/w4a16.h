@@ -125,7 +125,7 @@ w4a16_status awq_quantize(const float* W, const float* act_absmean, float alpha,
  *   - Decode path (M <= 16).  The GEMV splits the output row blocks evenly over a
  *     persistent grid.  Row blocks shared by two or more CTAs are combined through fp32
  *     partial tiles and per-row-block counters; w4a16_gemv_folded also writes its x / s
- *     there, and a CSR term goes there as N x M fp32.
+ *     there, and a CSR term goes there as N x M fp32 (with x transposed beside it).
  *   - Prefill path (the GEMM).  When the output tiles alone would leave SMs idle, the GEMM
  *     splits K over several CTAs per tile; their fp32 partial tiles and per-tile counters
  *     live in the workspace.  With a CSR term, x transposed (K x M' bf16) and the term
@@ -141,7 +141,8 @@ w4a16_status awq_quantize(const float* W, const float* act_absmean, float alpha,
  *   - After a call reports W4A16_ERR_TIMEOUT, zero the workspace again before reusing it.
  * Both functions return the size for the CURRENT device (it depends on the number of SMs),
  * or 0 for invalid sizes.  Decode: 128 KiB of counters, 16 KiB of partial tiles per SM,
- * M x K bf16 for the folded activations and N x M fp32 for the CSR term.  Prefill: 128 KiB
+ * M x K bf16 for the folded activations, N x M fp32 for the CSR term and K x 16 bf16 for
+ * the activations transposed for it.  Prefill: 128 KiB
  * of counters, the split-K partial tiles (none for grids that fill the GPU, else about
  * splits x M x N x 4 bytes, at most 64 MiB), then the CSR parts above.  Each part is
  * rounded up to 256 bytes.
@@ -308,7 +309,7 @@ w4a16_status w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16
  *   - Arguments, result and limits are those of w4a16_gemv, minus the workspace.
  *     N <= 131072 and at most 160 SMs on the device; otherwise W4A16_ERR_UNSUPPORTED.
  *   - With a CSR term, N x M <= 262144 as well (UNSUPPORTED otherwise).
- *   - Its scratch is a static device array of about 3.6 MiB inside the library.  Every GPU
+ *   - Its scratch is a static device array of about 3.5 MiB inside the library.  Every GPU
  *     that loads the library holds one until the process exits.  The call allocates
  *     nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - The first call on a device looks up the array's device address

@@ -130,7 +130,7 @@ struct LinearArgs {
     float* partials = nullptr;   // the GEMV's scratch (gemv_partial_bytes)
     unsigned* counters = nullptr;  // zero when the call starts (gemv_counter_bytes)
     float* ysp = nullptr;          // the CSR term: decode [N][M], prefill [N][ld] fp32 (only with a CSR)
-    uint16_t* xT = nullptr;        // prefill with a CSR: x transposed, [K][ld] bf16
+    uint16_t* xT = nullptr;        // with a CSR: x transposed, [K][ld] bf16 (decode: nullptr gathers from x)
 };
 
 w4a16_status validate_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
@@ -197,8 +197,10 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
     if (a.row_ptr != nullptr) {
         // the sparse term first, into the workspace; the GEMV streams its weights meanwhile
         if (a.ysp == nullptr) return W4A16_ERR_NULL;
-        st = from_cuda(launch_csr_rows(a.x, a.row_ptr, a.col_idx, a.vals, a.nnz, (int)a.M, (int)a.N, (int)a.K, a.ysp,
-                                       d->status, stream));
+        // x transposed first when an entry's tokens would otherwise be several scattered loads
+        uint16_t* xT = a.M > 2 ? a.xT : nullptr;
+        st = from_cuda(launch_csr_rows(a.x, xT, a.row_ptr, a.col_idx, a.vals, a.nnz, (int)a.M, (int)a.N, (int)a.K,
+                                       a.ysp, d->status, stream));
         if (st != W4A16_OK) return st;
         ysp = a.ysp;
     }
@@ -210,14 +212,17 @@ w4a16_status run_gemv(const LinearArgs& a, cudaStream_t stream, int schedule = W
 //   [0, kCounterRegionBytes)   the GEMV's row-block counters (zero between calls);
 //   then gemv_partial_bytes    its fp32 partial tiles;
 //   then M x K bf16            x / s of w4a16_gemv_folded, rounded up to 256 bytes;
-//   then N x M fp32            the CSR term, rounded up to 256 bytes.
+//   then N x M fp32            the CSR term, rounded up to 256 bytes;
+//   then K x 16 bf16           x transposed for the CSR term, rounded up to 256 bytes.
 // Only the last two parts depend on the call's sizes, and they lie after everything that must
 // stay zero, so one zeroed workspace serves calls of any sizes in stream order.
 size_t fold_region_bytes(int64_t M, int64_t K) { return ((size_t)M * (size_t)K * 2 + 255) / 256 * 256; }
 size_t csr_region_bytes(int64_t M, int64_t N) { return ((size_t)M * (size_t)N * 4 + 255) / 256 * 256; }
+size_t xt_region_bytes(int64_t K) { return ((size_t)K * 16 * 2 + 255) / 256 * 256; }
 
 size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
-    return kCounterRegionBytes + gemv_partial_bytes(num_sms) + fold_region_bytes(M, K) + csr_region_bytes(M, N);
+    return kCounterRegionBytes + gemv_partial_bytes(num_sms) + fold_region_bytes(M, K) + csr_region_bytes(M, N) +
+           xt_region_bytes(K);
 }
 
 // Checks the caller's decode workspace and points a at its parts; *fold = the x / s region.
@@ -234,6 +239,7 @@ w4a16_status take_decode_workspace(LinearArgs* a, void* workspace, size_t worksp
     a->partials = reinterpret_cast<float*>(ws + kCounterRegionBytes);
     if (fold) *fold = reinterpret_cast<uint16_t*>(ws + fold_off);
     a->ysp = reinterpret_cast<float*>(ws + fold_off + fold_region_bytes(a->M, a->K));
+    a->xT = reinterpret_cast<uint16_t*>(ws + fold_off + fold_region_bytes(a->M, a->K) + csr_region_bytes(a->M, a->N));
     return W4A16_OK;
 }
 

@@ -17,7 +17,10 @@
 // bits).  The 32 partial sums of each token are then added by a butterfly (xor 16, 8, 4, 2, 1),
 // whose order is fixed, so every call gives the same bits.  Lane m writes token m.  CTAs are
 // 4 warps, small enough in registers that many fit beside each other and the whole grid
-// starts at once.
+// starts at once.  With a workspace, x is first transposed (xT[k][m], token stride 8 or 16,
+// the transpose kernel below), so an entry's tokens are one 16- or 32-byte load instead of M
+// loads from M rows of x; without one (w4a16_gemv_noalloc) the kernel gathers from x.  Both
+// read the same values in the same order and give the same bits.
 //
 // Prefill (M > 16): the same term for many tokens.  Gathering x[m][col] for a fixed column
 // over many tokens would touch one 32-byte sector per token, so x is first transposed into
@@ -36,7 +39,8 @@ namespace w4a16 {
 constexpr int kCsrWarps = 4;  // warps (rows) per CTA of the decode kernel
 
 __global__ void __launch_bounds__(32 * kCsrWarps)
-csr_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+csr_rows_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ xT, int ld,
+                const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
                 const uint16_t* __restrict__ vals, long long nnz, int M, int N, int K, float* __restrict__ ysp,
                 unsigned* err) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -69,9 +73,21 @@ csr_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ row_
             record_error(err, kErrShape);
             continue;
         }
+        if (xT != nullptr) {  // the entry's tokens, contiguous (ld = 8 or 16)
+            uint4 q[2];
+            q[0] = __ldg(reinterpret_cast<const uint4*>(xT + (size_t)c * ld));
+            q[1] = ld > 8 ? __ldg(reinterpret_cast<const uint4*>(xT + (size_t)c * ld + 8)) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int m = 0; m < 16; ++m)
-            if (m < M) acc[m] = fmaf(v, bf16_bits_to_float(__ldg(x + (size_t)m * K + c)), acc[m]);
+            for (int m = 0; m < 16; ++m) {
+                const uint32_t pr = u4_get(q[m >> 3], (m & 7) >> 1);
+                const float xv = __uint_as_float((m & 1) ? (pr & 0xFFFF0000u) : (pr << 16));
+                if (m < M) acc[m] = fmaf(v, xv, acc[m]);
+            }
+        } else {
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+                if (m < M) acc[m] = fmaf(v, bf16_bits_to_float(__ldg(x + (size_t)m * K + c)), acc[m]);
+        }
     }
     float mine = 0.0f;
 #pragma unroll
@@ -86,8 +102,16 @@ csr_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ row_
     if (lane < M) ysp[(size_t)n * M + lane] = mine;
 }
 
-cudaError_t launch_csr_rows(const uint16_t* x, const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals,
-                            long long nnz, int M, int N, int K, float* ysp, unsigned* err, cudaStream_t stream) {
+cudaError_t launch_transpose_x(const uint16_t* x, uint16_t* xT, int M, int K, int ld, bool pdl, cudaStream_t stream);
+
+cudaError_t launch_csr_rows(const uint16_t* x, uint16_t* xT, const int32_t* row_ptr, const int32_t* col_idx,
+                            const uint16_t* vals, long long nnz, int M, int N, int K, float* ysp, unsigned* err,
+                            cudaStream_t stream) {
+    const int ld = csr_token_stride(M);
+    if (xT != nullptr) {
+        cudaError_t e = launch_transpose_x(x, xT, M, K, ld, true, stream);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((N + kCsrWarps - 1) / kCsrWarps), 1, 1);
     cfg.blockDim = dim3(32 * kCsrWarps, 1, 1);
@@ -97,14 +121,18 @@ cudaError_t launch_csr_rows(const uint16_t* x, const int32_t* row_ptr, const int
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, csr_rows_kernel, x, row_ptr, col_idx, vals, nnz, M, N, K, ysp, err);
+    return cudaLaunchKernelEx(&cfg, csr_rows_kernel, x, (const uint16_t*)xT, ld, row_ptr, col_idx, vals, nnz, M, N, K,
+                              ysp, err);
 }
 
 // xT[k][m] = x[m][k] for m < M; xT has ld (>= M, a multiple of 8) elements per row.  32 x 32
-// tiles through shared memory, so both the reads and the writes are coalesced.
+// tiles through shared memory, so both the reads and the writes are coalesced.  It reads x
+// only after the previous kernel on the stream has finished (a no-op when launched without
+// programmatic dependent launch).
 __global__ void __launch_bounds__(256)
 transpose_x_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xT, int M, int K, int ld) {
     __shared__ uint16_t tile[32][33];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int k0 = blockIdx.x * 32, m0 = blockIdx.y * 32;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of 32 per pass
 #pragma unroll
@@ -178,9 +206,7 @@ cudaError_t launch_csr_prefill(const uint16_t* x, const int32_t* row_ptr, const 
                                long long nnz, int M, int N, int K, uint16_t* xT, float* ysp, unsigned* err,
                                cudaStream_t stream) {
     const int ld = csr_token_stride(M);
-    dim3 tgrid(K / 32, (ld + 31) / 32);
-    transpose_x_kernel<<<tgrid, 256, 0, stream>>>(x, xT, M, K, ld);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_transpose_x(x, xT, M, K, ld, false, stream);
     if (e != cudaSuccess) return e;
     const long long warps = (long long)N * ((M + kSpmmTokens - 1) / kSpmmTokens);
     cudaLaunchConfig_t cfg = {};
@@ -194,6 +220,19 @@ cudaError_t launch_csr_prefill(const uint16_t* x, const int32_t* row_ptr, const 
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, csr_spmm_kernel, (const uint16_t*)xT, row_ptr, col_idx, vals, nnz, M, N, K, ld, ysp,
                               err);
+}
+
+cudaError_t launch_transpose_x(const uint16_t* x, uint16_t* xT, int M, int K, int ld, bool pdl, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(K / 32, (ld + 31) / 32, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, transpose_x_kernel, x, xT, M, K, ld);
 }
 
 }  // namespace w4a16

@@ -70,8 +70,11 @@ cudaError_t launch_gemv(const GemvMaps& maps, const GemvPlan& plan, int group_ra
 // The CSR term of the decode path: ysp[n][m] = sum_j float(val_j) * float(x[m][col_j]) over
 // row n's entries, in fp32 (see csr.cu).  1 <= M <= 16.  The next kernel on the stream may
 // start while it runs (programmatic dependent launch) and must wait for it before reading ysp.
-cudaError_t launch_csr_rows(const uint16_t* x, const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* vals,
-                            long long nnz, int M, int N, int K, float* ysp, unsigned* err, cudaStream_t stream);
+// xT: nullptr, or room for x transposed ([K][csr_token_stride(M)] bf16, written first by a
+// transpose kernel) so that each entry's tokens are one load.
+cudaError_t launch_csr_rows(const uint16_t* x, uint16_t* xT, const int32_t* row_ptr, const int32_t* col_idx,
+                            const uint16_t* vals, long long nnz, int M, int N, int K, float* ysp, unsigned* err,
+                            cudaStream_t stream);
 
 // The CSR term of the prefill path (see csr.cu): x is transposed into xT [K][ld] bf16, then
 // ysp[n][m] (row stride ld) is computed from it.  ld = csr_token_stride(M).  The GEMM launched
