@@ -81,6 +81,14 @@ def _L():
             "oracle_linear3_gs": ([P, I64, I64, I64, P, P, P, I64, P, P, P, I64, P, P], ctypes.c_int),
             "oracle_linear3_at_gs": ([P, I64, I64, I64, P, P, P, I64, P, P, P, I64, P, P, I64, P, P],
                                      ctypes.c_int),
+            "oracle_f32_to_e4m3": ([F], ctypes.c_uint8),
+            "oracle_e4m3_to_f32": ([ctypes.c_uint8], F),
+            "oracle_f32_to_e2m1": ([F], ctypes.c_uint8),
+            "oracle_e2m1_to_f32": ([ctypes.c_uint8], F),
+            "oracle_quantize_nvfp4_with_scales": ([P, P, I64, I64, P, P, P], ctypes.c_int),
+            "oracle_awq_quantize_nvfp4": ([P, P, F, I64, I64, P, P, P, P], ctypes.c_int),
+            "oracle_dequant_nvfp4": ([P, P, F, I64, I64, P], ctypes.c_int),
+            "oracle_linear_nvfp4": ([P, I64, I64, P, P, F, I64, P, P, P, I64, P, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(_lib, name)
@@ -322,3 +330,68 @@ def awq_search_alpha(W, act_absmean, x_bf16_bits, alphas):
     _check(_L().oracle_awq_search_alpha(_p(W), _p(a), _p(x), M, N, K, _p(al), al.size, _p(err)),
            "awq_search_alpha")
     return err
+
+
+# ---- NVFP4 weights (E2M1 codes, an E4M3 scale per 16 weights, an fp32 tensor scale) -----
+
+def f32_to_e4m3_bits(f: float) -> int:
+    return int(_L().oracle_f32_to_e4m3(ctypes.c_float(f)))
+
+
+def e4m3_bits_to_f32(b: int) -> float:
+    return float(_L().oracle_e4m3_to_f32(ctypes.c_uint8(b)))
+
+
+def f32_to_e2m1_code(f: float) -> int:
+    return int(_L().oracle_f32_to_e2m1(ctypes.c_float(f)))
+
+
+def e2m1_code_to_f32(c: int) -> float:
+    return float(_L().oracle_e2m1_to_f32(ctypes.c_uint8(c)))
+
+
+def quantize_nvfp4_with_scales(W, s):
+    """NVFP4 of W*s -> (qweight u32 [N][K/8], scales8 u8 [K/16][N], g float)."""
+    W = _c(W, np.float32)
+    s = _c(s, np.float32)
+    N, K = W.shape
+    qw = np.zeros((N, max(K // 8, 1)), np.uint32)
+    sc = np.zeros((max(K // 16, 1), N), np.uint8)
+    g = np.zeros(1, np.float32)
+    _check(_L().oracle_quantize_nvfp4_with_scales(_p(W), _p(s), N, K, _p(qw), _p(sc), _p(g)),
+           "quantize_nvfp4_with_scales")
+    return qw, sc, float(g[0])
+
+
+def awq_quantize_nvfp4(W, act_absmean, alpha: float):
+    """AWQ scaling then NVFP4 -> (qweight u32 [N][K/8], scales8 u8 [K/16][N], g float, s f32 [K])."""
+    W = _c(W, np.float32)
+    a = _c(act_absmean, np.float32)
+    N, K = W.shape
+    qw = np.zeros((N, max(K // 8, 1)), np.uint32)
+    sc = np.zeros((max(K // 16, 1), N), np.uint8)
+    g = np.zeros(1, np.float32)
+    s = np.zeros(K, np.float32)
+    _check(_L().oracle_awq_quantize_nvfp4(_p(W), _p(a), ctypes.c_float(alpha), N, K, _p(qw), _p(sc), _p(g), _p(s)),
+           "awq_quantize_nvfp4")
+    return qw, sc, float(g[0]), s
+
+
+def dequant_nvfp4(qweight, scales8, g: float, N: int, K: int) -> np.ndarray:
+    qw, sc = _c(qweight, np.uint32), _c(scales8, np.uint8)
+    out = np.zeros((N, K), np.float64)
+    _check(_L().oracle_dequant_nvfp4(_p(qw), _p(sc), ctypes.c_float(g), N, K, _p(out)), "dequant_nvfp4")
+    return out
+
+
+def linear_nvfp4(x_bf16_bits, qweight, scales8, g: float, N: int, csr=None, with_abs: bool = False):
+    """``linear`` on NVFP4 weights."""
+    x = _c(x_bf16_bits, np.uint16)
+    M, K = x.shape
+    qw, sc = _c(qweight, np.uint32), _c(scales8, np.uint8)
+    rp, ci, v, nnz = _csr_args(csr)
+    y = np.zeros((M, N), np.float64)
+    ya = np.zeros((M, N), np.float64) if with_abs else None
+    _check(_L().oracle_linear_nvfp4(_p(x), M, K, _p(qw), _p(sc), ctypes.c_float(g), N, _p(rp), _p(ci), _p(v), nnz,
+                                    _p(y), _p(ya)), "linear_nvfp4")
+    return (y, ya) if with_abs else y

@@ -23,6 +23,9 @@
  *     TinyChat's 4-bit weight packing];
  *   - a 3-bit variant: the same RTN with eight levels, 32 codes per three 32-bit words
  *     [SqueezeLLM article, sections 2.1-2.2: the dense part quantized as coarse as 3 bits];
+ *   - NVFP4 weights: FP4 E2M1 codes with an FP8 E4M3 scale per 16 weights and an fp32
+ *     scale per tensor [DeepCompressor README: FP4_E2M1 among its data types, NVFP4 rows in
+ *     its result tables; the format's layout is the published one, see its section];
  *   - the dense-and-sparse product  W x = W_dense x + W_sparse x  with an fp16 CSR
  *     W_sparse [SqueezeLLM article, sections 2.2 and 2.3; the page lost the "=" and
  *     "+" signs, read here as written above];
@@ -684,4 +687,196 @@ int oracle_split_outliers(const float* W, const float* act_absmean, float alpha,
     free(key);
     free(chosen);
     return st;
+}
+
+/* ------------------------------------------------------------------------------------
+ * NVFP4 weights [DeepCompressor README: the toolbox fake-quantizes to FP4_E2M1, and its
+ * result tables list NVFP4 models].  The pages name the format but do not define it; it is
+ * read here as the published layout:
+ *   - elements: FP4 E2M1, bit 3 the sign, bits 2..1 the exponent (bias 1), bit 0 the
+ *     mantissa: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6;
+ *   - one FP8 E4M3 scale per 16 consecutive weights along K of a row (bit 7 the sign, 4
+ *     exponent bits with bias 7, 3 mantissa bits; largest finite 448, no infinities);
+ *   - one fp32 scale per tensor.
+ * On W' = W * s (the same activation-aware scaling as the 4-bit path), with one IEEE float
+ * operation per step:
+ *   g   = amax|W'| / 2688                (2688 = 6 * 448; g = 1 when W' is all zero)
+ *   sb  = amax|block| / fp32(6 * g)
+ *   s8  = e4m3(sb): round to nearest, ties to the even mantissa, saturating at 448
+ *   S   = fp32(float(s8) * g)
+ *   q   = e2m1(fp32(w' / S)): nearest, ties to the even mantissa, saturating at 6, the sign
+ *         bit that of the quotient (also for a zero); q = 0 in a block whose S is 0
+ * Dequantization: w~ = e2m1(q) * float(s8) * g, exact in double.  Codes are packed 8 per
+ * 32-bit word with the 4-bit ORDER interleave (qweight [N][K/8]); the scales are bytes,
+ * group-major like the fp16 scales (scales8 [K/16][N]).
+ * ---------------------------------------------------------------------------------- */
+
+/* E4M3 from the format definition: normal values (1 + m/8) 2^(e-7), e = 1..15 (not
+ * e = 15 with m = 7, the NaN), subnormals m 2^-9.  Arithmetic in double is exact. */
+uint8_t oracle_f32_to_e4m3(float f) {
+    uint8_t sign = signbit(f) ? 0x80u : 0u;
+    if (isnan(f)) return (uint8_t)(sign | 0x7Fu);
+    double a = fabs((double)f);
+    if (a > 448.0) return (uint8_t)(sign | 0x7Eu); /* saturate */
+    if (a < ldexp(1.0, -6)) {                      /* subnormal range: step 2^-9 */
+        double m = rint(a * 512.0);                /* ties to even */
+        return (uint8_t)(sign | (uint8_t)m);       /* m = 8 is the smallest normal, 0x08 */
+    }
+    int ex;
+    frexp(a, &ex); /* a = fr 2^ex, fr in [0.5, 1) */
+    int e = ex - 1;
+    double m = rint((ldexp(a, -e) - 1.0) * 8.0);
+    if (m == 8.0) {
+        m = 0.0;
+        e += 1;
+    }
+    if (e > 8 || (e == 8 && m > 6.0)) return (uint8_t)(sign | 0x7Eu);
+    return (uint8_t)(sign | (uint8_t)((e + 7) << 3) | (uint8_t)m);
+}
+
+float oracle_e4m3_to_f32(uint8_t b) {
+    double s = (b & 0x80u) ? -1.0 : 1.0;
+    int e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) return (float)(s * ldexp((double)m, -9));
+    return (float)(s * ldexp(1.0 + m / 8.0, e - 7));
+}
+
+/* E2M1 magnitudes by code (bits 2..0). */
+static const double E2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+float oracle_e2m1_to_f32(uint8_t c) {
+    return (float)(((c & 8u) ? -1.0 : 1.0) * E2M1[c & 7u]);
+}
+
+/* Nearest E2M1 value, ties to the even mantissa (the code with bit 0 clear), saturating at
+ * 6; the sign bit is the argument's.  Returns 0xFF for NaN. */
+uint8_t oracle_f32_to_e2m1(float r) {
+    if (isnan(r)) return 0xFFu;
+    uint8_t sign = signbit(r) ? 8u : 0u;
+    double a = fabs((double)r);
+    int best = 0;
+    for (int c = 1; c < 8; ++c) {
+        double d = fabs(a - E2M1[c]), db = fabs(a - E2M1[best]);
+        if (d < db || (d == db && (c & 1) == 0)) best = c;
+    }
+    return (uint8_t)(sign | (uint8_t)best);
+}
+
+/* NVFP4 quantization of W' = W * s (see the section comment): qweight [N][K/8], scales8
+ * [K/16][N], *gscale = g.  K a multiple of 16, N of 8. */
+int oracle_quantize_nvfp4_with_scales(const float* W, const float* s, int64_t N, int64_t K, uint32_t* qweight,
+                                      uint8_t* scales8, float* gscale) {
+    if (!W || !s || !qweight || !scales8 || !gscale) return ORACLE_ERR_NULL;
+    if (N <= 0 || N % 8 != 0 || K <= 0 || K % 16 != 0) return ORACLE_ERR_SHAPE;
+    float amax = 0.0f;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            float w = W[n * K + k] * s[k];
+            if (!isfinite(w)) return ORACLE_ERR_VALUE;
+            if (fabsf(w) > amax) amax = fabsf(w);
+        }
+    float g = amax > 0.0f ? amax / 2688.0f : 1.0f;
+    float six_g = 6.0f * g;
+    int err = ORACLE_OK;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < K / 16; ++b) {
+            float wp[16];
+            float bmax = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                wp[i] = W[n * K + 16 * b + i] * s[16 * b + i];
+                if (fabsf(wp[i]) > bmax) bmax = fabsf(wp[i]);
+            }
+            float sb = bmax / six_g;
+            uint8_t s8 = oracle_f32_to_e4m3(sb);
+            float S = oracle_e4m3_to_f32(s8) * g;
+            uint8_t q[16];
+            for (int i = 0; i < 16; ++i) {
+                if (S == 0.0f) {
+                    q[i] = 0;
+                    continue;
+                }
+                uint8_t c = oracle_f32_to_e2m1(wp[i] / S);
+                if (c == 0xFFu) {
+#pragma omp atomic write
+                    err = ORACLE_ERR_VALUE;
+                    c = 0;
+                }
+                q[i] = c;
+            }
+            scales8[b * N + n] = s8;
+            oracle_pack8(&q[0], &qweight[n * (K / 8) + 2 * b]);
+            oracle_pack8(&q[8], &qweight[n * (K / 8) + 2 * b + 1]);
+        }
+    }
+    *gscale = g;
+    return err;
+}
+
+/* awq_quantize with NVFP4 weights: s from act_absmean and alpha, then the NVFP4 steps on W*s. */
+int oracle_awq_quantize_nvfp4(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                              uint32_t* qweight, uint8_t* scales8, float* gscale, float* s_out) {
+    if (!W || !act_absmean || !qweight || !scales8 || !gscale) return ORACLE_ERR_NULL;
+    if (N <= 0 || N % 8 != 0 || K <= 0 || K % 16 != 0) return ORACLE_ERR_SHAPE;
+    float* s = (float*)malloc(sizeof(float) * (size_t)K);
+    if (!s) return ORACLE_ERR_VALUE;
+    int st = oracle_awq_scales(act_absmean, K, alpha, s);
+    if (!st) st = oracle_quantize_nvfp4_with_scales(W, s, N, K, qweight, scales8, gscale);
+    if (!st && s_out) memcpy(s_out, s, sizeof(float) * (size_t)K);
+    free(s);
+    return st;
+}
+
+/* w~[n][k] = e2m1(q) * float(s8) * g, in double (exact). */
+int oracle_dequant_nvfp4(const uint32_t* qweight, const uint8_t* scales8, float g, int64_t N, int64_t K,
+                         double* out) {
+    if (!qweight || !scales8 || !out) return ORACLE_ERR_NULL;
+    if (N <= 0 || N % 8 != 0 || K <= 0 || K % 16 != 0) return ORACLE_ERR_SHAPE;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t codes[8];
+            oracle_unpack8(qweight[n * (K / 8) + k / 8], codes);
+            out[n * K + k] = (double)oracle_e2m1_to_f32(codes[k % 8]) *
+                             (double)oracle_e4m3_to_f32(scales8[(k / 16) * N + n]) * (double)g;
+        }
+    return ORACLE_OK;
+}
+
+/* y = x w~^T (+ x W_sparse^T) in double for all (m, n), as oracle_linear. */
+int oracle_linear_nvfp4(const uint16_t* x, int64_t M, int64_t K, const uint32_t* qweight, const uint8_t* scales8,
+                        float g, int64_t N, const int32_t* row_ptr, const int32_t* col_idx, const uint16_t* values,
+                        int64_t nnz, double* y, double* yabs) {
+    if (!x || !qweight || !scales8 || !y) return ORACLE_ERR_NULL;
+    if (M <= 0 || N <= 0 || N % 8 != 0 || K <= 0 || K % 16 != 0) return ORACLE_ERR_SHAPE;
+    int st = check_csr(row_ptr, col_idx, values, nnz, N, K);
+    if (st) return st;
+    double* w = (double*)malloc(sizeof(double) * (size_t)(N * K));
+    if (!w) return ORACLE_ERR_VALUE;
+    st = oracle_dequant_nvfp4(qweight, scales8, g, N, K, w);
+    if (st) {
+        free(w);
+        return st;
+    }
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = (double)oracle_bf16_to_f32(x[m * K + k]) * w[n * K + k];
+                acc += p;
+                aacc += fabs(p);
+            }
+            if (row_ptr)
+                for (int64_t j = row_ptr[n]; j < row_ptr[n + 1]; ++j) {
+                    double p = (double)oracle_bf16_to_f32(x[m * K + col_idx[j]]) *
+                               (double)oracle_f16_to_f32(values[j]);
+                    acc += p;
+                    aacc += fabs(p);
+                }
+            y[m * N + n] = acc;
+            if (yabs) yabs[m * N + n] = aacc;
+        }
+    free(w);
+    return ORACLE_OK;
 }
