@@ -600,12 +600,24 @@ def run_gpu(args, world, rank, local):
         del gt
         w4.check_device_status()
         tb = sum(c[3] for c in tcalls)
+        # NVFP4 weights on the same four layers (quantizer only; W is read twice, once for the
+        # tensor amax, but the rate counts it once)
+        nq_b, nq_ms = 0.0, 0.0
+        for W, act, N, K in quant:
+            ms1, gq = time_graph(torch, lambda: w4.awq_quantize_nvfp4(W, act, workloads.ALPHA), 5, 2)
+            del gq
+            nq_b += N * K * 4 + N * K // 2 + N * K // 16 + 4 + 2 * K * 4
+            nq_ms += ms1
+        w4.check_device_status()
+        tinfo_nv = {"value": nq_b / nq_ms / 1e6, "unit": "GB/s",
+                    "workload": "awq_quantize_nvfp4 on the four Llama-3-8B layers (no NVFP4 product kernel yet)"}
         tinfo = {"gemv": {"value": tb / (ms_t * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_t,
                           "frac_of_hbm": tb / (ms_t * 1e-3) / 1e9 / pk["hbm_gbs"],
                           "workload": "the decode sweep (4 Llama-3-8B shapes x M in {1, 4, 8, 16}) on 3-bit "
                                       "codes (w3a16_gemv), own weights per call"},
                  "quantize": {"value": tq_b / tq_ms / 1e6, "unit": "GB/s",
-                              "workload": "awq_quantize3 (g128) on the four Llama-3-8B layers"}}
+                              "workload": "awq_quantize3 (g128) on the four Llama-3-8B layers"},
+                 "nvfp4_quantize": tinfo_nv}
         del tcalls
 
     cinfo = None

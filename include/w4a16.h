@@ -266,6 +266,26 @@ w4a16_status w3a16_gemv(const uint16_t* x, const uint32_t* qweight3, const uint1
                         int64_t K, int64_t group_size, void* workspace, size_t workspace_bytes, int schedule,
                         void* stream);
 
+/*
+ * awq_quantize_nvfp4 -- the AWQ-scaled weights quantized to NVFP4 [DeepCompressor README:
+ *   FP4_E2M1 among the toolbox's data types, NVFP4 in its result tables; the pages do not
+ *   define the layout, which is read as the published one].  On w' = float(w * s_k):
+ *     g   = amax|W'| / 2688 (2688 = 6 * 448; 1 for an all-zero W'), written to *gscale;
+ *     per block of 16 consecutive k of a row: s8 = E4M3(amax|block| / fp32(6 g)), round to
+ *     nearest even, saturating at 448; S = fp32(float(s8) * g);
+ *     q = E2M1(fp32(w' / S)): nearest of +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}, ties to the even
+ *     code, saturating at 6, bit 3 the sign of the quotient; q = 0 where S = 0.
+ *   The dequantized weight is E2M1(q) * float(s8) * g.
+ *   qweight  [N][K/8] uint32, device: 8 codes a word, element ORDER[j] of 8 in nibble j.
+ *   scales8  [K/16][N] bytes (E4M3), device, group-major.
+ *   gscale   one fp32, device, 4-byte aligned.  s_out [K] fp32, device, required.
+ *   N a positive multiple of 8, K of 16.  Errors: NULL, SHAPE, ALIGN, VALUE (non-finite
+ *   alpha) when called; later, VALUE for a non-finite W' or s.  There is no NVFP4 product
+ *   kernel yet.
+ */
+w4a16_status awq_quantize_nvfp4(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                                uint32_t* qweight, uint8_t* scales8, float* gscale, float* s_out, void* stream);
+
 /* w4a16_gemv_folded -- the decode GEMV on the layer input BEFORE the AWQ scaling, as one call.
  * [AWQ translation, 3.2: the weights are multiplied by s and the activations divided by it.]
  *   x   [M][K] bf16 bits, device: the raw layer input.

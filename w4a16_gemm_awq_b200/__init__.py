@@ -7,6 +7,7 @@ mirror the C ABI in include/w4a16.h:
   awq_quantize_g128(W, act_absmean, alpha)      -> (qweight, scales, zeros, s)
   awq_quantize(W, act_absmean, alpha, gs)       -> the same with groups of gs along K (gs = K: per row)
   awq_quantize3(W, act_absmean, alpha, gs=128)  -> the same with 3-bit codes (qweight3 [N][3K/32])
+  awq_quantize_nvfp4(W, act_absmean, alpha)     -> (qweight, scales8, g, s): NVFP4 weights
   w3a16_gemv(x, qweight3, scales, zeros, csr)   -> y      (1 <= M <= 16, 3-bit codes)
   w4a16_linear(x, qweight, scales, zeros, csr)  -> y      (any M)
   w4a16_gemv(...)                               -> y      (1 <= M <= 16)
@@ -70,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.awq_quantize_g128.argtypes = [P, P, F, I64, I64, P, P, P, P, P]
         L.awq_quantize.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P]
         L.awq_quantize3.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P]
+        L.awq_quantize_nvfp4.argtypes = [P, P, F, I64, I64, P, P, P, P, P]
         L.w3a16_gemv.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, I64, P, ctypes.c_size_t,
                                  ctypes.c_int, P]
         L.w4a16_linear_ex.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, I64, P, ctypes.c_size_t,
@@ -192,6 +194,25 @@ def awq_quantize3(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, grou
                                _ptr(sc), _ptr(z), _ptr(s), _stream(dev))
     _check(code, "awq_quantize3")
     return qw, sc, z, s
+
+
+def awq_quantize_nvfp4(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, out=None):
+    """AWQ scaling then NVFP4 -> (qweight int32 [N][K/8] (E2M1 codes), scales8 uint8 [K/16][N]
+    (E4M3), g fp32 [1] (tensor scale), s fp32 [K])."""
+    _need(W, torch.float32, 2, "W")
+    _need(act_absmean, torch.float32, 1, "act_absmean")
+    N, K = W.shape
+    dev = W.device
+    if out is None:
+        out = (torch.empty(N, max(K // 8, 1), dtype=torch.int32, device=dev),
+               torch.empty(max(K // 16, 1), N, dtype=torch.uint8, device=dev),
+               torch.empty(1, dtype=torch.float32, device=dev),
+               torch.empty(K, dtype=torch.float32, device=dev))
+    qw, sc, g, s = out
+    code = lib().awq_quantize_nvfp4(_ptr(W), _ptr(act_absmean), ctypes.c_float(alpha), N, K, _ptr(qw), _ptr(sc),
+                                    _ptr(g), _ptr(s), _stream(dev))
+    _check(code, "awq_quantize_nvfp4")
+    return qw, sc, g, s
 
 
 def awq_quantize_g128(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, out=None):

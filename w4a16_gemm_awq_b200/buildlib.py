@@ -13,7 +13,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libw4a16.so")
-SOURCES = ["api.cu", "quantize.cu", "gemv.cu", "csr.cu", "gemm_tc.cu", "outliers.cu", "search.cu", "selftest.cu"]
+SOURCES = ["api.cu", "quantize.cu", "nvfp4.cu", "gemv.cu", "csr.cu", "gemm_tc.cu", "outliers.cu", "search.cu",
+           "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

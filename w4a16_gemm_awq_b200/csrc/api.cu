@@ -430,6 +430,21 @@ w4a16_status awq_quantize3(const float* W, const float* act_absmean, float alpha
                                          zeros, s_out, d->num_sms, d->status, static_cast<cudaStream_t>(stream), 3));
 }
 
+w4a16_status awq_quantize_nvfp4(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
+                                uint32_t* qweight, uint8_t* scales8, float* gscale, float* s_out, void* stream) {
+    if (!W || !act_absmean || !qweight || !scales8 || !gscale || !s_out) return W4A16_ERR_NULL;
+    if (N < 8 || N % 8 != 0 || N > kMaxN || K < 16 || K % 16 != 0 || K > kMaxK) return W4A16_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(act_absmean, 16) || !aligned(qweight, 16) || !aligned(gscale, 4) ||
+        !aligned(s_out, 16))
+        return W4A16_ERR_ALIGN;
+    if (!std::isfinite(alpha)) return W4A16_ERR_VALUE;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    return from_cuda(launch_awq_quantize_nvfp4(W, act_absmean, alpha, (int)N, (int)K, qweight, scales8, gscale, s_out,
+                                               d->num_sms, d->status, static_cast<cudaStream_t>(stream)));
+}
+
 w4a16_status w3a16_gemv(const uint16_t* x, const uint32_t* qweight3, const uint16_t* scales, const uint32_t* zeros,
                         const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t group_size,
                         void* workspace, size_t workspace_bytes, int schedule, void* stream) {

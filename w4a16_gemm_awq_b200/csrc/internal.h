@@ -22,6 +22,15 @@ cudaError_t launch_awq_quantize(const float* W, const float* act, float alpha, i
                                 uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* s_out, int num_sms,
                                 unsigned* err, cudaStream_t stream, int bits = 4);
 
+// s_k = max(float(pow(a_k, alpha)), 1e-4) into s_out (quantize.cu).
+cudaError_t launch_awq_scale(const float* act, float alpha, int K, float* s_out, unsigned* err, cudaStream_t stream);
+
+// NVFP4 weights (see nvfp4.cu): qweight [N][K/8] E2M1 codes, scales8 [K/16][N] E4M3, *gscale
+// the fp32 tensor scale, s_out [K] the channel scales.  N % 8 == 0, K % 16 == 0.
+cudaError_t launch_awq_quantize_nvfp4(const float* W, const float* act, float alpha, int N, int K, uint32_t* qweight,
+                                      uint8_t* scales8, float* gscale, float* s_out, int num_sms, unsigned* err,
+                                      cudaStream_t stream);
+
 // Tensor map the GEMV needs: qweight uint32 [N][K/8] seen as 3-D (16 words of a group,
 // N rows, K/128 groups; strides K/2 and 64 bytes), box 16 x 128 x 4, no swizzle.  One copy
 // brings 4 groups of 128 rows and lays them out group by group: [4][128 rows][64 bytes].

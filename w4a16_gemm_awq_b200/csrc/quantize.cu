@@ -373,6 +373,11 @@ awq_quantize_large_kernel(const float* __restrict__ W, const float* __restrict__
     }
 }
 
+cudaError_t launch_awq_scale(const float* act, float alpha, int K, float* s_out, unsigned* err, cudaStream_t stream) {
+    awq_scale_kernel<<<(K + 255) / 256, 256, 0, stream>>>(act, alpha, K, s_out, err);
+    return cudaGetLastError();
+}
+
 bool quantize_group_size_ok(int K, int gs) {
     if (gs == 128 || gs == 256 || gs == 512 || gs == 1024) return K % 1024 == 0;
     return gs > 1024 && gs % 1024 == 0 && gs <= kQuantMaxLargeGroup && K % gs == 0;
