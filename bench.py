@@ -610,14 +610,38 @@ def run_gpu(args, world, rank, local):
             nq_ms += ms1
         w4.check_device_status()
         tinfo_nv = {"value": nq_b / nq_ms / 1e6, "unit": "GB/s",
-                    "workload": "awq_quantize_nvfp4 on the four Llama-3-8B layers (no NVFP4 product kernel yet)"}
+                    "workload": "awq_quantize_nvfp4 on the four Llama-3-8B layers"}
+        # the decode sweep on NVFP4 weights (own weights per call)
+        ncalls = []
+        for W, act, N, K in quant:
+            qn, sn, gn, _ = w4.awq_quantize_nvfp4(W, act, workloads.ALPHA)
+            for j, M in enumerate(GEMV_MS):
+                packed = (qn, sn, gn) if j == 0 else (qn.clone(), sn.clone(), gn.clone())
+                x = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+                ncalls.append((x, packed, torch.empty(M, N, dtype=torch.bfloat16, device="cuda"),
+                               N * K // 2 + N * K // 16 + 4 + 2 * M * K + 2 * M * N))
+        w4.check_device_status()
+
+        def nstep():
+            for x, (qn, sn, gn), y, _ in ncalls:
+                w4.w4a16_gemv_nvfp4(x, qn, sn, gn, out=y)
+
+        ms_n, gnv = time_graph(torch, nstep, 200, 5)
+        del gnv
+        w4.check_device_status()
+        nb = sum(c[3] for c in ncalls)
+        tinfo_nvg = {"value": nb / (ms_n * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_n,
+                     "frac_of_hbm": nb / (ms_n * 1e-3) / 1e9 / pk["hbm_gbs"],
+                     "workload": "the decode sweep (4 Llama-3-8B shapes x M in {1, 4, 8, 16}) on NVFP4 weights "
+                                 "(w4a16_gemv_nvfp4), own weights per call"}
+        del ncalls
         tinfo = {"gemv": {"value": tb / (ms_t * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_t,
                           "frac_of_hbm": tb / (ms_t * 1e-3) / 1e9 / pk["hbm_gbs"],
                           "workload": "the decode sweep (4 Llama-3-8B shapes x M in {1, 4, 8, 16}) on 3-bit "
                                       "codes (w3a16_gemv), own weights per call"},
                  "quantize": {"value": tq_b / tq_ms / 1e6, "unit": "GB/s",
                               "workload": "awq_quantize3 (g128) on the four Llama-3-8B layers"},
-                 "nvfp4_quantize": tinfo_nv}
+                 "nvfp4_quantize": tinfo_nv, "nvfp4_gemv": tinfo_nvg}
         del tcalls
 
     cinfo = None

@@ -280,11 +280,23 @@ w4a16_status w3a16_gemv(const uint16_t* x, const uint32_t* qweight3, const uint1
  *   scales8  [K/16][N] bytes (E4M3), device, group-major.
  *   gscale   one fp32, device, 4-byte aligned.  s_out [K] fp32, device, required.
  *   N a positive multiple of 8, K of 16.  Errors: NULL, SHAPE, ALIGN, VALUE (non-finite
- *   alpha) when called; later, VALUE for a non-finite W' or s.  There is no NVFP4 product
- *   kernel yet.
+ *   alpha) when called; later, VALUE for a non-finite W' or s.  w4a16_gemv_nvfp4 is the
+ *   decode product on these weights.
  */
 w4a16_status awq_quantize_nvfp4(const float* W, const float* act_absmean, float alpha, int64_t N, int64_t K,
                                 uint32_t* qweight, uint8_t* scales8, float* gscale, float* s_out, void* stream);
+
+/*
+ * w4a16_gemv_nvfp4 -- the decode product on NVFP4 weights as awq_quantize_nvfp4 writes them:
+ *   y = bf16_rne( g * sum_b (s8_b / 2) * sum_{k in block b} (2 e2m1(q_k)) x'_k ), fp32 sums.
+ *   The doubled codes are exact bf16 integers fed to mma.sync m16n8k16 (16 k = one scale
+ *   block); each MMA's result is scaled by its block's E4M3 scale in fp32.  No CSR term, no
+ *   workspace.  1 <= M <= 16; N a positive multiple of 16; K of 16.  x [M][K] bf16 bits and
+ *   qweight 16-byte aligned; gscale the device fp32 tensor scale.
+ *   Errors: NULL, SHAPE, ALIGN when called.
+ */
+w4a16_status w4a16_gemv_nvfp4(const uint16_t* x, const uint32_t* qweight, const uint8_t* scales8,
+                              const float* gscale, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
 
 /* w4a16_gemv_folded -- the decode GEMV on the layer input BEFORE the AWQ scaling, as one call.
  * [AWQ translation, 3.2: the weights are multiplied by s and the activations divided by it.]

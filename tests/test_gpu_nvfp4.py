@@ -59,3 +59,47 @@ def test_nvfp4_reports_non_finite_and_bad_shapes():
     with pytest.raises(w4.W4A16Error) as e:
         w4.awq_quantize_nvfp4(torch.zeros(16, 40, device="cuda"), torch.ones(40, device="cuda"), 0.5)
     assert e.value.code == w4.ERR_SHAPE
+
+
+@pytest.mark.parametrize("M", [1, 5, 8, 9, 16])
+@pytest.mark.parametrize("N,K", [(256, 2048), (48, 1040)])
+def test_nvfp4_gemv_full_output(orc, N, K, M):
+    """The decode product on GPU-quantized weights (checked bit for bit against the oracle's)
+    against the oracle's double-precision product, within the GEMV's output bound: the
+    weights are exact, only fp32 sums round (16-term MMA blocks, then K/16 block sums)."""
+    from parity import check_close, dev_bf16, host_bf16_as_f64
+    L = workloads.make_layer(3 * N + K + M, K=K, N=N)
+    (qw, sc, g, _), (gqw, gsc, gg, _) = _both(orc, L.W, L.act_absmean)
+    assert np.array_equal(host_bits(gqw, np.uint32), qw) and np.array_equal(gsc.cpu().numpy(), sc)
+    x = workloads.make_activations(3 * N + K + M, M, L.mult)
+    y = w4.w4a16_gemv_nvfp4(dev_bf16(x), gqw, gsc, gg)
+    w4.check_device_status()
+    ref, ref_abs = orc.linear_nvfp4(x, qw, sc, g, N, with_abs=True)
+    check_close(host_bf16_as_f64(y), ref, ref_abs, 0.0, K // 16 + 64, f"nvfp4 gemv M={M}")
+    y2 = w4.w4a16_gemv_nvfp4(dev_bf16(x), gqw, gsc, gg)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+def test_nvfp4_gemv_full_shape(orc):
+    """4096 x 4096 at M = 16, every output."""
+    from parity import check_close, dev_bf16, host_bf16_as_f64
+    K, N, M = 4096, 4096, 16
+    L = workloads.make_layer(808, K=K, N=N)
+    (qw, sc, g, _), (gqw, gsc, gg, _) = _both(orc, L.W, L.act_absmean)
+    x = workloads.make_activations(808, M, L.mult)
+    y = w4.w4a16_gemv_nvfp4(dev_bf16(x), gqw, gsc, gg)
+    w4.check_device_status()
+    ref, ref_abs = orc.linear_nvfp4(x, qw, sc, g, N, with_abs=True)
+    check_close(host_bf16_as_f64(y), ref, ref_abs, 0.0, K // 16 + 64, "nvfp4 gemv 4096x4096")
+
+
+def test_nvfp4_gemv_shape_checks():
+    x = torch.zeros(17, 256, dtype=torch.bfloat16, device="cuda")
+    qw = torch.zeros(32, 32, dtype=torch.int32, device="cuda")
+    sc = torch.zeros(16, 32, dtype=torch.uint8, device="cuda")
+    g = torch.ones(1, device="cuda")
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.w4a16_gemv_nvfp4(x, qw, sc, g)
+    assert e.value.code == w4.ERR_SHAPE
+    with pytest.raises(ValueError):
+        w4.w4a16_gemv_nvfp4(x[:4], qw[:, :16], sc, g)

@@ -8,6 +8,7 @@ mirror the C ABI in include/w4a16.h:
   awq_quantize(W, act_absmean, alpha, gs)       -> the same with groups of gs along K (gs = K: per row)
   awq_quantize3(W, act_absmean, alpha, gs=128)  -> the same with 3-bit codes (qweight3 [N][3K/32])
   awq_quantize_nvfp4(W, act_absmean, alpha)     -> (qweight, scales8, g, s): NVFP4 weights
+  w4a16_gemv_nvfp4(x, qweight, scales8, g)      -> y      (1 <= M <= 16, NVFP4 weights)
   w3a16_gemv(x, qweight3, scales, zeros, csr)   -> y      (1 <= M <= 16, 3-bit codes)
   w4a16_linear(x, qweight, scales, zeros, csr)  -> y      (any M)
   w4a16_gemv(...)                               -> y      (1 <= M <= 16)
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
         L.awq_quantize.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P]
         L.awq_quantize3.argtypes = [P, P, F, I64, I64, I64, P, P, P, P, P]
         L.awq_quantize_nvfp4.argtypes = [P, P, F, I64, I64, P, P, P, P, P]
+        L.w4a16_gemv_nvfp4.argtypes = [P, P, P, P, P, I64, I64, I64, P]
         L.w3a16_gemv.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, I64, P, ctypes.c_size_t,
                                  ctypes.c_int, P]
         L.w4a16_linear_ex.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, I64, P, ctypes.c_size_t,
@@ -213,6 +215,24 @@ def awq_quantize_nvfp4(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float,
                                     _ptr(g), _ptr(s), _stream(dev))
     _check(code, "awq_quantize_nvfp4")
     return qw, sc, g, s
+
+
+def w4a16_gemv_nvfp4(x, qweight, scales8, gscale, out=None):
+    """Decode GEMV (M <= 16) on NVFP4 weights from awq_quantize_nvfp4 -> y bf16 [M][N]."""
+    _need(x, torch.bfloat16, 2, "x")
+    _need(qweight, torch.int32, 2, "qweight")
+    M, K = x.shape
+    N = qweight.shape[0]
+    if qweight.shape[1] * 8 != K or tuple(scales8.shape) != (K // 16, N) or scales8.dtype != torch.uint8:
+        raise ValueError(f"NVFP4 operands do not match x [{M}][{K}]: qweight {tuple(qweight.shape)}, "
+                         f"scales8 {tuple(scales8.shape)} {scales8.dtype}")
+    if gscale.numel() != 1 or gscale.dtype != torch.float32 or gscale.device != x.device:
+        raise ValueError("gscale: one fp32 value on the device of x")
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    code = lib().w4a16_gemv_nvfp4(_ptr(x), _ptr(qweight), _ptr(scales8), _ptr(gscale), _ptr(y), M, N, K,
+                                  _stream(x.device))
+    _check(code, "w4a16_gemv_nvfp4")
+    return y
 
 
 def awq_quantize_g128(W: torch.Tensor, act_absmean: torch.Tensor, alpha: float, out=None):

@@ -445,6 +445,19 @@ w4a16_status awq_quantize_nvfp4(const float* W, const float* act_absmean, float 
                                                d->num_sms, d->status, static_cast<cudaStream_t>(stream)));
 }
 
+w4a16_status w4a16_gemv_nvfp4(const uint16_t* x, const uint32_t* qweight, const uint8_t* scales8,
+                              const float* gscale, uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+    if (!x || !qweight || !scales8 || !gscale || !y) return W4A16_ERR_NULL;
+    if (M < 1 || M > 16 || N < 16 || N % 16 != 0 || N > kMaxN || K < 16 || K % 16 != 0 || K > kMaxK)
+        return W4A16_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(gscale, 4) || !aligned(y, 2)) return W4A16_ERR_ALIGN;
+    DeviceInfo* d = nullptr;
+    w4a16_status st = device_info(&d);
+    if (st != W4A16_OK) return st;
+    return from_cuda(launch_gemv_nvfp4(x, qweight, scales8, gscale, y, (int)M, (int)N, (int)K,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 w4a16_status w3a16_gemv(const uint16_t* x, const uint32_t* qweight3, const uint16_t* scales, const uint32_t* zeros,
                         const w4a16_csr* outliers, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t group_size,
                         void* workspace, size_t workspace_bytes, int schedule, void* stream) {

@@ -31,6 +31,10 @@ cudaError_t launch_awq_quantize_nvfp4(const float* W, const float* act, float al
                                       uint8_t* scales8, float* gscale, float* s_out, int num_sms, unsigned* err,
                                       cudaStream_t stream);
 
+// Decode GEMV on NVFP4 weights (see nvfp4.cu): 1 <= M <= 16, N % 16 == 0, K % 16 == 0.
+cudaError_t launch_gemv_nvfp4(const uint16_t* x, const uint32_t* qweight, const uint8_t* scales8, const float* gscale,
+                              uint16_t* y, int M, int N, int K, cudaStream_t stream);
+
 // Tensor map the GEMV needs: qweight uint32 [N][K/8] seen as 3-D (16 words of a group,
 // N rows, K/128 groups; strides K/2 and 64 bytes), box 16 x 128 x 4, no swizzle.  One copy
 // brings 4 groups of 128 rows and lays them out group by group: [4][128 rows][64 bytes].

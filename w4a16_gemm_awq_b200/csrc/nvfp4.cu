@@ -13,7 +13,7 @@
 // Codes are packed 8 per word with the 4-bit path's interleave (element ORDER[j] in nibble
 // j, ORDER = {0,2,4,6,1,3,5,7}), qweight [N][K/8]; scales8 [K/16][N] bytes, group-major.
 //
-// Three passes: the s kernel (launch_awq_scale, quantize.cu), a grid-wide amax of |W'|
+// Quantizer.  Three passes: the s kernel (launch_awq_scale, quantize.cu), a grid-wide amax of |W'|
 // (atomicMax on the bits of a non-negative float, into the tensor-scale slot), then one
 // thread per 16-weight block; a last one-thread kernel turns the amax into g.  The E4M3
 // conversions are CUDA's (cuda_fp8.h, round to nearest even with saturation); the E2M1
@@ -130,7 +130,123 @@ __global__ void __launch_bounds__(kNvThreads) nvfp4_quantize_kernel(const float*
 
 __global__ void nvfp4_gscale_kernel(float* gscale) { *gscale = tensor_scale(*reinterpret_cast<unsigned*>(gscale)); }
 
+// ---------------------------------------------------------------------------------------
+// Decode GEMV on NVFP4 weights (1 <= M <= 16):
+//   y[m][n] = bf16( g * sum_b (s8[b][n] / 2) * sum_{k in block b} (2 e2m1(q[n][k])) x[m][k] )
+// Twice an E2M1 value is one of the integers 0, 1, 2, 3, 4, 6, 8, 12, exact in bf16, so the
+// codes enter mma.sync m16n8k16 (rows: 16 channels, columns: 8 tokens, depth: 16 k = one
+// scale block) as exact bf16 values; each MMA's fp32 result is scaled by its block's E4M3
+// scale / 2 and accumulated, and the tensor scale multiplies the sum once.  A CTA of 8 warps
+// (three per SM) takes 16 rows; warp w takes an eighth of the blocks along K, issuing the
+// loads of four blocks at a time, and the warps' sums are added in warp order through shared memory.
+// Weights and x are read straight from global memory (a 32-byte sector of codes serves four
+// consecutive blocks through L1).
+
+// bf16 pair (2 e2m1(c_lo), 2 e2m1(c_hi)) of the nibble pair (c, c + 4) of a word: byte
+// lookups of the low and high bytes of the bf16 values, then the sign bits.
+__device__ __forceinline__ uint32_t e2m1x2_to_bf16x2(uint32_t word, int c) {
+    const uint32_t t = word >> (4 * c);
+    const uint32_t sel = (t & 0x7u) | ((t >> 12) & 0x70u);   // code of the low half, of the high half
+    const uint32_t lo = __byte_perm(0x40008000u, 0x4000C080u, sel);  // low bytes of bf16(0,1,2,3,4,6,8,12)
+    const uint32_t hi = __byte_perm(0x40403F00u, 0x41414040u, sel);  // high bytes
+    return __byte_perm(lo, hi, 0x5140u) | ((t & 0x00080008u) << 12);
+}
+
+constexpr int kNvGemvWarps = 8;   // warps per CTA, each a share of the blocks along K
+constexpr int kNvGemvBatch = 4;   // blocks whose loads are issued together
+
+template <int NT>
+__global__ void __launch_bounds__(32 * kNvGemvWarps, 3) nvfp4_gemv_kernel(const uint16_t* __restrict__ x,
+                                                                      const uint32_t* __restrict__ qweight,
+                                                                      const uint8_t* __restrict__ scales8,
+                                                                      const float* __restrict__ gscale,
+                                                                      uint16_t* __restrict__ y, int M, int N, int K) {
+    __shared__ float red[kNvGemvWarps][32][NT * 4];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int n0 = blockIdx.x * 16;
+    const int KB = K / 16, per = (KB + kNvGemvWarps - 1) / kNvGemvWarps;
+    const int b0 = min(KB, warp * per), b1 = min(KB, b0 + per);
+    const uint2* w0 = reinterpret_cast<const uint2*>(qweight + (size_t)(n0 + g) * (K / 8));
+    const uint2* w1 = reinterpret_cast<const uint2*>(qweight + (size_t)(n0 + g + 8) * (K / 8));
+    float acc[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[j][e] = 0.0f;
+    for (int bb = b0; bb < b1; bb += kNvGemvBatch) {
+        // the batch's loads first (blocks past b1 load nothing and add nothing)
+        uint2 q0[kNvGemvBatch], q1[kNvGemvBatch];
+        uint8_t s0[kNvGemvBatch], s1[kNvGemvBatch];
+        uint32_t xb[kNvGemvBatch][NT][2];
+#pragma unroll
+        for (int u = 0; u < kNvGemvBatch; ++u) {
+            const int b = bb + u;
+            const bool live = b < b1;
+            q0[u] = live ? __ldg(w0 + b) : make_uint2(0u, 0u);
+            q1[u] = live ? __ldg(w1 + b) : make_uint2(0u, 0u);
+            s0[u] = live ? __ldg(scales8 + (size_t)b * N + n0 + g) : (uint8_t)0;
+            s1[u] = live ? __ldg(scales8 + (size_t)b * N + n0 + g + 8) : (uint8_t)0;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int tok = 8 * j + g;
+                xb[u][j][0] = 0u;
+                xb[u][j][1] = 0u;
+                if (live && tok < M) {
+                    const uint32_t* xr = reinterpret_cast<const uint32_t*>(x + (size_t)tok * K + 16 * b + 2 * c);
+                    xb[u][j][0] = __ldg(xr);
+                    xb[u][j][1] = __ldg(xr + 4);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kNvGemvBatch; ++u) {
+            if (bb + u >= b1) break;
+            const uint32_t A[4] = {e2m1x2_to_bf16x2(q0[u].x, c), e2m1x2_to_bf16x2(q1[u].x, c),
+                                   e2m1x2_to_bf16x2(q0[u].y, c), e2m1x2_to_bf16x2(q1[u].y, c)};
+            const float sa = 0.5f * e4m3_to_float(s0[u]);
+            const float sb = 0.5f * e4m3_to_float(s1[u]);
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                float d[4];
+                mma_16816_bf16_zero(d, A, xb[u][j]);
+                acc[j][0] = fmaf(sa, d[0], acc[j][0]);
+                acc[j][1] = fmaf(sa, d[1], acc[j][1]);
+                acc[j][2] = fmaf(sb, d[2], acc[j][2]);
+                acc[j][3] = fmaf(sb, d[3], acc[j][3]);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) red[warp][lane][4 * j + e] = acc[j][e];
+    __syncthreads();
+    if (warp != 0) return;
+    const float gs = *gscale;
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float v = red[0][lane][4 * j + e];
+#pragma unroll
+            for (int w = 1; w < kNvGemvWarps; ++w) v += red[w][lane][4 * j + e];
+            const int tok = 8 * j + 2 * c + (e & 1), n = n0 + g + 8 * (e >> 1);
+            if (tok < M) y[(size_t)tok * N + n] = float_to_bf16_bits(__fmul_rn(gs, v));
+        }
+}
+
 }  // namespace
+
+cudaError_t launch_gemv_nvfp4(const uint16_t* x, const uint32_t* qweight, const uint8_t* scales8, const float* gscale,
+                              uint16_t* y, int M, int N, int K, cudaStream_t stream) {
+    if (M < 1 || M > 16 || N % 16 != 0 || K % 16 != 0) return cudaErrorInvalidValue;
+    if (M <= 8)
+        nvfp4_gemv_kernel<1><<<N / 16, 32 * kNvGemvWarps, 0, stream>>>(x, qweight, scales8, gscale, y, M, N, K);
+    else
+        nvfp4_gemv_kernel<2><<<N / 16, 32 * kNvGemvWarps, 0, stream>>>(x, qweight, scales8, gscale, y, M, N, K);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_awq_quantize_nvfp4(const float* W, const float* act, float alpha, int N, int K, uint32_t* qweight,
                                       uint8_t* scales8, float* gscale, float* s_out, int num_sms, unsigned* err,
