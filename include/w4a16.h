@@ -217,6 +217,14 @@ w4a16_status w4a16_gemv_ex(const uint16_t* x, const uint32_t* qweight, const uin
                            int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                            int schedule, void* stream);
 
+/* w4a16_gemm_plan -- the launch that the prefill GEMM would make on a device with num_sms
+ * SMs (host arithmetic only, no device needed): the token tile (32, 64, 128 or 256), the CTAs
+ * per output tile along K (splits, 1 = no split-K), the 128-k slices each of them takes, and
+ * the bytes of fp32 partial tiles split-K needs in the workspace.  Errors: SHAPE for sizes
+ * the GEMM does not take, VALUE for num_sms outside 1..4096. */
+w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int num_sms, int* token_tile, int* splits,
+                             int* slices_per_split, size_t* partial_bytes);
+
 /* w4a16_gemv_plan -- the launch that w4a16_gemv_ex(schedule) would make on the current
  * device, without launching: *resolved = STREAM_K or CLUSTER, *cluster_size = CTAs per
  * cluster (0 for STREAM_K), *ctas = CTAs of the grid.  Any output pointer may be NULL.

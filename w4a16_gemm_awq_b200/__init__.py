@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
         L.w4a16_gemv_noalloc.argtypes = [P, P, P, P, ctypes.POINTER(Csr), P, I64, I64, I64, P]
         PI = ctypes.POINTER(ctypes.c_int)
         L.w4a16_gemv_plan.argtypes = [I64, I64, I64, ctypes.c_int, PI, PI, PI]
+        L.w4a16_gemm_plan.argtypes = [I64, I64, I64, ctypes.c_int, PI, PI, PI, ctypes.POINTER(ctypes.c_size_t)]
         L.w4a16_workspace_bytes.argtypes = [I64, I64, I64]
         L.w4a16_workspace_bytes.restype = ctypes.c_size_t
         L.w4a16_workspace_bytes_ex.argtypes = [I64, I64, I64, ctypes.c_int]
@@ -352,6 +353,15 @@ def gemv_plan(M: int, N: int, K: int, schedule: int = GEMV_AUTO):
     return r.value, c.value, n.value
 
 
+def gemm_plan(M: int, N: int, K: int, num_sms: int):
+    """(token tile, splits along K, 128-k slices per split, partial-tile bytes) of the prefill GEMM on a
+    device with num_sms SMs (host arithmetic; needs no GPU)."""
+    bn, sp, sl, pb = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0), ctypes.c_size_t(0)
+    _check(lib().w4a16_gemm_plan(M, N, K, int(num_sms), ctypes.byref(bn), ctypes.byref(sp), ctypes.byref(sl),
+                                 ctypes.byref(pb)), "w4a16_gemm_plan")
+    return bn.value, sp.value, sl.value, pb.value
+
+
 def w4a16_gemm(x, qweight, scales, zeros, csr=None, out=None, workspace=None):
     return _linear("w4a16_gemm", x, qweight, scales, zeros, csr, out, workspace)
 
@@ -475,6 +485,7 @@ def w4a16_workspace_bytes_ex(M: int, N: int, K: int, with_csr: int) -> int:
 
 
 w4a16_gemv_plan = gemv_plan
+w4a16_gemm_plan = gemm_plan
 w4a16_check_device_status = check_device_status
 w4a16_selftest_timeout = selftest_timeout
 w4a16_selftest_quotient = selftest_quotient

@@ -499,6 +499,19 @@ w4a16_status w4a16_gemv_folded(const uint16_t* x, const float* s, const uint32_t
     return run_gemv(a, static_cast<cudaStream_t>(stream), schedule);
 }
 
+w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int num_sms, int* token_tile, int* splits,
+                             int* slices_per_split, size_t* partial_bytes) {
+    if (M < 1 || M > kMaxM || N < 128 || N % 128 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK)
+        return W4A16_ERR_SHAPE;
+    if (num_sms < 1 || num_sms > 4096) return W4A16_ERR_VALUE;
+    const GemmPlan g = gemm_plan(M, N, K, num_sms);
+    if (token_tile) *token_tile = g.bn;
+    if (splits) *splits = g.splits;
+    if (slices_per_split) *slices_per_split = g.slices;
+    if (partial_bytes) *partial_bytes = g.partial_bytes;
+    return W4A16_OK;
+}
+
 w4a16_status w4a16_gemv_plan(int64_t M, int64_t N, int64_t K, int schedule, int* resolved, int* cluster_size,
                              int* ctas) {
     if (M < 1 || M > 16 || N < 128 || N % 128 != 0 || N > kMaxN || K < 1024 || K % 1024 != 0 || K > kMaxK)
