@@ -215,3 +215,56 @@ def test_linear_shape_checks_before_any_launch():
     for fn in (w4.w4a16_gemv_noalloc, w4.w4a16_gemv):
         with pytest.raises(ValueError):
             fn(x, qw[:, :-1], sc, z)
+
+
+def test_three_bit_validation(L):
+    def q(gs=128, N=128, K=4096, W=FAKE, alpha=0.5):
+        return L.awq_quantize3(ctypes.c_void_p(W), ctypes.c_void_p(FAKE), ctypes.c_float(alpha), N, K, gs,
+                               ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), None, None)
+    assert q(W=0) == w4.ERR_NULL
+    for gs in (64, 192, 2048, 4096):          # the 3-bit quantizer takes 128 .. 1024
+        assert q(gs) == w4.ERR_SHAPE, gs
+    assert q(K=1000) == w4.ERR_SHAPE
+    assert q(alpha=float("nan")) == w4.ERR_VALUE
+
+    def g3(M=1, gs=128, schedule=0, x=FAKE, K=4096):
+        return L.w3a16_gemv(ctypes.c_void_p(x), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE),
+                            None, ctypes.c_void_p(FAKE), M, 128, K, gs, ctypes.c_void_p(FAKE), 1 << 30, schedule,
+                            None)
+    assert g3(x=0) == w4.ERR_NULL
+    assert g3(M=17) == w4.ERR_SHAPE           # decode only: no 3-bit prefill GEMM
+    assert g3(gs=192) == w4.ERR_SHAPE
+    assert g3(schedule=7) == w4.ERR_VALUE
+
+
+def test_nvfp4_validation(L):
+    def q(W=FAKE, N=128, K=4096, g=FAKE, s=FAKE, alpha=0.5):
+        return L.awq_quantize_nvfp4(ctypes.c_void_p(W), ctypes.c_void_p(FAKE), ctypes.c_float(alpha), N, K,
+                                    ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(g),
+                                    ctypes.c_void_p(s) if s else None, None)
+    assert q(W=0) == w4.ERR_NULL
+    assert q(s=0) == w4.ERR_NULL              # s_out is required: the kernels read it back
+    assert q(N=12) == w4.ERR_SHAPE
+    assert q(K=40) == w4.ERR_SHAPE
+    assert q(g=FAKE + 2) == w4.ERR_ALIGN
+    assert q(alpha=float("inf")) == w4.ERR_VALUE
+
+    def gv(M=1, N=128, K=4096, x=FAKE, g=FAKE):
+        return L.w4a16_gemv_nvfp4(ctypes.c_void_p(x), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE),
+                                  ctypes.c_void_p(g), ctypes.c_void_p(FAKE), M, N, K, None)
+    assert gv(x=0) == w4.ERR_NULL
+    assert gv(M=17) == w4.ERR_SHAPE
+    assert gv(N=24) == w4.ERR_SHAPE
+    assert gv(K=24) == w4.ERR_SHAPE
+    assert gv(x=FAKE + 4) == w4.ERR_ALIGN
+
+
+def test_variant_wrappers_check_shapes_first():
+    import torch
+    x = torch.zeros(2, 1024, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):           # a 4-bit qweight handed to the 3-bit GEMV
+        w4.w3a16_gemv(x, torch.zeros(128, 128, dtype=torch.int32), torch.zeros(8, 128, dtype=torch.int16),
+                      torch.zeros(8, 16, dtype=torch.int32))
+    with pytest.raises(ValueError):           # CPU tensors never reach the library
+        w4.w4a16_gemv_nvfp4(x, torch.zeros(128, 128, dtype=torch.int32), torch.zeros(64, 128, dtype=torch.uint8),
+                            torch.ones(1))
